@@ -1,0 +1,78 @@
+"""Seeded synthetic inputs shared by the tests, the oracle checks and the bench.
+
+This module holds no arithmetic of the method: it only draws random tensors
+with the shapes and value distributions of the workloads (x ~ N(0, 1),
+dY ~ N(0, 1e-2) read as a variance, weights ~ N(0, 1/fan_in) as in the
+eugen_sparse README's quick start, balancing bias ~ U(-0.1, 0.1)) and rounds
+them to the compute dtype.  Each tensor has its own torch CPU generator seeded
+from (workload seed, tensor id), so a tensor does not depend on the sizes of
+the others.  It imports nothing else from the package.
+"""
+from __future__ import annotations
+
+import torch
+
+# Workloads: shapes of the pages' SwiGLU configurations (FlashFFN model table:
+# d_model 768/2048 with d_ff 2048/5504, batch 8 at 2K-32K tokens per sequence)
+# and of the eugen_sparse training setting (d_ff 4096, 64 groups, 8 active).
+WORKLOADS = {
+    0: dict(name="dense_f32_m64_d128_f352", kind="dense", dtype="f32",
+            M=64, d_model=128, d_ff=352, seed=0),
+    1: dict(name="dense_bf16_m16384_d768_f2048", kind="dense", dtype="bf16",
+            M=16384, d_model=768, d_ff=2048, seed=1),
+    2: dict(name="dense_bf16_m32768_d2048_f5504", kind="dense", dtype="bf16",
+            M=32768, d_model=2048, d_ff=5504, seed=2),
+    3: dict(name="sparse_bf16_m16384_d1024_f4096_g64_k8_spg8", kind="sparse",
+            dtype="bf16", M=16384, d_model=1024, d_ff=4096, group_size=64,
+            num_active_groups=8, samples_per_group=8, seed=3),
+    4: dict(name="infer_bf16_m262144_d2048_f5504", kind="infer", dtype="bf16",
+            M=262144, d_model=2048, d_ff=5504, seed=4),
+}
+
+_TENSOR_IDS = {"x": 1, "w_gate": 2, "w_up": 3, "w_down": 4, "dy": 5, "bias": 6}
+
+DY_STD = 0.1  # N(0, 1e-2) as a variance
+
+
+def torch_dtype(name: str) -> torch.dtype:
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+def _gen(seed: int, tensor: str) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) * 1_000_003 + _TENSOR_IDS[tensor])
+    return g
+
+
+def normal(shape, std, seed, tensor, dtype=torch.bfloat16):
+    """std * N(0, 1) drawn in fp32 and rounded (nearest-even) to ``dtype``."""
+    t = torch.randn(*shape, generator=_gen(seed, tensor), dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def dense_inputs(M, d_model, d_ff, seed, dtype=torch.bfloat16, with_dy=True):
+    """x [M, d_model], w_gate / w_up [d_ff, d_model], w_down [d_model, d_ff]
+    (nn.Linear layout), dy [M, d_model]; CPU tensors."""
+    out = {
+        "x": normal((M, d_model), 1.0, seed, "x", dtype),
+        "w_gate": normal((d_ff, d_model), d_model ** -0.5, seed, "w_gate", dtype),
+        "w_up": normal((d_ff, d_model), d_model ** -0.5, seed, "w_up", dtype),
+        "w_down": normal((d_model, d_ff), d_ff ** -0.5, seed, "w_down", dtype),
+    }
+    if with_dy:
+        out["dy"] = normal((M, d_model), DY_STD, seed, "dy", dtype)
+    return out
+
+
+def balance_bias(num_groups, seed, lo=-0.1, hi=0.1):
+    """Per-group load-balance bias ~ U(lo, hi), fp32."""
+    u = torch.rand(num_groups, generator=_gen(seed, "bias"), dtype=torch.float32)
+    return u * (hi - lo) + lo
+
+
+def workload_inputs(cfg_id: int, with_dy=True):
+    w = WORKLOADS[cfg_id]
+    return dense_inputs(w["M"], w["d_model"], w["d_ff"], w["seed"],
+                        torch_dtype(w["dtype"]), with_dy=with_dy and w["kind"] != "infer")
