@@ -1,0 +1,214 @@
+/*
+ * swiglu_ffn.h -- C ABI of the SwiGLU feed-forward library for NVIDIA B200 (sm_100a).
+ *
+ * The block is y = (SiLU(x W_gate^T) * (x W_up^T)) W_down^T with SiLU(z) = z * sigmoid(z)
+ * (flash-swiglu-mlp overview: fused gate/up projections with SiLU gating, then the down
+ * projection; training saves intermediates, inference does not), plus the group-sparse
+ * variant of the eugen_sparse README ("What it does": grouped_topk_select picks, per token,
+ * the num_active_groups groups of group_size FFN rows with the largest energy
+ * sum |SiLU(x W_gate^T)|, optionally on a fixed row subsample and with a balancing bias;
+ * sparse_swiglu_ffn computes only the selected groups, forward and backward).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller, row-major and contiguous,
+ *    16-byte aligned (SWF_ERR_ALIGNMENT otherwise).  Weights use the nn.Linear layout:
+ *    w_gate, w_up are [d_ff, d_model]; w_down is [d_model, d_ff].  Activations are
+ *    [M, d_model] with M the number of tokens.
+ *  - `dtype` (swf_dtype) is the element type of every floating tensor except the balancing
+ *    bias and the energies, which are always fp32.  bf16 runs on the tcgen05 tensor cores with
+ *    fp32 accumulation; fp32 runs in full fp32 on the CUDA cores.
+ *  - `stream` is a cudaStream_t (passed as void*).  Calls only enqueue work on it and return;
+ *    nothing allocates device memory, nothing synchronises.  Buffers that the work needs
+ *    beyond its inputs and outputs come from the caller's `workspace` of `workspace_bytes`
+ *    bytes (size it with swf_workspace_bytes; SWF_ERR_WORKSPACE if too small).
+ *  - Argument errors are detected on the host before anything is enqueued; then no work is
+ *    launched and outputs are untouched.  There is never a CPU or library fallback: a shape
+ *    outside the rules returns SWF_ERR_UNSUPPORTED.
+ *  - Weight gradients are overwritten, not accumulated.
+ *  - Every wait inside a kernel is bounded in time; a wait that runs out records
+ *    SWF_ERR_TIMEOUT in a per-device status word (read with swf_device_status) and the kernel
+ *    returns instead of hanging.
+ *
+ * Shape rules (eugen_sparse README, "Parameters and how to choose them" and "Pitfalls"):
+ *  - bf16: d_model and d_ff multiples of 16 (TMA rows must be 16-byte multiples).
+ *  - fp32: any positive d_model, d_ff.
+ *  - sparse / selection: group_size a power of two in [16, 64]; d_ff a multiple of group_size
+ *    with at least 2 groups; 1 <= num_active_groups <= d_ff / group_size; 1 <= samples_per_group
+ *    <= group_size; M * num_active_groups < 2^31.
+ */
+#ifndef SWIGLU_FFN_H
+#define SWIGLU_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum swf_status {
+  SWF_OK = 0,
+  SWF_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum */
+  SWF_ERR_UNSUPPORTED = 2,  /* shape or dtype outside the rules above */
+  SWF_ERR_ALIGNMENT = 3,    /* a pointer not 16-byte aligned */
+  SWF_ERR_WORKSPACE = 4,    /* workspace (or sparse saved buffer) smaller than required */
+  SWF_ERR_LAUNCH = 5,       /* the CUDA runtime refused a launch or a query */
+  SWF_ERR_TIMEOUT = 6       /* a bounded in-kernel wait ran out (see swf_device_status) */
+} swf_status;
+
+typedef enum swf_dtype { SWF_F32 = 0, SWF_BF16 = 1 } swf_dtype;
+
+typedef enum swf_op {
+  SWF_OP_FWD = 0,         /* swiglu_ffn_fwd */
+  SWF_OP_FWD_INFER = 1,   /* swiglu_ffn_fwd_infer */
+  SWF_OP_BWD = 2,         /* swiglu_ffn_bwd */
+  SWF_OP_SELECT = 3,      /* grouped_topk_select */
+  SWF_OP_SPARSE_FWD = 4,  /* sparse_swiglu_ffn_fwd */
+  SWF_OP_SPARSE_BWD = 5,  /* sparse_swiglu_ffn_bwd */
+  SWF_OP_BUCKETS = 6      /* swf_group_buckets */
+} swf_op;
+
+/* How an operation will run (eugen_sparse README: plan() reports how the work is split,
+ * without touching the GPU).  Filled by swf_plan. */
+typedef struct swf_plan_info {
+  int32_t path;            /* 0 = fp32 CUDA cores, 1 = bf16 tcgen05 tensor cores */
+  int32_t tile_m, tile_n, tile_k;
+  int32_t stages;          /* shared-memory pipeline depth of the GEMM kernels */
+  int32_t grid;            /* CTAs of the persistent GEMM kernels (<= number of SMs) */
+  int32_t num_kernels;     /* kernels one call launches */
+  int32_t deterministic;   /* 1 if repeated calls give bitwise-identical results */
+  int64_t gemm_tiles;      /* output tiles over all GEMMs of the call */
+  int64_t flops;           /* algorithmic FLOPs of the call */
+  size_t workspace_bytes;  /* = swf_workspace_bytes(...) */
+  size_t saved_bytes;      /* sparse forward: = swf_sparse_saved_bytes(...), else 0 */
+} swf_plan_info;
+
+/* ------------------------------------------------------------------ dense SwiGLU FFN */
+
+/* Training forward (flash-swiglu-mlp overview, "Fused train forward" storing intermediates;
+ * parameter-golf PR 1105 "Fused MLP Kernels": store the activation gradient, not the
+ * pre-activation).  Computes g = x W_gate^T, u = x W_up^T (fp32 accumulation, never written
+ * to memory), and writes
+ *   saved_h = SiLU(g) * u,  saved_a = u * SiLU'(g),  saved_b = SiLU(g)   (each [M, d_ff]),
+ *   y = saved_h W_down^T                                                   ([M, d_model]).
+ * saved_* are outputs the caller keeps for swiglu_ffn_bwd.  No workspace. */
+swf_status swiglu_ffn_fwd(const void* x, const void* w_gate, const void* w_up, const void* w_down,
+                          void* y, void* saved_h, void* saved_a, void* saved_b,
+                          int64_t M, int64_t d_model, int64_t d_ff, swf_dtype dtype, void* stream);
+
+/* Inference forward (flash-swiglu-mlp overview: "inference skips saving gate/up activations").
+ * Same y as swiglu_ffn_fwd; the product h lives only in `workspace`
+ * (swf_workspace_bytes(SWF_OP_FWD_INFER, ...) bytes). */
+swf_status swiglu_ffn_fwd_infer(const void* x, const void* w_gate, const void* w_up,
+                                const void* w_down, void* y, void* workspace,
+                                size_t workspace_bytes, int64_t M, int64_t d_model, int64_t d_ff,
+                                swf_dtype dtype, void* stream);
+
+/* Backward of the training forward (flash-swiglu-mlp: activation-gradient, weight-gradient and
+ * input-gradient steps; parameter-golf "Fused MLP Kernels": the down-projection gradient is
+ * multiplied by the stored activation-gradient factor inside the GEMM epilogue):
+ *   dH = dy W_down;  dG = dH * saved_a;  dU = dH * saved_b        (workspace, [M, 2 d_ff])
+ *   dx = dG W_gate + dU W_up;  dw_gate = dG^T x;  dw_up = dU^T x;  dw_down = dy^T saved_h.
+ * dx [M, d_model]; dw_gate, dw_up [d_ff, d_model]; dw_down [d_model, d_ff] (overwritten). */
+swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate, const void* w_up,
+                          const void* w_down, const void* saved_h, const void* saved_a,
+                          const void* saved_b, void* dx, void* dw_gate, void* dw_up,
+                          void* dw_down, void* workspace, size_t workspace_bytes, int64_t M,
+                          int64_t d_model, int64_t d_ff, swf_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------ group-sparse variant */
+
+/* Subsample index (eugen_sparse README, make_subsample_index; drawn once per layer).  HOST
+ * function, no GPU work.  Writes out[c * spg + i], c < d_ff / group_size, i < spg: the absolute
+ * gate-row ids of group c's sample, ascending, drawn by a partial Fisher-Yates shuffle of the
+ * group's offsets driven by one splitmix64 stream seeded with `seed` (groups in order). */
+swf_status swf_make_subsample_index(int64_t d_ff, int32_t group_size, int32_t samples_per_group,
+                                    uint64_t seed, int32_t* out);
+
+/* Grouped top-k selection (eugen_sparse README, grouped_topk_select; hard top-k, no gradient,
+ * deterministic).  For token t and group c (rows [c*G, (c+1)*G) of w_gate):
+ *   s[t,c] = sum_{j in S_c} |SiLU(x_t . w_gate[j])|  (+ load_balance_bias[c] when non-null)
+ * where S_c is the group's subsample subsample_idx[c*spg .. c*spg+spg) (absolute row ids, as
+ * written by swf_make_subsample_index), or all G rows when subsample_idx is NULL (then
+ * samples_per_group is ignored).  The bias is additive and affects selection only.
+ * group_idx [M, K] int32 receives each token's K best groups (ties: lower group index wins),
+ * ascending within the row.  energies, if non-null, receives s [M, d_ff/G] fp32. */
+swf_status grouped_topk_select(const void* x, const void* w_gate, const int32_t* subsample_idx,
+                               int32_t samples_per_group, const float* load_balance_bias,
+                               int32_t group_size, int32_t num_active_groups, int32_t* group_idx,
+                               float* energies, void* workspace, size_t workspace_bytes,
+                               int64_t M, int64_t d_model, int64_t d_ff, swf_dtype dtype,
+                               void* stream);
+
+/* Group-major bucketing of the (token, group) pairs (eugen_sparse README, "Pitfalls": the
+ * CSR bucketing is deterministic).  offsets [num_groups + 1] int32 and tokens [M * K] int32:
+ * tokens[offsets[c] .. offsets[c+1]) are the ids of the tokens whose group_idx row holds c, in
+ * ascending order.  group_idx rows must hold distinct in-range groups (unchecked). */
+swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t num_active_groups,
+                             int32_t num_groups, int32_t* offsets, int32_t* tokens,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Sparse forward (eugen_sparse README, sparse_swiglu_ffn):
+ *   y[t] = sum over c in group_idx[t] of (SiLU(x_t W_gate[c]^T) * x_t W_up[c]^T) W_down[:, c]^T
+ * with W_*[c] the group's G rows.  y is accumulated in fp32 (fp32 atomics, as the README
+ * describes; the summation order may vary between runs) and written in `dtype`.  `saved`
+ * (swf_sparse_saved_bytes bytes) receives what the backward needs: the bucketing and the
+ * compact per-pair h, a, b; the caller keeps it for sparse_swiglu_ffn_bwd. */
+swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, const void* w_up,
+                                 const void* w_down, const int32_t* group_idx, int32_t group_size,
+                                 int32_t num_active_groups, void* y, void* saved,
+                                 size_t saved_bytes, void* workspace, size_t workspace_bytes,
+                                 int64_t M, int64_t d_model, int64_t d_ff, swf_dtype dtype,
+                                 void* stream);
+
+/* Sparse backward: gradients to x and all three weights of L = sum(dy * y) for the forward
+ * above.  Only selected groups get weight gradients; rows (dw_gate, dw_up) and columns
+ * (dw_down) of groups no token selected are written as exact zeros (eugen_sparse README,
+ * "Hard selection").  dx accumulates in fp32 (atomics); weight gradients are deterministic. */
+swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate,
+                                 const void* w_up, const void* w_down, const int32_t* group_idx,
+                                 const void* saved, size_t saved_bytes, void* dx, void* dw_gate,
+                                 void* dw_up, void* dw_down, void* workspace,
+                                 size_t workspace_bytes, int64_t M, int64_t d_model, int64_t d_ff,
+                                 int32_t group_size, int32_t num_active_groups, swf_dtype dtype,
+                                 void* stream);
+
+/* ------------------------------------------------------------------ planning and queries */
+
+/* Workspace bytes `op` needs (0 if none).  group_size / num_active_groups are ignored by the
+ * dense ops; returns 0 for arguments that swf_supported rejects. */
+size_t swf_workspace_bytes(swf_op op, int64_t M, int64_t d_model, int64_t d_ff,
+                           int32_t group_size, int32_t num_active_groups, swf_dtype dtype);
+
+/* Bytes of the `saved` buffer of sparse_swiglu_ffn_fwd / _bwd (0 for rejected arguments). */
+size_t swf_sparse_saved_bytes(int64_t M, int64_t d_model, int64_t d_ff, int32_t group_size,
+                              int32_t num_active_groups, swf_dtype dtype);
+
+/* SWF_OK if `op` runs for these sizes, else the status the op would return (eugen_sparse
+ * README, kernel_supported).  Host only. */
+swf_status swf_supported(swf_op op, int64_t M, int64_t d_model, int64_t d_ff, int32_t group_size,
+                         int32_t num_active_groups, int32_t samples_per_group, swf_dtype dtype);
+
+/* How `op` will run (eugen_sparse README, plan): fills *out.  Host only. */
+swf_status swf_plan(swf_op op, int64_t M, int64_t d_model, int64_t d_ff, int32_t group_size,
+                    int32_t num_active_groups, int32_t samples_per_group, swf_dtype dtype,
+                    swf_plan_info* out);
+
+/* Synchronises `stream`, then reads and clears the current device's status word: SWF_OK, or
+ * SWF_ERR_TIMEOUT if a kernel's bounded wait ran out since the last read. */
+swf_status swf_device_status(void* stream);
+
+/* Failure-detection self test: launches one kernel that waits on a barrier that nothing
+ * completes, with a limit of `limit_us` microseconds (1 .. 1000000), so that the wait runs
+ * out and the kernel records SWF_ERR_TIMEOUT and returns.  Returns the launch status. */
+swf_status swf_selftest_wait_timeout(int32_t limit_us, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* swf_status_string(swf_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWIGLU_FFN_H */

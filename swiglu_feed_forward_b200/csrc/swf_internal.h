@@ -1,0 +1,54 @@
+// Host-side internals shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/swiglu_ffn.h"
+
+namespace swf {
+
+struct DevCtx {
+  int device;
+  int num_sms;
+  int* status;  // device address of the status word
+};
+
+// Current device's context (SM count, status word address); cached per device.
+swf_status get_ctx(DevCtx* out);
+
+// 2-D bf16 tensor map with 128-byte swizzle over a row-major matrix of `rows` x `cols`
+// elements whose rows are `row_elems` apart; box of box_cols x box_rows.  Out-of-range
+// elements of a box read as zero.
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                      uint64_t row_elems, uint32_t box_cols, uint32_t box_rows);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Default bound on a single in-kernel wait (ns).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+// ---- dense path (swf_dense.cu) ----
+swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const void* wd, void* y,
+                          void* h, void* a, void* b, int64_t M, int64_t d, int64_t f, bool infer,
+                          cudaStream_t st);
+swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
+                          const void* wd, const void* h, const void* a, const void* b, void* dx,
+                          void* dwg, void* dwu, void* dwd, void* dgu, int64_t M, int64_t d,
+                          int64_t f, cudaStream_t st);
+swf_status dense_fwd_f32(const float* x, const float* wg, const float* wu, const float* wd,
+                         float* y, float* h, float* a, float* b, int64_t M, int64_t d, int64_t f,
+                         bool infer, cudaStream_t st);
+swf_status dense_bwd_f32(const float* dy, const float* x, const float* wg, const float* wu,
+                         const float* wd, const float* h, const float* a, const float* b,
+                         float* dx, float* dwg, float* dwu, float* dwd, float* dgu, int64_t M,
+                         int64_t d, int64_t f, cudaStream_t st);
+
+// Tile count and launch shape of the dense bf16 GEMMs (for swf_plan).
+int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f);
+
+}  // namespace swf

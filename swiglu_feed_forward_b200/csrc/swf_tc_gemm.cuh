@@ -1,0 +1,357 @@
+// Persistent, warp-specialised tcgen05 GEMM for sm_100a with fused SwiGLU epilogues.
+//
+//   C[m, n] = sum_k A(m, k) * B(n, k)      bf16 operands, fp32 accumulation in TMEM
+//
+// One CTA per SM walks a static list of 128 x BN output tiles.  Warp 0 streams A/B tiles
+// into a ring of shared-memory stages with TMA (128-byte swizzle), warp 1 allocates TMEM and
+// one of its threads issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators,
+// warps 2..5 drain the other accumulator with tcgen05.ld, apply the epilogue in fp32
+// registers and store to global memory, so the epilogue of tile i overlaps the main loop of
+// tile i+1.  Either operand may be K-major (rows of K contiguous) or MN-major (rows of M or N
+// contiguous); the tensor-core descriptors read both layouts, so no transposes are needed.
+//
+// Epilogues (flash-swiglu-mlp overview; parameter-golf PR 1105 "Fused MLP Kernels"):
+//   kEpiStore     C -> bf16, row m < row_split to out0 else out1 (two weight-gradient halves)
+//   kEpiSwiGLU    gate|up dual tile: h = SiLU(g)*u, a = u*SiLU'(g), b = SiLU(g) -> bf16
+//   kEpiSwiGLUInf same, h only
+//   kEpiDGate     C = dH: dG = dH*a -> out0[:, n], dU = dH*b -> out0[:, d_ff + n]
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "swf_ptx.cuh"
+
+namespace swf {
+
+enum : int { kEpiStore = 0, kEpiSwiGLU = 1, kEpiSwiGLUInf = 2, kEpiDGate = 3 };
+
+constexpr int kTileM = 128;
+constexpr int kTileK = 64;  // one 128-byte swizzle row of bf16
+constexpr int kUmmaK = 16;
+constexpr int kGemmThreads = 192;
+
+struct TcGemmArgs {
+  int M;            // rows of C
+  int N;            // columns of C that exist (kEpiSwiGLU*: d_ff)
+  int num_m_blk, num_n_blk;
+  int raster;       // m-blocks per raster group
+  int kb_seg0;      // 64-wide k-blocks in K segment 0
+  int kb_total;     // k-blocks in total (segment 1 = the rest)
+  int a_koff1;      // A's K coordinate where segment 1 starts
+  // epilogue
+  void* out0;
+  void* out1;
+  int64_t ld_out;   // elements
+  int row_split;    // kEpiStore: rows >= row_split go to out1 (row - row_split)
+  const void* aux0; // kEpiSwiGLU: saved_a out; kEpiDGate: saved_a in
+  const void* aux1; // kEpiSwiGLU: saved_b out; kEpiDGate: saved_b in
+  int64_t ld_aux;
+  int d_ff;         // kEpiDGate: column offset of dU in out0
+  int* status;      // device status word
+  uint64_t wait_limit_ns;
+};
+
+template <int BN>
+struct TcSmem {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = kTileM * kTileK * 2;
+  static constexpr int kBBytes = BN * kTileK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTileBytes = kStages * kStageBytes;
+  static constexpr int kBarOffset = kTileBytes;
+  static constexpr int kBytes = kTileBytes + 256 + 1024;  // barriers + alignment slack
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int raster, int& mb,
+                                            int& nb) {
+  const int per_group = raster * num_n;
+  const int g = tile / per_group;
+  const int r = tile - g * per_group;
+  const int m0 = g * raster;
+  const int gm = min(raster, num_m - m0);
+  mb = m0 + r % gm;
+  nb = r / gm;
+}
+
+// 16-byte vector store of 8 bf16 values held as 4 packed words.
+__device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
+}
+
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, const TcGemmArgs args) {
+  using L = TcSmem<BN>;
+  constexpr int S = L::kStages;
+  constexpr uint32_t kIdesc = idesc_bf16(kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+  constexpr int kTmemCols = 2 * BN;  // two accumulators
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = args.num_m_blk * args.num_n_blk;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (B_DUAL || args.kb_seg0 < args.kb_total) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, args.num_m_blk, args.num_n_blk, args.raster, mb, nb);
+        for (int kb = 0; kb < args.kb_total; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* sA = smem + s * L::kStageBytes;
+          uint8_t* sB = sA + L::kABytes;
+          mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+          const bool seg1 = kb >= args.kb_seg0;
+          const int kk = (seg1 ? kb - args.kb_seg0 : kb) * kTileK;  // K inside the segment
+          const int ka = seg1 ? args.a_koff1 + kk : kk;
+          if (A_MN) {
+            tma_load_2d(sA, &tmA, mb * kTileM, ka, &full[s]);
+            tma_load_2d(sA + 8192, &tmA, mb * kTileM + 64, ka, &full[s]);
+          } else {
+            tma_load_2d(sA, &tmA, ka, mb * kTileM, &full[s]);
+          }
+          const CUtensorMap* mapB = seg1 ? &tmB1 : &tmB0;
+          if (B_DUAL) {
+            tma_load_2d(sB, &tmB0, kk, nb * (BN / 2), &full[s]);
+            tma_load_2d(sB + (BN / 2) * 128, &tmB1, kk, nb * (BN / 2), &full[s]);
+          } else if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sB + j * 8192, mapB, nb * BN + j * 64, kk, &full[s]);
+          } else {
+            tma_load_2d(sB, mapB, kk, nb * BN, &full[s]);
+          }
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA leaves (bounded).
+        WaitCtl quick{abort_flag, args.status, 100000000ull};
+        volatile int no_abort = 0;
+        quick.abort = &no_abort;
+        const uint32_t first = it > (uint32_t)S ? it - S : 0;
+        for (uint32_t j = first; j < it; ++j) mbar_wait(&full[j % S], (j / S) & 1u, quick);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < args.kb_total; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&full[s], ph, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * L::kStageBytes);
+          const uint32_t b0 = a0 + L::kABytes;
+#pragma unroll
+          for (int k = 0; k < kTileK / kUmmaK; ++k) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
+                                     : smem_desc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
+                                     : smem_desc_sw128(b0 + k * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          issued = true;
+        }
+        if (!ok) break;
+        if (args.kb_total > 0) umma_commit(&tfull[buf]);
+        else mbar_arrive(&tfull[buf]);
+      }
+      if (!ok && issued) {
+        umma_commit(drain);
+        WaitCtl quick{abort_flag, args.status, 100000000ull};
+        volatile int no_abort = 0;
+        quick.abort = &no_abort;
+        mbar_wait(drain, 0, quick);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 2..5
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      int mb, nb;
+      tile_coords(tile, args.num_m_blk, args.num_n_blk, args.raster, mb, nb);
+      const int buf = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const bool ready = mbar_wait(&tfull[buf], use & 1u, ctl);
+      __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
+      const bool have_acc = args.kb_total > 0;
+      const int m = mb * kTileM + row;
+      const bool row_ok = m < args.M;
+
+      if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          float g[32], u[32];
+          if (have_acc) {
+            tmem_ld32(t_acc + c, g);
+            tmem_ld32(t_acc + BN / 2 + c, u);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
+          }
+          const int n0 = nb * (BN / 2) + c;
+          if (row_ok) {
+            __nv_bfloat16* hp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
+            __nv_bfloat16* ap = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux0)) +
+                                (int64_t)m * args.ld_aux + n0;
+            __nv_bfloat16* bp = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux1)) +
+                                (int64_t)m * args.ld_aux + n0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + v * 8 + 8 <= args.N) {
+                uint32_t hw[4], aw[4], bw[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                  float hv[2], av[2], bv[2];
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const int j = v * 8 + p * 2 + e;
+                    const float s = sigmoidf_(g[j]);
+                    bv[e] = g[j] * s;
+                    hv[e] = bv[e] * u[j];
+                    av[e] = u[j] * s * (1.f + g[j] * (1.f - s));
+                  }
+                  hw[p] = pack_bf16x2(hv[0], hv[1]);
+                  aw[p] = pack_bf16x2(av[0], av[1]);
+                  bw[p] = pack_bf16x2(bv[0], bv[1]);
+                }
+                st_v4(hp + v * 8, hw[0], hw[1], hw[2], hw[3]);
+                if constexpr (EPI == kEpiSwiGLU) {
+                  st_v4(ap + v * 8, aw[0], aw[1], aw[2], aw[3]);
+                  st_v4(bp + v * 8, bw[0], bw[1], bw[2], bw[3]);
+                }
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float acc[32];
+          if (have_acc) {
+            tmem_ld32(t_acc + c, acc);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+          }
+          const int n0 = nb * BN + c;
+          if (!row_ok) continue;
+          if constexpr (EPI == kEpiStore) {
+            __nv_bfloat16* op =
+                m < args.row_split
+                    ? static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0
+                    : static_cast<__nv_bfloat16*>(args.out1) +
+                          (int64_t)(m - args.row_split) * args.ld_out + n0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + v * 8 + 8 <= args.N) {
+                st_v4(op + v * 8, pack_bf16x2(acc[v * 8 + 0], acc[v * 8 + 1]),
+                      pack_bf16x2(acc[v * 8 + 2], acc[v * 8 + 3]),
+                      pack_bf16x2(acc[v * 8 + 4], acc[v * 8 + 5]),
+                      pack_bf16x2(acc[v * 8 + 6], acc[v * 8 + 7]));
+              }
+            }
+          } else if constexpr (EPI == kEpiDGate) {
+            const __nv_bfloat16* ap =
+                static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
+            const __nv_bfloat16* bp =
+                static_cast<const __nv_bfloat16*>(args.aux1) + (int64_t)m * args.ld_aux + n0;
+            __nv_bfloat16* gp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
+            __nv_bfloat16* up = gp + args.d_ff;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + v * 8 + 8 <= args.N) {
+                const uint4 av = *reinterpret_cast<const uint4*>(ap + v * 8);
+                const uint4 bv = *reinterpret_cast<const uint4*>(bp + v * 8);
+                const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+                uint32_t gw[4], uw[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                  const float d0 = acc[v * 8 + p * 2], d1 = acc[v * 8 + p * 2 + 1];
+                  gw[p] = pack_bf16x2(d0 * bf16_lo(aw[p]), d1 * bf16_hi(aw[p]));
+                  uw[p] = pack_bf16x2(d0 * bf16_lo(bw[p]), d1 * bf16_hi(bw[p]));
+                }
+                st_v4(gp + v * 8, gw[0], gw[1], gw[2], gw[3]);
+                st_v4(up + v * 8, uw[0], uw[1], uw[2], uw[3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace swf
