@@ -204,6 +204,46 @@ swf_status swf_device_status(void* stream);
  * out and the kernel records SWF_ERR_TIMEOUT and returns.  Returns the launch status. */
 swf_status swf_selftest_wait_timeout(int32_t limit_us, void* stream);
 
+/* ------------------------------------------------------------------ profiling aid */
+
+/* Kernel kinds the library launches (indices of swf_profile_read's arrays). */
+typedef enum swf_kernel_kind {
+  SWF_K_GATE_UP = 0,       /* training forward: x [W_g|W_u]^T with the SwiGLU epilogue */
+  SWF_K_GATE_UP_INFER = 1, /* inference forward: same, h only */
+  SWF_K_DOWN = 2,          /* y = h W_d^T */
+  SWF_K_DGATE = 3,         /* dH = dY W_d with the gating epilogue -> [dG | dU] */
+  SWF_K_DX = 4,            /* dx = [dG | dU] [W_g ; W_u] */
+  SWF_K_DW_GATE_UP = 5,    /* [dW_g ; dW_u] = [dG | dU]^T x */
+  SWF_K_DW_DOWN = 6,       /* dW_d = dY^T h */
+  SWF_K_F32_GEMM = 7,      /* fp32 CUDA-core GEMM (any dense step) */
+  SWF_K_SELECT_GATHER = 8, /* gather of the subsampled gate rows */
+  SWF_K_SELECT_SCORE = 9,  /* scoring GEMM with the energy epilogue */
+  SWF_K_SELECT_TOPK = 10,  /* warp-level grouped top-k */
+  SWF_K_BUCKETS = 11,      /* group bucketing (count, scan, place) */
+  SWF_K_SPARSE_GATHER = 12,/* gather of token rows into group-major order */
+  SWF_K_SPARSE_UP = 13,    /* sparse gate|up GEMM with the SwiGLU epilogue */
+  SWF_K_SPARSE_DOWN = 14,  /* sparse down GEMM with scatter-add into fp32 */
+  SWF_K_SPARSE_DGATE = 15, /* sparse dH GEMM with the gating epilogue */
+  SWF_K_SPARSE_DX = 16,    /* sparse dx GEMM with scatter-add into fp32 */
+  SWF_K_SPARSE_DW = 17,    /* sparse weight-gradient GEMMs */
+  SWF_K_ELEMENTWISE = 18,  /* zero fill, fp32 -> output dtype conversion */
+  SWF_K_NUM_KINDS = 19
+} swf_kernel_kind;
+
+/* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on
+ * its stream (events are created by the library on first use and reused).  Enabling or
+ * disabling clears the accumulated statistics.  Not thread-safe against concurrent calls of
+ * the other entry points. */
+swf_status swf_profile_enable(int32_t enable);
+
+/* Waits for the recorded events, then adds each bracketed launch to launches[kind] and its
+ * duration (ms) to total_ms[kind] for kind < max_kinds (both arrays zeroed by the call),
+ * and forgets the events.  Returns the number of kinds (SWF_K_NUM_KINDS) or -1 on error. */
+int32_t swf_profile_read(int32_t max_kinds, int64_t* launches, double* total_ms);
+
+/* Static name of a kernel kind ("?" when out of range). */
+const char* swf_kernel_name(int32_t kind);
+
 /* Static, human-readable name of a status code. */
 const char* swf_status_string(swf_status status);
 

@@ -47,6 +47,9 @@ SIGNATURES = {
     "swf_device_status": (I32, [P]),
     "swf_selftest_wait_timeout": (I32, [I32, P]),
     "swf_status_string": (C.c_char_p, [I32]),
+    "swf_profile_enable": (I32, [I32]),
+    "swf_profile_read": (I32, [I32, P, P]),
+    "swf_kernel_name": (C.c_char_p, [I32]),
 }
 
 

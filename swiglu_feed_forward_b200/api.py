@@ -217,3 +217,21 @@ def device_status(stream=None) -> int:
 
 def selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check("swf_selftest_wait_timeout", _lib.lib().swf_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+# ------------------------------------------------------------------ profiling aid
+def profile_enable(enable: bool = True) -> None:
+    _check("swf_profile_enable", _lib.lib().swf_profile_enable(1 if enable else 0))
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total ms)} for the launches bracketed since the last read."""
+    import numpy as np
+    n = 64
+    launches = np.zeros(n, dtype=np.int64)
+    total = np.zeros(n, dtype=np.float64)
+    k = _lib.lib().swf_profile_read(n, C.c_void_p(launches.ctypes.data), C.c_void_p(total.ctypes.data))
+    if k < 0:
+        raise SwfError("swf_profile_read", _lib.SWF_ERR_LAUNCH if hasattr(_lib, "SWF_ERR_LAUNCH") else 5)
+    return {_lib.lib().swf_kernel_name(i).decode(): (int(launches[i]), float(total[i]))
+            for i in range(k) if launches[i] > 0}

@@ -22,8 +22,8 @@ namespace {
 constexpr int kRaster = 8;
 
 template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
-swf_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
-                     TcGemmArgs args, cudaStream_t st) {
+swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
+                     const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
   DevCtx ctx;
   swf_status s = get_ctx(&ctx);
   if (s != SWF_OK) return s;
@@ -37,6 +37,7 @@ swf_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtens
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
+  ProfScope prof(kind, st);
   kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, args);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
@@ -80,14 +81,14 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
   k1.aux0 = a;
   k1.aux1 = b;
   k1.ld_aux = f;
-  swf_status s = infer ? launch_tc<256, false, false, true, kEpiSwiGLUInf>(tx, twg, twu, k1, st)
-                       : launch_tc<256, false, false, true, kEpiSwiGLU>(tx, twg, twu, k1, st);
+  swf_status s = infer ? launch_tc<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, k1, st)
+                       : launch_tc<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, k1, st);
   if (s != SWF_OK) return s;
   // K2: y = h W_d^T
   TcGemmArgs k2 = base_args(M, d, 256, f);
   k2.out0 = y;
   k2.ld_out = d;
-  return launch_tc<256, false, false, false, kEpiStore>(th, twd, twd, k2, st);
+  return launch_tc<256, false, false, false, kEpiStore>(SWF_K_DOWN, th, twd, twd, k2, st);
 }
 
 swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
@@ -106,7 +107,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     k3.aux1 = b;
     k3.ld_aux = f;
     k3.d_ff = (int)f;
-    s = launch_tc<256, false, true, false, kEpiDGate>(tdy, twd, twd, k3, st);
+    s = launch_tc<256, false, true, false, kEpiDGate>(SWF_K_DGATE, tdy, twd, twd, k3, st);
     if (s != SWF_OK) return s;
   }
   {  // K4: dx = dG W_g + dU W_u: A = dGU (K-major, K = 2f), B segments W_g / W_u (MN-major)
@@ -120,7 +121,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     k4.a_koff1 = (int)f;
     k4.out0 = dx;
     k4.ld_out = d;
-    s = launch_tc<256, false, true, false, kEpiStore>(tdgu, twg, twu, k4, st);
+    s = launch_tc<256, false, true, false, kEpiStore>(SWF_K_DX, tdgu, twg, twu, k4, st);
     if (s != SWF_OK) return s;
   }
   {  // K5: [dW_g ; dW_u] = dGU^T x: A = dGU viewed [K=M rows, 2f cols] (MN-major), B = x (MN)
@@ -132,7 +133,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     k5.out1 = dwu;
     k5.row_split = (int)f;
     k5.ld_out = d;
-    s = launch_tc<256, true, true, false, kEpiStore>(tdgu, tx, tx, k5, st);
+    s = launch_tc<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, k5, st);
     if (s != SWF_OK) return s;
   }
   {  // K6: dW_d = dY^T h: A = dY viewed [K=M rows, d cols] (MN), B = h [K=M rows, f cols] (MN)
@@ -142,7 +143,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     TcGemmArgs k6 = base_args(d, f, 256, M);
     k6.out0 = dwd;
     k6.ld_out = f;
-    s = launch_tc<256, true, true, false, kEpiStore>(tdy, th, th, k6, st);
+    s = launch_tc<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, k6, st);
   }
   return s;
 }
@@ -153,6 +154,7 @@ template <int EPI, bool DUAL>
 swf_status launch_simt(const SimtArgs& a, cudaStream_t st) {
   if (a.M == 0 || a.N == 0) return SWF_OK;
   dim3 grid(cdiv(a.N, kSimtTile), cdiv(a.M, kSimtTile));
+  ProfScope prof(SWF_K_F32_GEMM, st);
   simt_gemm_f32<EPI, DUAL><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }

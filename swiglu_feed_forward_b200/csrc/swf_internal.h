@@ -29,6 +29,17 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Brackets one kernel launch with CUDA events while profiling is enabled (swf_profile_*).
+class ProfScope {
+ public:
+  ProfScope(int kind, cudaStream_t st);
+  ~ProfScope();
+ private:
+  int kind_;
+  cudaStream_t st_;
+  cudaEvent_t ev0_ = nullptr;
+};
+
 // Default bound on a single in-kernel wait (ns).
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
