@@ -117,6 +117,28 @@ swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate, con
                           void* dw_down, void* workspace, size_t workspace_bytes, int64_t M,
                           int64_t d_model, int64_t d_ff, swf_dtype dtype, void* stream);
 
+/* Size of the fixed device scratch used by swiglu_ffn_fwd_infer_noalloc (32 MiB). */
+#define SWF_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* Inference forward that allocates nothing and takes no workspace.  The pages have no
+ * counterpart: it exists for callers that cannot provide device memory for the intermediate
+ * h, such as a host program that reaches the library only through this ABI and has no device
+ * allocator, a plug-in inside a runtime that forbids allocation on its execution path, or code
+ * recording a stream capture in a mode where cudaMalloc is an error.  Computes the same y as
+ * swiglu_ffn_fwd_infer, keeping h [M, d_ff] in a file-scope device array of
+ * SWF_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the process exits.
+ *  - Returns SWF_ERR_WORKSPACE, launching nothing, when M * d_ff * element size exceeds
+ *    SWF_NOALLOC_SCRATCH_BYTES (e.g. at most 3048 tokens for bf16 with d_ff = 5504).
+ *  - The first call on each device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture on the device.
+ *  - All calls share the array and it keeps the last call's contents (nothing in it needs to
+ *    start at zero).  Calls whose kernels overlap on the GPU, e.g. on two streams, race on it:
+ *    serialise them.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine. */
+swf_status swiglu_ffn_fwd_infer_noalloc(const void* x, const void* w_gate, const void* w_up,
+                                        const void* w_down, void* y, int64_t M, int64_t d_model,
+                                        int64_t d_ff, swf_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------------ group-sparse variant */
 
 /* Subsample index (eugen_sparse README, make_subsample_index; drawn once per layer).  HOST

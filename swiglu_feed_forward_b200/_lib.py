@@ -33,6 +33,7 @@ IP = C.POINTER(C.c_int32)
 SIGNATURES = {
     "swiglu_ffn_fwd": (I32, [P, P, P, P, P, P, P, P, I64, I64, I64, I32, P]),
     "swiglu_ffn_fwd_infer": (I32, [P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
+    "swiglu_ffn_fwd_infer_noalloc": (I32, [P, P, P, P, P, I64, I64, I64, I32, P]),
     "swiglu_ffn_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swf_make_subsample_index": (I32, [I64, I32, I32, U64, P]),
     "grouped_topk_select": (I32, [P, P, P, I32, P, I32, I32, P, P, P, SZ, I64, I64, I64, I32, P]),
