@@ -9,55 +9,11 @@
 //   K4  dx = dGU [W_g ; W_u]                               (K = 2 d_ff, two B segments)
 //   K5  [dW_g ; dW_u] = dGU^T x                            (K = M)
 //   K6  dW_d = dY^T h                                      (K = M)
-#include <algorithm>
-
 #include "swf_internal.h"
+#include "swf_launch.cuh"
 #include "swf_simt.cuh"
-#include "swf_tc_gemm.cuh"
 
 namespace swf {
-
-namespace {
-
-constexpr int kRaster = 8;
-
-template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
-swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
-                     const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
-  DevCtx ctx;
-  swf_status s = get_ctx(&ctx);
-  if (s != SWF_OK) return s;
-  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk;
-  if (tiles == 0) return SWF_OK;
-  args.status = ctx.status;
-  if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
-  args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI>;
-  constexpr int smem = TcSmem<BN>::kBytes;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return SWF_ERR_LAUNCH;
-  const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
-  ProfScope prof(kind, st);
-  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, args);
-  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
-}
-
-inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
-
-TcGemmArgs base_args(int64_t M, int64_t N, int n_blk_cols, int64_t K) {
-  TcGemmArgs a{};
-  a.M = (int)M;
-  a.N = (int)N;
-  a.num_m_blk = cdiv(M, kTileM);
-  a.num_n_blk = cdiv(N, n_blk_cols);
-  a.raster = kRaster;
-  a.kb_total = cdiv(K, kTileK);
-  a.kb_seg0 = a.kb_total;
-  a.row_split = (int)M;
-  return a;
-}
-
-}  // namespace
 
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f) {
   auto t = [](int64_t m, int64_t n, int64_t bn) { return (int64_t)cdiv(m, kTileM) * cdiv(n, bn); };

@@ -1,0 +1,50 @@
+// Host launcher of the tcgen05 GEMM template, shared by the dense and group-sparse paths.
+#pragma once
+#include <algorithm>
+
+#include "swf_internal.h"
+#include "swf_tc_gemm.cuh"
+
+namespace swf {
+
+inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+// Launches tc_gemm_kernel on min(tiles, SMs) persistent CTAs, bracketed for profiling as `kind`.
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense>
+swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
+                     const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
+  DevCtx ctx;
+  swf_status s = get_ctx(&ctx);
+  if (s != SWF_OK) return s;
+  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk *
+                        (MODE == kModeKGrouped ? args.n_groups : 1);
+  if (tiles == 0) return SWF_OK;
+  if (tiles > INT32_MAX) return SWF_ERR_UNSUPPORTED;
+  args.status = ctx.status;
+  if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
+  args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE>;
+  constexpr int smem = TcSmem<BN>::kBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
+  ProfScope prof(kind, st);
+  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, args);
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
+// Arguments of a dense GEMM of M x N (N-blocks of n_blk_cols columns) over K.
+inline TcGemmArgs base_args(int64_t M, int64_t N, int n_blk_cols, int64_t K) {
+  TcGemmArgs a{};
+  a.M = (int)M;
+  a.N = (int)N;
+  a.num_m_blk = cdiv(M, kTileM);
+  a.num_n_blk = cdiv(N, n_blk_cols);
+  a.raster = 8;
+  a.kb_total = cdiv(K, kTileK);
+  a.kb_seg0 = a.kb_total;
+  a.row_split = (int)M;
+  return a;
+}
+
+}  // namespace swf

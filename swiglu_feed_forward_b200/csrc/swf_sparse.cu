@@ -1,23 +1,519 @@
-// Group-sparse SwiGLU FFN (eugen_sparse README): subsample index, grouped top-k selection,
-// group bucketing, sparse forward and backward.
+// Group-sparse SwiGLU FFN (eugen_sparse README, "What it does", "Parameters and how to choose
+// them", "Pitfalls and limitations"): subsample index, grouped top-k selection, group
+// bucketing, sparse forward and backward.
+//
+// Layout of the group-major ("padded") row space shared by the sparse kernels: the
+// (token, group) pairs are bucketed by group, ascending token within a group; group g owns the
+// rows [seg_start[g], seg_start[g] + seg_rows[g]) where seg_rows[g] is its pair count rounded
+// up to 128, so that every 128-row tile belongs to one group (tile_group[tile], -1 when the
+// tile is past the last group).  row_token[r] is the token of padded row r (-1: padding);
+// padding rows of every group-major buffer are zero, so they add nothing to any sum.
+#include <algorithm>
 #include <vector>
 
+#include "swf_launch.cuh"
 #include "swf_sparse.h"
 
 namespace swf {
 
-size_t select_workspace_bytes(int64_t, int64_t, int64_t, int32_t, int32_t) { return 0; }
-size_t sparse_fwd_workspace_bytes(int64_t, int64_t, int64_t, int32_t, int32_t) { return 0; }
-size_t sparse_bwd_workspace_bytes(int64_t, int64_t, int64_t, int32_t, int32_t) { return 0; }
-size_t buckets_workspace_bytes(int64_t, int32_t, int32_t) { return 0; }
-size_t sparse_saved_bytes(int64_t, int64_t, int64_t, int32_t, int32_t) { return 0; }
-void sparse_plan(int, int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, swf_plan_info* p) {
-  p->num_kernels = 0;
+namespace {
+
+constexpr int kBucketSmemBytes = 98304;
+
+struct SparseDims {
+  int64_t M, d, f;
+  int G, K, ng;
+  int64_t pairs;
+  int64_t rmax;   // rows of the padded space (upper bound)
+  int mblk;       // 128-row tiles of the padded space
+  int words;      // 32-token words per bucketing block
+  int tok_blk;    // tokens per bucketing block
+  int nblk;       // bucketing blocks
+};
+
+SparseDims dims_of(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
+  SparseDims s{};
+  s.M = M, s.d = d, s.f = f, s.G = G, s.K = K;
+  s.ng = (int)(f / G);
+  s.pairs = M * K;
+  s.rmax = (int64_t)round_up((size_t)(s.pairs + (int64_t)s.ng * 127), 128);
+  s.mblk = (int)(s.rmax / 128);
+  s.words = std::max(1, std::min(32, kBucketSmemBytes / (8 * std::max(1, s.ng))));
+  s.tok_blk = 32 * s.words;
+  s.nblk = (int)((M + s.tok_blk - 1) / s.tok_blk);
+  return s;
+}
+
+// Carves consecutive 256-byte aligned pieces out of one buffer.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = round_up(off + count * sizeof(T), 256);
+    return p;
+  }
+};
+
+struct SavedView {
+  int32_t *offs, *tokens, *seg_start, *seg_rows, *tile_group, *row_token;
+  __nv_bfloat16 *h, *a, *b;
+};
+
+SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
+  Carver c{static_cast<char*>(base)};
+  SavedView v;
+  v.offs = c.take<int32_t>(s.ng + 1);
+  v.tokens = c.take<int32_t>(s.pairs);
+  v.seg_start = c.take<int32_t>(s.ng + 1);
+  v.seg_rows = c.take<int32_t>(s.ng);
+  v.tile_group = c.take<int32_t>(s.mblk);
+  v.row_token = c.take<int32_t>(s.rmax);
+  v.h = c.take<__nv_bfloat16>(s.rmax * s.G);
+  v.a = c.take<__nv_bfloat16>(s.rmax * s.G);
+  v.b = c.take<__nv_bfloat16>(s.rmax * s.G);
+  if (bytes) *bytes = c.off;
+  return v;
+}
+
+struct FwdWs {
+  int32_t* counts;
+  __nv_bfloat16* xc;
+  float* y32;
+};
+FwdWs fwd_ws(void* base, const SparseDims& s, size_t* bytes) {
+  Carver c{static_cast<char*>(base)};
+  FwdWs w;
+  w.counts = c.take<int32_t>((size_t)s.nblk * s.ng);
+  w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
+  w.y32 = c.take<float>(s.M * s.d);
+  if (bytes) *bytes = c.off;
+  return w;
+}
+
+struct BwdWs {
+  __nv_bfloat16 *xc, *dyc, *dgu;
+  float* dx32;
+};
+BwdWs bwd_ws(void* base, const SparseDims& s, size_t* bytes) {
+  Carver c{static_cast<char*>(base)};
+  BwdWs w;
+  w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
+  w.dyc = c.take<__nv_bfloat16>(s.rmax * s.d);
+  w.dgu = c.take<__nv_bfloat16>(s.rmax * 128);
+  w.dx32 = c.take<float>(s.M * s.d);
+  if (bytes) *bytes = c.off;
+  return w;
+}
+
+int pow2_at_least(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+struct SelWs {
+  __nv_bfloat16* wsub;
+  float* energies;
+};
+SelWs sel_ws(void* base, int64_t M, int64_t d, int ng, int P, bool need_wsub, bool need_e,
+             size_t* bytes) {
+  Carver c{static_cast<char*>(base)};
+  SelWs w{nullptr, nullptr};
+  if (need_wsub) w.wsub = c.take<__nv_bfloat16>((size_t)ng * P * d);
+  if (need_e) w.energies = c.take<float>((size_t)M * ng);
+  if (bytes) *bytes = c.off;
+  return w;
+}
+
+// ------------------------------------------------------------------ device kernels
+
+// Slot k of a group_idx row counts only if its group is in range and not repeated earlier in
+// the row (duplicates and out-of-range values are outside the contract; they are dropped so
+// that no kernel reads or writes out of bounds).
+__device__ __forceinline__ bool valid_slot(const int32_t* row, int k, int ng) {
+  const int c = row[k];
+  if (c < 0 || c >= ng) return false;
+  for (int j = 0; j < k; ++j)
+    if (row[j] == c) return false;
+  return true;
+}
+
+__global__ void bucket_count_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
+                                    int tok_blk, int32_t* __restrict__ counts) {
+  extern __shared__ int32_t hist[];
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * tok_blk;
+  for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
+    const int64_t t = t0 + i / K;
+    if (t >= M) break;
+    const int32_t* row = idx + t * K;
+    const int k = i % K;
+    if (valid_slot(row, k, ng)) atomicAdd(&hist[row[k]], 1);
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) counts[(int64_t)blockIdx.x * ng + c] = hist[c];
+}
+
+// One block: turns per-block counts into exclusive per-block bases, writes the CSR offsets
+// and, when seg_start is given, the padded segments and the tile -> group table.
+__global__ void bucket_scan_kernel(int32_t* __restrict__ counts, int nblk, int ng,
+                                   int32_t* __restrict__ offs, int32_t* __restrict__ seg_start,
+                                   int32_t* __restrict__ seg_rows, int32_t* __restrict__ tile_group,
+                                   int mblk) {
+  extern __shared__ int32_t sh[];
+  int32_t* tot = sh;            // [ng]
+  int32_t* sstart = sh + ng;    // [ng + 1]
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) {
+    int32_t run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int32_t v = counts[(int64_t)b * ng + c];
+      counts[(int64_t)b * ng + c] = run;
+      run += v;
+    }
+    tot[c] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t o = 0, p = 0;
+    for (int c = 0; c < ng; ++c) {
+      offs[c] = o;
+      sstart[c] = p;
+      o += tot[c];
+      p += (tot[c] + 127) / 128 * 128;
+    }
+    offs[ng] = o;
+    sstart[ng] = p;
+  }
+  __syncthreads();
+  if (seg_start == nullptr) return;
+  for (int c = threadIdx.x; c <= ng; c += blockDim.x) {
+    seg_start[c] = sstart[c];
+    if (c < ng) seg_rows[c] = sstart[c + 1] - sstart[c];
+  }
+  for (int mb = threadIdx.x; mb < mblk; mb += blockDim.x) {
+    const int r = mb * 128;
+    int g = -1;
+    if (r < sstart[ng]) {
+      int lo = 0, hi = ng - 1;  // last group with sstart[g] <= r
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (sstart[mid] <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      g = lo;
+    }
+    tile_group[mb] = g;
+  }
+}
+
+// Places every valid (token, group) pair: rank among the block's tokens of the same group from
+// a per-group bitmap of the block's tokens, so the order within a group is ascending token id.
+__global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
+                                    int words, const int32_t* __restrict__ counts,
+                                    const int32_t* __restrict__ offs, int32_t* __restrict__ tokens,
+                                    const int32_t* __restrict__ seg_start,
+                                    int32_t* __restrict__ row_token) {
+  extern __shared__ uint32_t smem_bits[];
+  uint32_t* bits = smem_bits;                                        // [ng][words]
+  int32_t* pre = reinterpret_cast<int32_t*>(smem_bits + (size_t)ng * words);  // [ng][words]
+  const int tok_blk = 32 * words;
+  for (int i = threadIdx.x; i < ng * words; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * tok_blk;
+  for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
+    const int tl = i / K;
+    const int64_t t = t0 + tl;
+    if (t >= M) break;
+    const int32_t* row = idx + t * K;
+    const int k = i % K;
+    if (valid_slot(row, k, ng)) atomicOr(&bits[row[k] * words + (tl >> 5)], 1u << (tl & 31));
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < words; ++w) {
+      pre[c * words + w] = run;
+      run += __popc(bits[c * words + w]);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
+    const int tl = i / K;
+    const int64_t t = t0 + tl;
+    if (t >= M) break;
+    const int32_t* row = idx + t * K;
+    const int k = i % K;
+    if (!valid_slot(row, k, ng)) continue;
+    const int c = row[k];
+    const int w = tl >> 5;
+    const int rank = pre[c * words + w] + __popc(bits[c * words + w] & ((1u << (tl & 31)) - 1u));
+    const int32_t base = counts[(int64_t)blockIdx.x * ng + c] + rank;
+    tokens[offs[c] + base] = (int32_t)t;
+    if (row_token) row_token[seg_start[c] + base] = (int32_t)t;
+  }
+}
+
+__global__ void fill_i32_kernel(int32_t* __restrict__ p, int64_t n, int32_t v) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+__global__ void zero_f32_kernel(float4* __restrict__ p, int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+// dst[r, :] = src[row_token[r], :] (zero for padding) for the padded rows in use; one warp per
+// row, 16-byte vectors.
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ row_token,
+                                   const int32_t* __restrict__ seg_start_total, int64_t row_vecs,
+                                   uint4* __restrict__ dst) {
+  const int64_t rows = *seg_start_total;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int32_t tok = row_token[r];
+    uint4* d = dst + r * row_vecs;
+    if (tok < 0) {
+      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      const uint4* s = src + (int64_t)tok * row_vecs;
+      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = s[v];
+    }
+  }
+}
+
+// Wsub[c*P + i, :] = w_gate[sub[c*spg + i], :] for i < spg, zero rows for spg <= i < P (zero rows
+// add |SiLU(0)| = 0 to the energy).  Row ids outside group c are treated as zero rows.
+__global__ void select_gather_kernel(const uint4* __restrict__ w, const int32_t* __restrict__ sub,
+                                     int ng, int G, int spg, int P, int64_t row_vecs,
+                                     uint4* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)ng * P;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int c = (int)(r / P), i = (int)(r % P);
+    int src = -1;
+    if (i < spg) {
+      src = sub[(int64_t)c * spg + i];
+      if (src < c * G || src >= (c + 1) * G) src = -1;
+    }
+    uint4* d = dst + r * row_vecs;
+    if (src < 0) {
+      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      const uint4* s = w + (int64_t)src * row_vecs;
+      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = s[v];
+    }
+  }
+}
+
+// One warp per token: K rounds of a warp-wide argmax over the group scores (larger score first,
+// lower group index among equal scores), then the chosen groups written in ascending order.
+template <int VPL>
+__global__ void topk_kernel(const float* __restrict__ E, int64_t M, int ng, int K,
+                            int32_t* __restrict__ idx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (m >= M) return;  // uniform per warp
+  const float* row = E + m * ng;
+  float v[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int c = lane + 32 * j;
+    v[j] = c < ng ? row[c] : -INFINITY;
+  }
+  uint64_t taken = 0;
+  int chosen = 0;
+  for (int r = 0; r < K; ++r) {
+    float bv = -INFINITY;
+    int bc = INT32_MAX;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int c = lane + 32 * j;
+      if (c < ng && !((taken >> j) & 1ull) && (v[j] > bv || (v[j] == bv && c < bc))) {
+        bv = v[j];
+        bc = c;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
+      if (ov > bv || (ov == bv && oc < bc)) {
+        bv = ov;
+        bc = oc;
+      }
+    }
+    if (bc >= ng) break;  // nothing left that compares (only NaN scores remain)
+    if ((bc & 31) == lane) taken |= 1ull << (bc >> 5);
+    ++chosen;
+  }
+  int base = 0;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const bool bit = (taken >> j) & 1ull;
+    const unsigned mask = __ballot_sync(0xffffffffu, bit);
+    if (bit) idx[m * K + base + __popc(mask & ((1u << lane) - 1u))] = lane + 32 * j;
+    base += __popc(mask);
+  }
+  for (int p = chosen + lane; p < K; p += 32) idx[m * K + p] = -1;
+}
+
+// ------------------------------------------------------------------ host helpers
+
+inline int grid_for(int64_t work, int per_block) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>((work + per_block - 1) / per_block, 148 * 16));
+}
+
+swf_status launched() { return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH; }
+
+swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts, int32_t* offs,
+                       int32_t* tokens, int32_t* seg_start, int32_t* seg_rows,
+                       int32_t* tile_group, int32_t* row_token, cudaStream_t st) {
+  {
+    ProfScope prof(SWF_K_BUCKETS, st);
+    bucket_count_kernel<<<s.nblk, 256, s.ng * sizeof(int32_t), st>>>(idx, s.M, s.K, s.ng, s.tok_blk, counts);
+    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
+  }
+  const size_t scan_smem = (2 * (size_t)s.ng + 1) * sizeof(int32_t);
+  if (scan_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(bucket_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  {
+    ProfScope prof(SWF_K_BUCKETS, st);
+    bucket_scan_kernel<<<1, 1024, scan_smem, st>>>(counts, s.nblk, s.ng, offs, seg_start, seg_rows,
+                                                   tile_group, s.mblk);
+    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
+  }
+  if (row_token) {
+    ProfScope prof(SWF_K_ELEMENTWISE, st);
+    fill_i32_kernel<<<grid_for(s.rmax, 256), 256, 0, st>>>(row_token, s.rmax, -1);
+    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
+  }
+  const size_t place_smem = (size_t)8 * s.ng * s.words;
+  if (cudaFuncSetAttribute(bucket_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)place_smem) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  ProfScope prof(SWF_K_BUCKETS, st);
+  bucket_place_kernel<<<s.nblk, 256, place_smem, st>>>(idx, s.M, s.K, s.ng, s.words, counts, offs,
+                                                       tokens, seg_start, row_token);
+  return launched();
+}
+
+swf_status run_gather(const void* src, const SavedView& v, const SparseDims& s, void* dst,
+                      cudaStream_t st) {
+  ProfScope prof(SWF_K_SPARSE_GATHER, st);
+  gather_rows_kernel<<<148 * 8, 256, 0, st>>>(static_cast<const uint4*>(src), v.row_token,
+                                              v.seg_start + s.ng, s.d / 8, static_cast<uint4*>(dst));
+  return launched();
+}
+
+swf_status run_zero(float* p, int64_t n, cudaStream_t st) {
+  ProfScope prof(SWF_K_ELEMENTWISE, st);
+  zero_f32_kernel<<<grid_for(n / 4, 256), 256, 0, st>>>(reinterpret_cast<float4*>(p), n / 4);
+  return launched();
+}
+
+swf_status run_convert(const float* src, void* dst, int64_t n, cudaStream_t st) {
+  ProfScope prof(SWF_K_ELEMENTWISE, st);
+  f32_to_bf16_kernel<<<grid_for(n / 4, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(src),
+                                                           static_cast<uint2*>(dst), n / 4);
+  return launched();
+}
+
+template <int VPL>
+swf_status launch_topk(const float* E, int64_t M, int ng, int K, int32_t* idx, cudaStream_t st) {
+  ProfScope prof(SWF_K_SELECT_TOPK, st);
+  topk_kernel<VPL><<<(unsigned)((M + 7) / 8), 256, 0, st>>>(E, M, ng, K, idx);
+  return launched();
+}
+
+constexpr int kMaxSelectGroups = 2048;
+
+}  // namespace
+
+// ------------------------------------------------------------------ sizes and plans
+
+size_t select_workspace_bytes(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
+  (void)K;
+  const int ng = (int)(f / G);
+  size_t bytes = 0;
+  // worst case: subsample given (P = G) and energies not supplied by the caller
+  sel_ws(nullptr, M, d, ng, G, true, true, &bytes);
+  return bytes;
+}
+
+size_t sparse_fwd_workspace_bytes(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
+  size_t bytes = 0;
+  fwd_ws(nullptr, dims_of(M, d, f, G, K), &bytes);
+  return bytes;
+}
+
+size_t sparse_bwd_workspace_bytes(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
+  size_t bytes = 0;
+  bwd_ws(nullptr, dims_of(M, d, f, G, K), &bytes);
+  return bytes;
+}
+
+size_t buckets_workspace_bytes(int64_t M, int32_t K, int32_t ng) {
+  const SparseDims s = dims_of(M, 16, (int64_t)ng * 16, 16, K);
+  return round_up((size_t)s.nblk * s.ng * sizeof(int32_t), 256);
+}
+
+size_t sparse_saved_bytes(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
+  size_t bytes = 0;
+  saved_view(nullptr, dims_of(M, d, f, G, K), &bytes);
+  return bytes;
+}
+
+void sparse_plan(int op, int64_t M, int64_t d, int64_t f, int32_t G, int32_t K, int32_t spg,
+                 swf_plan_info* p) {
+  const SparseDims s = dims_of(M, d, f, G, K);
+  p->deterministic = (op == SWF_OP_SELECT || op == SWF_OP_BUCKETS) ? 1 : 0;
+  p->saved_bytes = (op == SWF_OP_SPARSE_FWD || op == SWF_OP_SPARSE_BWD) ? sparse_saved_bytes(M, d, f, G, K) : 0;
+  const int P = spg > 0 ? pow2_at_least(spg) : G;
+  switch (op) {
+    case SWF_OP_SELECT:
+      p->num_kernels = spg > 0 ? 3 : 2;
+      p->flops = 2 * M * d * (int64_t)s.ng * (spg > 0 ? spg : G);
+      p->gemm_tiles = (int64_t)cdiv(M, 128) * cdiv((int64_t)s.ng * P, 256);
+      break;
+    case SWF_OP_SPARSE_FWD:
+      p->num_kernels = 8;
+      p->flops = 6 * M * d * (int64_t)K * G;
+      p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256));
+      p->tile_n = 2 * G;
+      break;
+    case SWF_OP_SPARSE_BWD:
+      p->num_kernels = 8;
+      p->flops = 12 * M * d * (int64_t)K * G;
+      p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256)) + (int64_t)s.ng * (cdiv(d, 256) + cdiv(d, 128));
+      break;
+    case SWF_OP_BUCKETS:
+      p->num_kernels = 3;
+      p->flops = 0;
+      p->gemm_tiles = 0;
+      break;
+    default:
+      break;
+  }
 }
 
 }  // namespace swf
 
 using namespace swf;
+
+// ------------------------------------------------------------------ subsample (host)
 
 // splitmix64 (Steele, Lea & Flood, OOPSLA 2014): one output per call.
 static inline uint64_t splitmix64_next(uint64_t& state) {
@@ -40,40 +536,247 @@ extern "C" swf_status swf_make_subsample_index(int64_t d_ff, int32_t G, int32_t 
     for (int32_t i = 0; i < spg; ++i) {
       const uint64_t r = splitmix64_next(state);
       const int32_t j = i + (int32_t)(r % (uint64_t)(G - i));
-      const int32_t t = perm[i];
-      perm[i] = perm[j];
-      perm[j] = t;
+      std::swap(perm[i], perm[j]);
     }
-    // ascending order of the chosen offsets (insertion sort; spg <= G is small)
-    for (int32_t i = 1; i < spg; ++i) {
-      const int32_t v = perm[i];
-      int32_t k = i - 1;
-      while (k >= 0 && perm[k] > v) { perm[k + 1] = perm[k]; --k; }
-      perm[k + 1] = v;
-    }
+    std::sort(perm.begin(), perm.begin() + spg);
     for (int32_t i = 0; i < spg; ++i) out[c * spg + i] = (int32_t)(c * G + perm[i]);
   }
   return SWF_OK;
 }
 
-extern "C" swf_status grouped_topk_select(const void*, const void*, const int32_t*, int32_t,
-                                          const float*, int32_t, int32_t, int32_t*, float*, void*,
-                                          size_t, int64_t, int64_t, int64_t, swf_dtype, void*) {
-  return SWF_ERR_UNSUPPORTED;
+// ------------------------------------------------------------------ selection
+
+extern "C" swf_status grouped_topk_select(const void* x, const void* w_gate,
+                                          const int32_t* subsample_idx, int32_t spg,
+                                          const float* bias, int32_t G, int32_t K,
+                                          int32_t* group_idx, float* energies, void* workspace,
+                                          size_t ws_bytes, int64_t M, int64_t d, int64_t f,
+                                          swf_dtype dt, void* stream) {
+  if (!x || !w_gate || !group_idx) return SWF_ERR_INVALID_ARG;
+  swf_status s = check_sparse_shape(M, d, f, G, K, dt);
+  if (s != SWF_OK) return s;
+  const int ng = (int)(f / G);
+  if (ng > kMaxSelectGroups) return SWF_ERR_UNSUPPORTED;
+  if (subsample_idx && (spg < 1 || spg > G)) return SWF_ERR_UNSUPPORTED;
+  for (const void* p : {x, w_gate, (const void*)group_idx})
+    if (!aligned16(p)) return SWF_ERR_ALIGNMENT;
+  if ((energies && !aligned16(energies)) || (subsample_idx && !aligned16(subsample_idx)) ||
+      (bias && !aligned16(bias)) || (workspace && !aligned16(workspace)))
+    return SWF_ERR_ALIGNMENT;
+  const int P = subsample_idx ? pow2_at_least(spg) : G;
+  size_t need = 0;
+  SelWs w = sel_ws(workspace, M, d, ng, P, subsample_idx != nullptr, energies == nullptr, &need);
+  if (need > 0 && (!workspace || ws_bytes < need)) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* E = energies ? energies : w.energies;
+
+  const void* wrows = w_gate;
+  if (subsample_idx) {
+    ProfScope prof(SWF_K_SELECT_GATHER, st);
+    select_gather_kernel<<<grid_for((int64_t)ng * P, 8), 256, 0, st>>>(
+        static_cast<const uint4*>(w_gate), subsample_idx, ng, G, spg, P, d / 8,
+        reinterpret_cast<uint4*>(w.wsub));
+    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
+    wrows = w.wsub;
+  }
+  // scoring GEMM: E[m, c] = sum over the group's P columns of |SiLU(x . w_row)| (+ bias)
+  CUtensorMap tx, tw;
+  const int64_t ncols = (int64_t)ng * P;
+  if (!encode_tmap_bf16(&tx, x, d, M, d, 64, 128) || !encode_tmap_bf16(&tw, wrows, d, ncols, d, 64, 256))
+    return SWF_ERR_LAUNCH;
+  TcGemmArgs a = base_args(M, ncols, 256, d);
+  a.out0 = E;
+  a.ld_out = ng;
+  a.energy_p = P;
+  a.n_groups = ng;
+  a.bias = bias;
+  s = launch_tc<256, false, false, false, kEpiEnergy>(SWF_K_SELECT_SCORE, tx, tw, tw, a, st);
+  if (s != SWF_OK) return s;
+  if (ng <= 32) return launch_topk<1>(E, M, ng, K, group_idx, st);
+  if (ng <= 64) return launch_topk<2>(E, M, ng, K, group_idx, st);
+  if (ng <= 128) return launch_topk<4>(E, M, ng, K, group_idx, st);
+  if (ng <= 256) return launch_topk<8>(E, M, ng, K, group_idx, st);
+  if (ng <= 512) return launch_topk<16>(E, M, ng, K, group_idx, st);
+  if (ng <= 1024) return launch_topk<32>(E, M, ng, K, group_idx, st);
+  return launch_topk<64>(E, M, ng, K, group_idx, st);
 }
-extern "C" swf_status swf_group_buckets(const int32_t*, int64_t, int32_t, int32_t, int32_t*,
-                                        int32_t*, void*, size_t, void*) {
-  return SWF_ERR_UNSUPPORTED;
+
+// ------------------------------------------------------------------ bucketing
+
+extern "C" swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t K, int32_t ng,
+                                        int32_t* offsets, int32_t* tokens, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  if (!group_idx || !offsets || !tokens || !workspace) return SWF_ERR_INVALID_ARG;
+  swf_status s = swf_supported(SWF_OP_BUCKETS, M, 0, 0, ng, K, 0, SWF_BF16);
+  if (s != SWF_OK) return s;
+  if (ng > 12288) return SWF_ERR_UNSUPPORTED;
+  if (!aligned16(workspace)) return SWF_ERR_ALIGNMENT;
+  if (ws_bytes < buckets_workspace_bytes(M, K, ng)) return SWF_ERR_WORKSPACE;
+  const SparseDims d = dims_of(M, 16, (int64_t)ng * 16, 16, K);
+  return run_buckets(group_idx, d, static_cast<int32_t*>(workspace), offsets, tokens, nullptr,
+                     nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
-extern "C" swf_status sparse_swiglu_ffn_fwd(const void*, const void*, const void*, const void*,
-                                            const int32_t*, int32_t, int32_t, void*, void*, size_t,
-                                            void*, size_t, int64_t, int64_t, int64_t, swf_dtype,
-                                            void*) {
-  return SWF_ERR_UNSUPPORTED;
+
+// ------------------------------------------------------------------ sparse forward
+
+namespace {
+swf_status check_sparse_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p) return SWF_ERR_INVALID_ARG;
+  for (const void* p : ps)
+    if (!aligned16(p)) return SWF_ERR_ALIGNMENT;
+  return SWF_OK;
 }
-extern "C" swf_status sparse_swiglu_ffn_bwd(const void*, const void*, const void*, const void*,
-                                            const void*, const int32_t*, const void*, size_t, void*,
-                                            void*, void*, void*, void*, size_t, int64_t, int64_t,
-                                            int64_t, int32_t, int32_t, swf_dtype, void*) {
-  return SWF_ERR_UNSUPPORTED;
+}  // namespace
+
+extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, const void* w_up,
+                                            const void* w_down, const int32_t* group_idx,
+                                            int32_t G, int32_t K, void* y, void* saved,
+                                            size_t saved_bytes, void* workspace, size_t ws_bytes,
+                                            int64_t M, int64_t d, int64_t f, swf_dtype dt,
+                                            void* stream) {
+  swf_status s = check_sparse_ptrs({x, w_gate, w_up, w_down, group_idx, y, saved, workspace});
+  if (s != SWF_OK) return s;
+  if ((s = check_sparse_shape(M, d, f, G, K, dt)) != SWF_OK) return s;
+  if ((int64_t)(f / G) > 12288) return SWF_ERR_UNSUPPORTED;
+  const SparseDims sd = dims_of(M, d, f, G, K);
+  size_t need_saved = 0, need_ws = 0;
+  const SavedView v = saved_view(saved, sd, &need_saved);
+  const FwdWs w = fwd_ws(workspace, sd, &need_ws);
+  if (saved_bytes < need_saved || ws_bytes < need_ws) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if ((s = run_buckets(group_idx, sd, w.counts, v.offs, v.tokens, v.seg_start, v.seg_rows,
+                       v.tile_group, v.row_token, st)) != SWF_OK)
+    return s;
+  if ((s = run_gather(x, v, sd, w.xc, st)) != SWF_OK) return s;
+
+  {  // gate|up per group: [h|a|b] rows = SiLU/gating of Xc [W_g[g] | W_u[g]]^T
+    CUtensorMap txc, twg, twu;
+    if (!encode_tmap_bf16(&txc, w.xc, d, sd.rmax, d, 64, 128) ||
+        !encode_tmap_bf16(&twg, w_gate, d, f, d, 64, G) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, G))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(sd.rmax, G, 2 * G, d);
+    a.num_n_blk = 1;
+    a.tile_group = v.tile_group;
+    a.grp_b_n = G;
+    a.out0 = v.h;
+    a.ld_out = G;
+    a.aux0 = v.a;
+    a.aux1 = v.b;
+    a.ld_aux = G;
+    if (G == 16) s = launch_tc<32, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
+    else if (G == 32) s = launch_tc<64, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
+    else s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
+    if (s != SWF_OK) return s;
+  }
+  if ((s = run_zero(w.y32, M * d, st)) != SWF_OK) return s;
+  {  // down per group: y32[token] += h_row W_d[:, g*G .. g*G+G]^T
+    CUtensorMap th, twd;
+    if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 256))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(sd.rmax, d, 256, G);
+    a.tile_group = v.tile_group;
+    a.grp_b_k = G;
+    a.row_token = v.row_token;
+    a.acc32 = w.y32;
+    a.ld_acc = d;
+    s = launch_tc<256, false, false, false, kEpiScatterAdd, kModeRowGrouped>(SWF_K_SPARSE_DOWN, th, twd, twd, a, st);
+    if (s != SWF_OK) return s;
+  }
+  return run_convert(w.y32, y, M * d, st);
+}
+
+// ------------------------------------------------------------------ sparse backward
+
+extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate,
+                                            const void* w_up, const void* w_down,
+                                            const int32_t* group_idx, const void* saved,
+                                            size_t saved_bytes, void* dx, void* dw_gate,
+                                            void* dw_up, void* dw_down, void* workspace,
+                                            size_t ws_bytes, int64_t M, int64_t d, int64_t f,
+                                            int32_t G, int32_t K, swf_dtype dt, void* stream) {
+  swf_status s = check_sparse_ptrs({dy, x, w_gate, w_up, w_down, group_idx, saved, dx, dw_gate,
+                                    dw_up, dw_down, workspace});
+  if (s != SWF_OK) return s;
+  if ((s = check_sparse_shape(M, d, f, G, K, dt)) != SWF_OK) return s;
+  if ((int64_t)(f / G) > 12288) return SWF_ERR_UNSUPPORTED;
+  const SparseDims sd = dims_of(M, d, f, G, K);
+  size_t need_saved = 0, need_ws = 0;
+  const SavedView v = saved_view(const_cast<void*>(saved), sd, &need_saved);
+  const BwdWs w = bwd_ws(workspace, sd, &need_ws);
+  if (saved_bytes < need_saved || ws_bytes < need_ws) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if ((s = run_gather(x, v, sd, w.xc, st)) != SWF_OK) return s;
+  if ((s = run_gather(dy, v, sd, w.dyc, st)) != SWF_OK) return s;
+  {  // dH = dYc W_d[:, g]; dG = dH * a, dU = dH * b -> dgu [R, 128] (halves padded to 64)
+    CUtensorMap tdyc, twd;
+    if (!encode_tmap_bf16(&tdyc, w.dyc, d, sd.rmax, d, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(sd.rmax, G, 64, d);
+    a.num_n_blk = 1;
+    a.tile_group = v.tile_group;
+    a.grp_b_n = G;
+    a.out0 = w.dgu;
+    a.ld_out = 128;
+    a.d_ff = 64;
+    a.pad_cols = 64;
+    a.aux0 = v.a;
+    a.aux1 = v.b;
+    a.ld_aux = G;
+    s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped>(SWF_K_SPARSE_DGATE, tdyc, twd, twd, a, st);
+    if (s != SWF_OK) return s;
+  }
+  if ((s = run_zero(w.dx32, M * d, st)) != SWF_OK) return s;
+  {  // dx32[token] += dG_row W_g[g] + dU_row W_u[g]
+    CUtensorMap tdgu, twg, twu;
+    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 128) ||
+        !encode_tmap_bf16(&twg, w_gate, d, f, d, 64, 64) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(sd.rmax, d, 256, 128);
+    a.kb_seg0 = 1;
+    a.kb_total = 2;
+    a.a_koff1 = 64;
+    a.tile_group = v.tile_group;
+    a.grp_b_k = G;
+    a.row_token = v.row_token;
+    a.acc32 = w.dx32;
+    a.ld_acc = d;
+    s = launch_tc<256, false, true, false, kEpiScatterAdd, kModeRowGrouped>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st);
+    if (s != SWF_OK) return s;
+  }
+  if ((s = run_convert(w.dx32, dx, M * d, st)) != SWF_OK) return s;
+  {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ Xc_seg
+    CUtensorMap tdgu, txc;
+    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64) ||
+        !encode_tmap_bf16(&txc, w.xc, d, sd.rmax, d, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(128, d, 256, 0);
+    a.n_groups = sd.ng;
+    a.seg_start = v.seg_start;
+    a.seg_rows = v.seg_rows;
+    a.kb_seg0 = 1 << 30;
+    a.group_size = G;
+    a.out0 = dw_gate;
+    a.out1 = dw_up;
+    a.ld_out = d;
+    s = launch_tc<256, true, true, false, kEpiGroupDWgu, kModeKGrouped>(SWF_K_SPARSE_DW, tdgu, txc, txc, a, st);
+    if (s != SWF_OK) return s;
+  }
+  {  // per group: dW_d[:, g] = dYc_segᵀ h_seg
+    CUtensorMap tdyc, th;
+    if (!encode_tmap_bf16(&tdyc, w.dyc, d, sd.rmax, d, 64, 64) || !encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(d, G, 64, 0);
+    a.n_groups = sd.ng;
+    a.seg_start = v.seg_start;
+    a.seg_rows = v.seg_rows;
+    a.kb_seg0 = 1 << 30;
+    a.group_size = G;
+    a.out0 = dw_down;
+    a.ld_out = f;
+    s = launch_tc<64, true, true, false, kEpiGroupDWd, kModeKGrouped>(SWF_K_SPARSE_DW, tdyc, th, th, a, st);
+  }
+  return s;
 }

@@ -10,11 +10,25 @@
 // tile i+1.  Either operand may be K-major (rows of K contiguous) or MN-major (rows of M or N
 // contiguous); the tensor-core descriptors read both layouts, so no transposes are needed.
 //
-// Epilogues (flash-swiglu-mlp overview; parameter-golf PR 1105 "Fused MLP Kernels"):
-//   kEpiStore     C -> bf16, row m < row_split to out0 else out1 (two weight-gradient halves)
-//   kEpiSwiGLU    gate|up dual tile: h = SiLU(g)*u, a = u*SiLU'(g), b = SiLU(g) -> bf16
-//   kEpiSwiGLUInf same, h only
-//   kEpiDGate     C = dH: dG = dH*a -> out0[:, n], dU = dH*b -> out0[:, d_ff + n]
+// Tile modes:
+//   kModeDense       one GEMM; tiles rasterised in groups of `raster` M-blocks
+//   kModeRowGrouped  the rows are group-major padded segments (group-sparse path): M-block mb
+//                    belongs to group tile_group[mb] (-1: unused, skipped), whose B tile sits
+//                    at n + g*grp_b_n, k + g*grp_b_k
+//   kModeKGrouped    one small GEMM per group g over the rows [seg_start[g], +seg_rows[g]) of
+//                    the group-major buffers (weight gradients of the group-sparse path)
+//
+// Epilogues (flash-swiglu-mlp overview; parameter-golf PR 1105 "Fused MLP Kernels";
+// eugen_sparse README "What it does" and "Pitfalls and limitations"):
+//   kEpiStore      C -> bf16, row m < row_split to out0 else out1 (two weight-gradient halves)
+//   kEpiSwiGLU     gate|up dual tile: h = SiLU(g)*u, a = u*SiLU'(g), b = SiLU(g) -> bf16
+//   kEpiSwiGLUInf  same, h only
+//   kEpiDGate      C = dH: dG = dH*a -> out0[:, n], dU = dH*b -> out0[:, d_ff + n]; columns
+//                  [N, pad_cols) of both halves are written as zeros
+//   kEpiEnergy     per group of energy_p columns: sum |SiLU(C)| (+ bias[g]) -> fp32 out0
+//   kEpiScatterAdd fp32 C row r added (red.global.add) into acc32[row_token[r], :]
+//   kEpiGroupDWgu  per-group [dG|dU]^T X: rows [0,G) -> out0 rows g*G.., [64,64+G) -> out1
+//   kEpiGroupDWd   per-group dY^T h: columns [0,G) -> out0[:, g*G ..]
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -24,7 +38,17 @@
 
 namespace swf {
 
-enum : int { kEpiStore = 0, kEpiSwiGLU = 1, kEpiSwiGLUInf = 2, kEpiDGate = 3 };
+enum : int {
+  kEpiStore = 0,
+  kEpiSwiGLU = 1,
+  kEpiSwiGLUInf = 2,
+  kEpiDGate = 3,
+  kEpiEnergy = 4,
+  kEpiScatterAdd = 5,
+  kEpiGroupDWgu = 6,
+  kEpiGroupDWd = 7
+};
+enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
 
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;  // one 128-byte swizzle row of bf16
@@ -32,8 +56,8 @@ constexpr int kUmmaK = 16;
 constexpr int kGemmThreads = 192;
 
 struct TcGemmArgs {
-  int M;            // rows of C
-  int N;            // columns of C that exist (kEpiSwiGLU*: d_ff)
+  int M;            // rows of C (kModeKGrouped: rows of each group's C)
+  int N;            // columns of C that exist (kEpiSwiGLU*: d_ff; sparse: group_size)
   int num_m_blk, num_n_blk;
   int raster;       // m-blocks per raster group
   int kb_seg0;      // 64-wide k-blocks in K segment 0
@@ -48,16 +72,29 @@ struct TcGemmArgs {
   const void* aux1; // kEpiSwiGLU: saved_b out; kEpiDGate: saved_b in
   int64_t ld_aux;
   int d_ff;         // kEpiDGate: column offset of dU in out0
-  int* status;      // device status word
+  int pad_cols;     // kEpiDGate: zero-filled columns up to here
+  // group-sparse modes
+  const int* tile_group;  // kModeRowGrouped
+  const int* seg_start;   // kModeKGrouped: first padded row of each group
+  const int* seg_rows;    // kModeKGrouped: padded rows of each group (multiple of 128)
+  int grp_b_n, grp_b_k;   // kModeRowGrouped: B coordinate offsets per group
+  int group_size;
+  const int* row_token;   // kEpiScatterAdd: token of each padded row (-1: padding)
+  float* acc32;           // kEpiScatterAdd destination [tokens, N]
+  int64_t ld_acc;
+  const float* bias;      // kEpiEnergy (nullable)
+  int energy_p;           // kEpiEnergy: columns per group
+  int n_groups;           // kEpiEnergy: groups (columns of out0)
+  int* status;            // device status word
   uint64_t wait_limit_ns;
 };
 
 template <int BN>
 struct TcSmem {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr int kABytes = kTileM * kTileK * 2;
   static constexpr int kBBytes = BN * kTileK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kTileBytes = kStages * kStageBytes;
   static constexpr int kBarOffset = kTileBytes;
   static constexpr int kBytes = kTileBytes + 256 + 1024;  // barriers + alignment slack
@@ -74,19 +111,78 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   nb = r / gm;
 }
 
+// What one tile computes: output block (mb, nb), group (-1: skip), TMA coordinates of its first
+// k-block, and its number of k-blocks.
+struct Tile {
+  int mb, nb, grp;
+  int a_m, a_k, b_n, b_k;
+  int kb;
+};
+
+template <int BN, bool B_DUAL, int MODE>
+__device__ __forceinline__ Tile decode_tile(int tile, const TcGemmArgs& a) {
+  Tile t;
+  if constexpr (MODE == kModeKGrouped) {
+    const int per = a.num_m_blk * a.num_n_blk;
+    t.grp = tile / per;
+    const int r = tile - t.grp * per;
+    t.mb = r % a.num_m_blk;
+    t.nb = r / a.num_m_blk;
+    const int s0 = a.seg_start[t.grp];
+    t.a_m = t.mb * kTileM;
+    t.a_k = s0;
+    t.b_n = t.nb * BN;
+    t.b_k = s0;
+    t.kb = a.seg_rows[t.grp] / kTileK;
+  } else {
+    tile_coords(tile, a.num_m_blk, a.num_n_blk, a.raster, t.mb, t.nb);
+    t.grp = MODE == kModeRowGrouped ? a.tile_group[t.mb] : 0;
+    const int g = t.grp < 0 ? 0 : t.grp;
+    t.a_m = t.mb * kTileM;
+    t.a_k = 0;
+    t.b_n = t.nb * (B_DUAL ? BN / 2 : BN) + g * a.grp_b_n;
+    t.b_k = g * a.grp_b_k;
+    t.kb = a.kb_total;
+  }
+  return t;
+}
+
 // 16-byte vector store of 8 bf16 values held as 4 packed words.
 __device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
 }
 
-template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// CW consecutive fp32 columns of this thread's TMEM lane (CW = 16 or 32).
+template <int CW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[32]) {
+  if constexpr (CW == 32) {
+    tmem_ld32(taddr, v);
+  } else {
+    tmem_ld16(taddr, v);
+  }
+}
+
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float* v) {
+  st_v4(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+        pack_bf16x2(v[6], v[7]));
+}
+
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const TcGemmArgs args) {
   using L = TcSmem<BN>;
   constexpr int S = L::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
-  constexpr int kTmemCols = 2 * BN;  // two accumulators
+  constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-column boxes");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -101,7 +197,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_tiles = args.num_m_blk * args.num_n_blk;
+  const int num_tiles = MODE == kModeKGrouped ? args.num_m_blk * args.num_n_blk * args.n_groups
+                                              : args.num_m_blk * args.num_n_blk;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -136,9 +233,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, args.num_m_blk, args.num_n_blk, args.raster, mb, nb);
-        for (int kb = 0; kb < args.kb_total; ++kb, ++it) {
+        const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+        if (t.grp < 0) continue;
+        for (int kb = 0; kb < t.kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) { ok = false; break; }
@@ -147,23 +244,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full[s], L::kStageBytes);
           const bool seg1 = kb >= args.kb_seg0;
           const int kk = (seg1 ? kb - args.kb_seg0 : kb) * kTileK;  // K inside the segment
-          const int ka = seg1 ? args.a_koff1 + kk : kk;
+          const int ka = t.a_k + (seg1 ? args.a_koff1 + kk : kk);
           if (A_MN) {
-            tma_load_2d(sA, &tmA, mb * kTileM, ka, &full[s]);
-            tma_load_2d(sA + 8192, &tmA, mb * kTileM + 64, ka, &full[s]);
+            tma_load_2d(sA, &tmA, t.a_m, ka, &full[s]);
+            tma_load_2d(sA + 8192, &tmA, t.a_m + 64, ka, &full[s]);
           } else {
-            tma_load_2d(sA, &tmA, ka, mb * kTileM, &full[s]);
+            tma_load_2d(sA, &tmA, ka, t.a_m, &full[s]);
           }
           const CUtensorMap* mapB = seg1 ? &tmB1 : &tmB0;
           if (B_DUAL) {
-            tma_load_2d(sB, &tmB0, kk, nb * (BN / 2), &full[s]);
-            tma_load_2d(sB + (BN / 2) * 128, &tmB1, kk, nb * (BN / 2), &full[s]);
+            tma_load_2d(sB, &tmB0, t.b_k + kk, t.b_n, &full[s]);
+            tma_load_2d(sB + (BN / 2) * 128, &tmB1, t.b_k + kk, t.b_n, &full[s]);
           } else if (B_MN) {
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sB + j * 8192, mapB, nb * BN + j * 64, kk, &full[s]);
+              tma_load_2d(sB + j * 8192, mapB, t.b_n + j * 64, t.b_k + kk, &full[s]);
           } else {
-            tma_load_2d(sB, mapB, kk, nb * BN, &full[s]);
+            tma_load_2d(sB, mapB, t.b_k + kk, t.b_n, &full[s]);
           }
         }
       }
@@ -183,13 +280,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int local = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+        if (t.grp < 0) continue;
         const int buf = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
+        ++local;
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
-        for (int kb = 0; kb < args.kb_total; ++kb, ++it) {
+        for (int kb = 0; kb < t.kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&full[s], ph, ctl)) { ok = false; break; }
@@ -208,7 +308,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           issued = true;
         }
         if (!ok) break;
-        if (args.kb_total > 0) umma_commit(&tfull[buf]);
+        if (t.kb > 0) umma_commit(&tfull[buf]);
         else mbar_arrive(&tfull[buf]);
       }
       if (!ok && issued) {
@@ -224,33 +324,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      int mb, nb;
-      tile_coords(tile, args.num_m_blk, args.num_n_blk, args.raster, mb, nb);
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+      if (t.grp < 0) continue;
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
+      ++local;
       const bool ready = mbar_wait(&tfull[buf], use & 1u, ctl);
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
-      const bool have_acc = args.kb_total > 0;
-      const int m = mb * kTileM + row;
+      const bool have_acc = t.kb > 0;
+      const int m = t.a_m + row;
       const bool row_ok = m < args.M;
 
       if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
+        constexpr int CW = BN / 2 < 32 ? BN / 2 : 32;
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
+        for (int c = 0; c < BN / 2; c += CW) {
           float g[32], u[32];
           if (have_acc) {
-            tmem_ld32(t_acc + c, g);
-            tmem_ld32(t_acc + BN / 2 + c, u);
+            tmem_ld_cols<CW>(t_acc + c, g);
+            tmem_ld_cols<CW>(t_acc + BN / 2 + c, u);
             tmem_ld_wait();
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
           }
-          const int n0 = nb * (BN / 2) + c;
+          const int n0 = t.nb * (BN / 2) + c;
           if (row_ok) {
             __nv_bfloat16* hp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
             __nv_bfloat16* ap = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux0)) +
@@ -258,34 +360,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             __nv_bfloat16* bp = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux1)) +
                                 (int64_t)m * args.ld_aux + n0;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
+            for (int v = 0; v < CW / 8; ++v) {
               if (n0 + v * 8 + 8 <= args.N) {
-                uint32_t hw[4], aw[4], bw[4];
+                float hv[8], av[8], bv[8];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                  float hv[2], av[2], bv[2];
-#pragma unroll
-                  for (int e = 0; e < 2; ++e) {
-                    const int j = v * 8 + p * 2 + e;
-                    const float s = sigmoidf_(g[j]);
-                    bv[e] = g[j] * s;
-                    hv[e] = bv[e] * u[j];
-                    av[e] = u[j] * s * (1.f + g[j] * (1.f - s));
-                  }
-                  hw[p] = pack_bf16x2(hv[0], hv[1]);
-                  aw[p] = pack_bf16x2(av[0], av[1]);
-                  bw[p] = pack_bf16x2(bv[0], bv[1]);
+                for (int e = 0; e < 8; ++e) {
+                  const int j = v * 8 + e;
+                  const float s = sigmoidf_(g[j]);
+                  bv[e] = g[j] * s;
+                  hv[e] = bv[e] * u[j];
+                  av[e] = u[j] * s * (1.f + g[j] * (1.f - s));
                 }
-                st_v4(hp + v * 8, hw[0], hw[1], hw[2], hw[3]);
+                store_bf16x8(hp + v * 8, hv);
                 if constexpr (EPI == kEpiSwiGLU) {
-                  st_v4(ap + v * 8, aw[0], aw[1], aw[2], aw[3]);
-                  st_v4(bp + v * 8, bw[0], bw[1], bw[2], bw[3]);
+                  store_bf16x8(ap + v * 8, av);
+                  store_bf16x8(bp + v * 8, bv);
                 }
               }
             }
           }
         }
       } else {
+        float run = 0.f;  // kEpiEnergy: running sum of the current group
+        static_assert(EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf || BN % 32 == 0, "chunking");
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float acc[32];
@@ -296,7 +393,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] = 0.f;
           }
-          const int n0 = nb * BN + c;
+          const int n0 = t.nb * BN + c;
           if (!row_ok) continue;
           if constexpr (EPI == kEpiStore) {
             __nv_bfloat16* op =
@@ -305,14 +402,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     : static_cast<__nv_bfloat16*>(args.out1) +
                           (int64_t)(m - args.row_split) * args.ld_out + n0;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (n0 + v * 8 + 8 <= args.N) {
-                st_v4(op + v * 8, pack_bf16x2(acc[v * 8 + 0], acc[v * 8 + 1]),
-                      pack_bf16x2(acc[v * 8 + 2], acc[v * 8 + 3]),
-                      pack_bf16x2(acc[v * 8 + 4], acc[v * 8 + 5]),
-                      pack_bf16x2(acc[v * 8 + 6], acc[v * 8 + 7]));
-              }
-            }
+            for (int v = 0; v < 4; ++v)
+              if (n0 + v * 8 + 8 <= args.N) store_bf16x8(op + v * 8, acc + v * 8);
           } else if constexpr (EPI == kEpiDGate) {
             const __nv_bfloat16* ap =
                 static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
@@ -336,8 +427,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 st_v4(gp + v * 8, gw[0], gw[1], gw[2], gw[3]);
                 st_v4(up + v * 8, uw[0], uw[1], uw[2], uw[3]);
+              } else if (n0 + v * 8 < args.pad_cols) {
+                st_v4(gp + v * 8, 0u, 0u, 0u, 0u);
+                st_v4(up + v * 8, 0u, 0u, 0u, 0u);
               }
             }
+          } else if constexpr (EPI == kEpiEnergy) {
+            float* ep = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
+            const int pm = args.energy_p - 1;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float z = acc[j];
+              run += fabsf(z * sigmoidf_(z));
+              const int n = n0 + j;
+              if ((n & pm) == pm) {
+                const int grp = n / args.energy_p;
+                if (grp < args.n_groups) ep[grp] = run + (args.bias ? args.bias[grp] : 0.f);
+                run = 0.f;
+              }
+            }
+          } else if constexpr (EPI == kEpiScatterAdd) {
+            const int tok = args.row_token[m];
+            if (tok >= 0) {
+              float* dst = args.acc32 + (int64_t)tok * args.ld_acc + n0;
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                if (n0 + v * 4 + 4 <= args.N)
+                  red_add_v4(dst + v * 4, acc[v * 4], acc[v * 4 + 1], acc[v * 4 + 2], acc[v * 4 + 3]);
+            }
+          } else if constexpr (EPI == kEpiGroupDWgu) {
+            const int G = args.group_size;
+            __nv_bfloat16* op = nullptr;
+            if (m < G)
+              op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)(t.grp * G + m) * args.ld_out + n0;
+            else if (m >= 64 && m < 64 + G)
+              op = static_cast<__nv_bfloat16*>(args.out1) +
+                   (int64_t)(t.grp * G + m - 64) * args.ld_out + n0;
+            if (op) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                if (n0 + v * 8 + 8 <= args.N) store_bf16x8(op + v * 8, acc + v * 8);
+            }
+          } else if constexpr (EPI == kEpiGroupDWd) {
+            const int G = args.group_size;
+            __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out +
+                                t.grp * G + n0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              if (n0 + v * 8 + 8 <= G) store_bf16x8(op + v * 8, acc + v * 8);
           }
         }
       }
