@@ -173,8 +173,10 @@ swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t num_ac
 
 /* Sparse forward (eugen_sparse README, sparse_swiglu_ffn):
  *   y[t] = sum over c in group_idx[t] of (SiLU(x_t W_gate[c]^T) * x_t W_up[c]^T) W_down[:, c]^T
- * with W_*[c] the group's G rows.  y is accumulated in fp32 (fp32 atomics, as the README
- * describes; the summation order may vary between runs) and written in `dtype`.  `saved`
+ * with W_*[c] the group's G rows.  Each (token, group) contribution is computed in fp32 and
+ * stored in `dtype`; a token's contributions are then summed in fp32 in the order of its
+ * group_idx slots, so y is bitwise deterministic (the README's kernel uses fp32 atomics
+ * instead).  `saved`
  * (swf_sparse_saved_bytes bytes) receives what the backward needs: the bucketing and the
  * compact per-pair h, a, b; the caller keeps it for sparse_swiglu_ffn_bwd. */
 swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, const void* w_up,
@@ -187,7 +189,7 @@ swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, const void* 
 /* Sparse backward: gradients to x and all three weights of L = sum(dy * y) for the forward
  * above.  Only selected groups get weight gradients; rows (dw_gate, dw_up) and columns
  * (dw_down) of groups no token selected are written as exact zeros (eugen_sparse README,
- * "Hard selection").  dx accumulates in fp32 (atomics); weight gradients are deterministic. */
+ * "Hard selection").  dx is reduced like y in the forward; every output is deterministic. */
 swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate,
                                  const void* w_up, const void* w_down, const int32_t* group_idx,
                                  const void* saved, size_t saved_bytes, void* dx, void* dw_gate,
@@ -244,12 +246,13 @@ typedef enum swf_kernel_kind {
   SWF_K_BUCKETS = 11,      /* group bucketing (count, scan, place) */
   SWF_K_SPARSE_GATHER = 12,/* gather of token rows into group-major order */
   SWF_K_SPARSE_UP = 13,    /* sparse gate|up GEMM with the SwiGLU epilogue */
-  SWF_K_SPARSE_DOWN = 14,  /* sparse down GEMM with scatter-add into fp32 */
+  SWF_K_SPARSE_DOWN = 14,  /* sparse down GEMM: per-pair contributions to y */
   SWF_K_SPARSE_DGATE = 15, /* sparse dH GEMM with the gating epilogue */
-  SWF_K_SPARSE_DX = 16,    /* sparse dx GEMM with scatter-add into fp32 */
+  SWF_K_SPARSE_DX = 16,    /* sparse dx GEMM: per-pair contributions to dx */
   SWF_K_SPARSE_DW = 17,    /* sparse weight-gradient GEMMs */
-  SWF_K_ELEMENTWISE = 18,  /* zero fill, fp32 -> output dtype conversion */
-  SWF_K_NUM_KINDS = 19
+  SWF_K_ELEMENTWISE = 18,  /* fills */
+  SWF_K_PAIR_SUM = 19,     /* per-token sum of the per-pair contributions (y, dx) */
+  SWF_K_NUM_KINDS = 20
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

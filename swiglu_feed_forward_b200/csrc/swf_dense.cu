@@ -17,8 +17,9 @@ namespace swf {
 
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f) {
   auto t = [](int64_t m, int64_t n, int64_t bn) { return (int64_t)cdiv(m, kTileM) * cdiv(n, bn); };
-  if (op == SWF_OP_FWD || op == SWF_OP_FWD_INFER) return t(M, f, 128) + t(M, d, 256);
-  if (op == SWF_OP_BWD) return t(M, f, 256) + t(M, d, 256) + t(2 * f, d, 256) + t(d, f, 256);
+  // pair-mode tiles of 256 rows
+  if (op == SWF_OP_FWD || op == SWF_OP_FWD_INFER) return (t(M, f, 128) + t(M, d, 256) + 1) / 2;
+  if (op == SWF_OP_BWD) return (t(M, f, 256) + t(M, d, 256) + t(2 * f, d, 256) + t(d, f, 256) + 1) / 2;
   return 0;
 }
 
@@ -28,23 +29,24 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
   CUtensorMap tx, twg, twu, th, twd;
   if (!encode_tmap_bf16(&tx, x, d, M, d, 64, 128) || !encode_tmap_bf16(&twg, wg, d, f, d, 64, 128) ||
       !encode_tmap_bf16(&twu, wu, d, f, d, 64, 128) || !encode_tmap_bf16(&th, h, f, M, f, 64, 128) ||
-      !encode_tmap_bf16(&twd, wd, f, d, f, 64, 256))
+      !encode_tmap_bf16(&twd, wd, f, d, f, 64, 128))
     return SWF_ERR_LAUNCH;
   // K1: gate|up dual tile, 128 columns of each per tile
-  TcGemmArgs k1 = base_args(M, f, 128, d);
+  TcGemmArgs k1 = base_args(M, f, 128, d, 2 * kTileM);
   k1.out0 = h;
   k1.ld_out = f;
   k1.aux0 = a;
   k1.aux1 = b;
   k1.ld_aux = f;
-  swf_status s = infer ? launch_tc<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, k1, st)
-                       : launch_tc<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, k1, st);
+  swf_status s =
+      infer ? launch_tc_pair<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, k1, st)
+            : launch_tc_pair<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, k1, st);
   if (s != SWF_OK) return s;
   // K2: y = h W_d^T
-  TcGemmArgs k2 = base_args(M, d, 256, f);
+  TcGemmArgs k2 = base_args(M, d, 256, f, 2 * kTileM);
   k2.out0 = y;
   k2.ld_out = d;
-  return launch_tc<256, false, false, false, kEpiStore>(SWF_K_DOWN, th, twd, twd, k2, st);
+  return launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_DOWN, th, twd, twd, k2, st);
 }
 
 swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
@@ -56,14 +58,14 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     CUtensorMap tdy, twd;
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k3 = base_args(M, f, 256, d);
+    TcGemmArgs k3 = base_args(M, f, 256, d, 2 * kTileM);
     k3.out0 = dgu;
     k3.ld_out = 2 * f;
     k3.aux0 = a;
     k3.aux1 = b;
     k3.ld_aux = f;
     k3.d_ff = (int)f;
-    s = launch_tc<256, false, true, false, kEpiDGate>(SWF_K_DGATE, tdy, twd, twd, k3, st);
+    s = launch_tc_pair<256, false, true, false, kEpiDGate>(SWF_K_DGATE, tdy, twd, twd, k3, st);
     if (s != SWF_OK) return s;
   }
   {  // K4: dx = dG W_g + dU W_u: A = dGU (K-major, K = 2f), B segments W_g / W_u (MN-major)
@@ -71,35 +73,35 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     if (!encode_tmap_bf16(&tdgu, dgu, 2 * f, M, 2 * f, 64, 128) ||
         !encode_tmap_bf16(&twg, wg, d, f, d, 64, 64) || !encode_tmap_bf16(&twu, wu, d, f, d, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k4 = base_args(M, d, 256, 0);
+    TcGemmArgs k4 = base_args(M, d, 256, 0, 2 * kTileM);
     k4.kb_seg0 = cdiv(f, kTileK);
     k4.kb_total = 2 * k4.kb_seg0;
     k4.a_koff1 = (int)f;
     k4.out0 = dx;
     k4.ld_out = d;
-    s = launch_tc<256, false, true, false, kEpiStore>(SWF_K_DX, tdgu, twg, twu, k4, st);
+    s = launch_tc_pair<256, false, true, false, kEpiStore>(SWF_K_DX, tdgu, twg, twu, k4, st);
     if (s != SWF_OK) return s;
   }
   {  // K5: [dW_g ; dW_u] = dGU^T x: A = dGU viewed [K=M rows, 2f cols] (MN-major), B = x (MN)
     CUtensorMap tdgu, tx;
     if (!encode_tmap_bf16(&tdgu, dgu, 2 * f, M, 2 * f, 64, 64) || !encode_tmap_bf16(&tx, x, d, M, d, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k5 = base_args(2 * f, d, 256, M);
+    TcGemmArgs k5 = base_args(2 * f, d, 256, M, 2 * kTileM);
     k5.out0 = dwg;
     k5.out1 = dwu;
     k5.row_split = (int)f;
     k5.ld_out = d;
-    s = launch_tc<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, k5, st);
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, k5, st);
     if (s != SWF_OK) return s;
   }
   {  // K6: dW_d = dY^T h: A = dY viewed [K=M rows, d cols] (MN), B = h [K=M rows, f cols] (MN)
     CUtensorMap tdy, th;
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 64) || !encode_tmap_bf16(&th, h, f, M, f, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k6 = base_args(d, f, 256, M);
+    TcGemmArgs k6 = base_args(d, f, 256, M, 2 * kTileM);
     k6.out0 = dwd;
     k6.ld_out = f;
-    s = launch_tc<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, k6, st);
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, k6, st);
   }
   return s;
 }

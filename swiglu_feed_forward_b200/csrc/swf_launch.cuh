@@ -33,12 +33,49 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 
-// Arguments of a dense GEMM of M x N (N-blocks of n_blk_cols columns) over K.
-inline TcGemmArgs base_args(int64_t M, int64_t N, int n_blk_cols, int64_t K) {
+// Launches the pair-mode (cta_group::2) dense GEMM as clusters of two CTAs: min(tiles, SMs / 2)
+// clusters, each walking 256 x BN tiles.
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
+swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
+                          const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
+  DevCtx ctx;
+  swf_status s = get_ctx(&ctx);
+  if (s != SWF_OK) return s;
+  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk;
+  if (tiles == 0) return SWF_OK;
+  if (tiles > INT32_MAX) return SWF_ERR_UNSUPPORTED;
+  args.status = ctx.status;
+  if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
+  args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, kModeDense, true>;
+  constexpr int smem = TcSmem<BN, true>::kBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  const int clusters = (int)std::min<int64_t>(tiles, ctx.num_sms / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfScope prof(kind, st);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb0, tb1, args) != cudaSuccess) return SWF_ERR_LAUNCH;
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
+// Arguments of a dense GEMM of M x N (N-blocks of n_blk_cols columns) over K, with M-blocks of
+// m_tile rows (256 in pair mode).
+inline TcGemmArgs base_args(int64_t M, int64_t N, int n_blk_cols, int64_t K, int m_tile = kTileM) {
   TcGemmArgs a{};
   a.M = (int)M;
   a.N = (int)N;
-  a.num_m_blk = cdiv(M, kTileM);
+  a.num_m_blk = cdiv(M, m_tile);
   a.num_n_blk = cdiv(N, n_blk_cols);
   a.raster = 8;
   a.kb_total = cdiv(K, kTileK);

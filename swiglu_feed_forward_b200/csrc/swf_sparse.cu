@@ -38,7 +38,9 @@ SparseDims dims_of(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
   s.pairs = M * K;
   s.rmax = (int64_t)round_up((size_t)(s.pairs + (int64_t)s.ng * 127), 128);
   s.mblk = (int)(s.rmax / 128);
-  s.words = std::max(1, std::min(32, kBucketSmemBytes / (8 * std::max(1, s.ng))));
+  const int words_smem = std::max(1, std::min(32, kBucketSmemBytes / (8 * std::max(1, s.ng))));
+  const int64_t words_fill = (M + 32 * 296 - 1) / (32 * 296);  // about two blocks per SM
+  s.words = (int)std::max<int64_t>(1, std::min<int64_t>(words_smem, words_fill));
   s.tok_blk = 32 * s.words;
   s.nblk = (int)((M + s.tok_blk - 1) / s.tok_blk);
   return s;
@@ -57,7 +59,7 @@ struct Carver {
 };
 
 struct SavedView {
-  int32_t *offs, *tokens, *seg_start, *seg_rows, *tile_group, *row_token;
+  int32_t *offs, *tokens, *seg_start, *seg_rows, *tile_group, *row_token, *pair_row;
   __nv_bfloat16 *h, *a, *b;
 };
 
@@ -70,6 +72,7 @@ SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
   v.seg_rows = c.take<int32_t>(s.ng);
   v.tile_group = c.take<int32_t>(s.mblk);
   v.row_token = c.take<int32_t>(s.rmax);
+  v.pair_row = c.take<int32_t>(s.pairs);
   v.h = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.a = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.b = c.take<__nv_bfloat16>(s.rmax * s.G);
@@ -80,21 +83,21 @@ SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
 struct FwdWs {
   int32_t* counts;
   __nv_bfloat16* xc;
-  float* y32;
+  __nv_bfloat16* yc;  // per-pair contributions to y, group-major rows
 };
 FwdWs fwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   Carver c{static_cast<char*>(base)};
   FwdWs w;
   w.counts = c.take<int32_t>((size_t)s.nblk * s.ng);
   w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
-  w.y32 = c.take<float>(s.M * s.d);
+  w.yc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
   return w;
 }
 
 struct BwdWs {
   __nv_bfloat16 *xc, *dyc, *dgu;
-  float* dx32;
+  __nv_bfloat16* dxc;  // per-pair contributions to dx, group-major rows
 };
 BwdWs bwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   Carver c{static_cast<char*>(base)};
@@ -102,7 +105,7 @@ BwdWs bwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.dyc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.dgu = c.take<__nv_bfloat16>(s.rmax * 128);
-  w.dx32 = c.take<float>(s.M * s.d);
+  w.dxc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
   return w;
 }
@@ -154,11 +157,12 @@ __global__ void bucket_count_kernel(const int32_t* __restrict__ idx, int64_t M, 
     if (valid_slot(row, k, ng)) atomicAdd(&hist[row[k]], 1);
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < ng; c += blockDim.x) counts[(int64_t)blockIdx.x * ng + c] = hist[c];
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) counts[(int64_t)c * gridDim.x + blockIdx.x] = hist[c];
 }
 
-// One block: turns per-block counts into exclusive per-block bases, writes the CSR offsets
-// and, when seg_start is given, the padded segments and the tile -> group table.
+// One block: turns the per-block counts (group-major, [ng][nblk]) into exclusive per-block
+// bases with one warp-wide scan per group, writes the CSR offsets and, when seg_start is given,
+// the padded segments and the tile -> group table.
 __global__ void bucket_scan_kernel(int32_t* __restrict__ counts, int nblk, int ng,
                                    int32_t* __restrict__ offs, int32_t* __restrict__ seg_start,
                                    int32_t* __restrict__ seg_rows, int32_t* __restrict__ tile_group,
@@ -166,26 +170,52 @@ __global__ void bucket_scan_kernel(int32_t* __restrict__ counts, int nblk, int n
   extern __shared__ int32_t sh[];
   int32_t* tot = sh;            // [ng]
   int32_t* sstart = sh + ng;    // [ng + 1]
-  for (int c = threadIdx.x; c < ng; c += blockDim.x) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int c = warp; c < ng; c += nwarps) {
+    int32_t* row = counts + (int64_t)c * nblk;
     int32_t run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int32_t v = counts[(int64_t)b * ng + c];
-      counts[(int64_t)b * ng + c] = run;
-      run += v;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int b = b0 + lane;
+      const int32_t v = b < nblk ? row[b] : 0;
+      int32_t incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      if (b < nblk) row[b] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    tot[c] = run;
+    if (lane == 0) tot[c] = run;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     int32_t o = 0, p = 0;
-    for (int c = 0; c < ng; ++c) {
-      offs[c] = o;
-      sstart[c] = p;
-      o += tot[c];
-      p += (tot[c] + 127) / 128 * 128;
+    for (int c0 = 0; c0 < ng; c0 += 32) {
+      const int c = c0 + lane;
+      const int32_t t = c < ng ? tot[c] : 0;
+      const int32_t pt = (t + 127) / 128 * 128;
+      int32_t it = t, ip = pt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t n1 = __shfl_up_sync(0xffffffffu, it, off);
+        const int32_t n2 = __shfl_up_sync(0xffffffffu, ip, off);
+        if (lane >= off) {
+          it += n1;
+          ip += n2;
+        }
+      }
+      if (c < ng) {
+        offs[c] = o + it - t;
+        sstart[c] = p + ip - pt;
+      }
+      o += __shfl_sync(0xffffffffu, it, 31);
+      p += __shfl_sync(0xffffffffu, ip, 31);
     }
-    offs[ng] = o;
-    sstart[ng] = p;
+    if (lane == 0) {
+      offs[ng] = o;
+      sstart[ng] = p;
+    }
   }
   __syncthreads();
   if (seg_start == nullptr) return;
@@ -215,7 +245,8 @@ __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, 
                                     int words, const int32_t* __restrict__ counts,
                                     const int32_t* __restrict__ offs, int32_t* __restrict__ tokens,
                                     const int32_t* __restrict__ seg_start,
-                                    int32_t* __restrict__ row_token) {
+                                    int32_t* __restrict__ row_token,
+                                    int32_t* __restrict__ pair_row) {
   extern __shared__ uint32_t smem_bits[];
   uint32_t* bits = smem_bits;                                        // [ng][words]
   int32_t* pre = reinterpret_cast<int32_t*>(smem_bits + (size_t)ng * words);  // [ng][words]
@@ -246,13 +277,17 @@ __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, 
     if (t >= M) break;
     const int32_t* row = idx + t * K;
     const int k = i % K;
-    if (!valid_slot(row, k, ng)) continue;
+    if (!valid_slot(row, k, ng)) {
+      if (pair_row) pair_row[t * K + k] = -1;
+      continue;
+    }
     const int c = row[k];
     const int w = tl >> 5;
     const int rank = pre[c * words + w] + __popc(bits[c * words + w] & ((1u << (tl & 31)) - 1u));
-    const int32_t base = counts[(int64_t)blockIdx.x * ng + c] + rank;
+    const int32_t base = counts[(int64_t)c * gridDim.x + blockIdx.x] + rank;
     tokens[offs[c] + base] = (int32_t)t;
     if (row_token) row_token[seg_start[c] + base] = (int32_t)t;
+    if (pair_row) pair_row[t * K + k] = seg_start[c] + base;
   }
 }
 
@@ -261,15 +296,30 @@ __global__ void fill_i32_kernel(int32_t* __restrict__ p, int64_t n, int32_t v) {
     p[i] = v;
 }
 
-__global__ void zero_f32_kernel(float4* __restrict__ p, int64_t n4) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t n4) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 v = src[i];
-    dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+// out[t, :] = sum over t's valid slots k (in slot order) of rows[pair_row[t*K + k], :], fp32
+// accumulation, bf16 result: the deterministic reduction of the per-pair contributions.
+__global__ void pair_sum_kernel(const uint4* __restrict__ rows, const int32_t* __restrict__ pair_row,
+                                int64_t M, int K, int64_t row_vecs, uint4* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < M; t += warps) {
+    const int32_t* pr = pair_row + t * K;
+    for (int64_t v = lane; v < row_vecs; v += 32) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int k = 0; k < K; ++k) {
+        const int32_t r = pr[k];
+        if (r < 0) continue;
+        const uint4 q = rows[(int64_t)r * row_vecs + v];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += bf16_lo(w[i]);
+          acc[2 * i + 1] += bf16_hi(w[i]);
+        }
+      }
+      out[t * row_vecs + v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
   }
 }
 
@@ -380,7 +430,7 @@ swf_status launched() { return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_
 
 swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts, int32_t* offs,
                        int32_t* tokens, int32_t* seg_start, int32_t* seg_rows,
-                       int32_t* tile_group, int32_t* row_token, cudaStream_t st) {
+                       int32_t* tile_group, int32_t* row_token, int32_t* pair_row, cudaStream_t st) {
   {
     ProfScope prof(SWF_K_BUCKETS, st);
     bucket_count_kernel<<<s.nblk, 256, s.ng * sizeof(int32_t), st>>>(idx, s.M, s.K, s.ng, s.tok_blk, counts);
@@ -406,7 +456,7 @@ swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts,
     return SWF_ERR_LAUNCH;
   ProfScope prof(SWF_K_BUCKETS, st);
   bucket_place_kernel<<<s.nblk, 256, place_smem, st>>>(idx, s.M, s.K, s.ng, s.words, counts, offs,
-                                                       tokens, seg_start, row_token);
+                                                       tokens, seg_start, row_token, pair_row);
   return launched();
 }
 
@@ -418,16 +468,11 @@ swf_status run_gather(const void* src, const SavedView& v, const SparseDims& s, 
   return launched();
 }
 
-swf_status run_zero(float* p, int64_t n, cudaStream_t st) {
-  ProfScope prof(SWF_K_ELEMENTWISE, st);
-  zero_f32_kernel<<<grid_for(n / 4, 256), 256, 0, st>>>(reinterpret_cast<float4*>(p), n / 4);
-  return launched();
-}
-
-swf_status run_convert(const float* src, void* dst, int64_t n, cudaStream_t st) {
-  ProfScope prof(SWF_K_ELEMENTWISE, st);
-  f32_to_bf16_kernel<<<grid_for(n / 4, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(src),
-                                                           static_cast<uint2*>(dst), n / 4);
+swf_status run_pair_sum(const void* rows, const int32_t* pair_row, const SparseDims& s, void* out,
+                        cudaStream_t st) {
+  ProfScope prof(SWF_K_PAIR_SUM, st);
+  pair_sum_kernel<<<grid_for(s.M, 8), 256, 0, st>>>(static_cast<const uint4*>(rows), pair_row, s.M, s.K,
+                                                   s.d / 8, static_cast<uint4*>(out));
   return launched();
 }
 
@@ -479,7 +524,7 @@ size_t sparse_saved_bytes(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K)
 void sparse_plan(int op, int64_t M, int64_t d, int64_t f, int32_t G, int32_t K, int32_t spg,
                  swf_plan_info* p) {
   const SparseDims s = dims_of(M, d, f, G, K);
-  p->deterministic = (op == SWF_OP_SELECT || op == SWF_OP_BUCKETS) ? 1 : 0;
+  p->deterministic = 1;
   p->saved_bytes = (op == SWF_OP_SPARSE_FWD || op == SWF_OP_SPARSE_BWD) ? sparse_saved_bytes(M, d, f, G, K) : 0;
   const int P = spg > 0 ? pow2_at_least(spg) : G;
   switch (op) {
@@ -614,7 +659,7 @@ extern "C" swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int
   if (ws_bytes < buckets_workspace_bytes(M, K, ng)) return SWF_ERR_WORKSPACE;
   const SparseDims d = dims_of(M, 16, (int64_t)ng * 16, 16, K);
   return run_buckets(group_idx, d, static_cast<int32_t*>(workspace), offsets, tokens, nullptr,
-                     nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+                     nullptr, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------ sparse forward
@@ -647,7 +692,7 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   if ((s = run_buckets(group_idx, sd, w.counts, v.offs, v.tokens, v.seg_start, v.seg_rows,
-                       v.tile_group, v.row_token, st)) != SWF_OK)
+                       v.tile_group, v.row_token, v.pair_row, st)) != SWF_OK)
     return s;
   if ((s = run_gather(x, v, sd, w.xc, st)) != SWF_OK) return s;
 
@@ -670,21 +715,19 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     else s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
     if (s != SWF_OK) return s;
   }
-  if ((s = run_zero(w.y32, M * d, st)) != SWF_OK) return s;
-  {  // down per group: y32[token] += h_row W_d[:, g*G .. g*G+G]^T
+  {  // down per group: yc[r] = h_row W_d[:, g*G .. g*G+G]^T
     CUtensorMap th, twd;
     if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 256))
       return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, d, 256, G);
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
-    a.row_token = v.row_token;
-    a.acc32 = w.y32;
-    a.ld_acc = d;
-    s = launch_tc<256, false, false, false, kEpiScatterAdd, kModeRowGrouped>(SWF_K_SPARSE_DOWN, th, twd, twd, a, st);
+    a.out0 = w.yc;
+    a.ld_out = d;
+    s = launch_tc<256, false, false, false, kEpiStore, kModeRowGrouped>(SWF_K_SPARSE_DOWN, th, twd, twd, a, st);
     if (s != SWF_OK) return s;
   }
-  return run_convert(w.y32, y, M * d, st);
+  return run_pair_sum(w.yc, v.pair_row, sd, y, st);
 }
 
 // ------------------------------------------------------------------ sparse backward
@@ -728,8 +771,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped>(SWF_K_SPARSE_DGATE, tdyc, twd, twd, a, st);
     if (s != SWF_OK) return s;
   }
-  if ((s = run_zero(w.dx32, M * d, st)) != SWF_OK) return s;
-  {  // dx32[token] += dG_row W_g[g] + dU_row W_u[g]
+  {  // dxc[r] = dG_row W_g[g] + dU_row W_u[g]
     CUtensorMap tdgu, twg, twu;
     if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 128) ||
         !encode_tmap_bf16(&twg, w_gate, d, f, d, 64, 64) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, 64))
@@ -740,13 +782,12 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.a_koff1 = 64;
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
-    a.row_token = v.row_token;
-    a.acc32 = w.dx32;
-    a.ld_acc = d;
-    s = launch_tc<256, false, true, false, kEpiScatterAdd, kModeRowGrouped>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st);
+    a.out0 = w.dxc;
+    a.ld_out = d;
+    s = launch_tc<256, false, true, false, kEpiStore, kModeRowGrouped>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st);
     if (s != SWF_OK) return s;
   }
-  if ((s = run_convert(w.dx32, dx, M * d, st)) != SWF_OK) return s;
+  if ((s = run_pair_sum(w.dxc, v.pair_row, sd, dx, st)) != SWF_OK) return s;
   {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ Xc_seg
     CUtensorMap tdgu, txc;
     if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64) ||

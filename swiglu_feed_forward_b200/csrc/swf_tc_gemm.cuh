@@ -26,7 +26,6 @@
 //   kEpiDGate      C = dH: dG = dH*a -> out0[:, n], dU = dH*b -> out0[:, d_ff + n]; columns
 //                  [N, pad_cols) of both halves are written as zeros
 //   kEpiEnergy     per group of energy_p columns: sum |SiLU(C)| (+ bias[g]) -> fp32 out0
-//   kEpiScatterAdd fp32 C row r added (red.global.add) into acc32[row_token[r], :]
 //   kEpiGroupDWgu  per-group [dG|dU]^T X: rows [0,G) -> out0 rows g*G.., [64,64+G) -> out1
 //   kEpiGroupDWd   per-group dY^T h: columns [0,G) -> out0[:, g*G ..]
 #pragma once
@@ -44,9 +43,8 @@ enum : int {
   kEpiSwiGLUInf = 2,
   kEpiDGate = 3,
   kEpiEnergy = 4,
-  kEpiScatterAdd = 5,
-  kEpiGroupDWgu = 6,
-  kEpiGroupDWd = 7
+  kEpiGroupDWgu = 5,
+  kEpiGroupDWd = 6
 };
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
 
@@ -79,9 +77,6 @@ struct TcGemmArgs {
   const int* seg_rows;    // kModeKGrouped: padded rows of each group (multiple of 128)
   int grp_b_n, grp_b_k;   // kModeRowGrouped: B coordinate offsets per group
   int group_size;
-  const int* row_token;   // kEpiScatterAdd: token of each padded row (-1: padding)
-  float* acc32;           // kEpiScatterAdd destination [tokens, N]
-  int64_t ld_acc;
   const float* bias;      // kEpiEnergy (nullable)
   int energy_p;           // kEpiEnergy: columns per group
   int n_groups;           // kEpiEnergy: groups (columns of out0)
@@ -89,10 +84,13 @@ struct TcGemmArgs {
   uint64_t wait_limit_ns;
 };
 
-template <int BN>
+// Shared-memory plan of one CTA.  In pair mode (cta_group::2) each CTA holds 128 rows of A and
+// BN/2 rows of B; the pair computes a 256 x BN tile.
+template <int BN, bool PAIR = false>
 struct TcSmem {
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;
   static constexpr int kABytes = kTileM * kTileK * 2;
-  static constexpr int kBBytes = BN * kTileK * 2;
+  static constexpr int kBBytes = kBRows * kTileK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kTileBytes = kStages * kStageBytes;
@@ -152,12 +150,6 @@ __device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t 
   *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
 }
 
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
 // CW consecutive fp32 columns of this thread's TMEM lane (CW = 16 or 32).
 template <int CW>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[32]) {
@@ -173,16 +165,23 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float* v) {
         pack_bf16x2(v[6], v[7]));
 }
 
-template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense>
+// PAIR: launched as clusters of 2 CTAs; the even CTA issues tcgen05.mma.cta_group::2 over both
+// CTAs' shared memory, each CTA keeps its 128 rows of the 256 x BN accumulator in its own TMEM
+// and runs its own epilogue.  Both CTAs' TMA loads complete on the even CTA's stage barrier,
+// and the MMA commits arrive on the stage and accumulator barriers of both CTAs.
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense,
+          bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const TcGemmArgs args) {
-  using L = TcSmem<BN>;
+  using L = TcSmem<BN, PAIR>;
   constexpr int S = L::kStages;
-  constexpr uint32_t kIdesc = idesc_bf16(kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+  constexpr uint32_t kIdesc = idesc_bf16(PAIR ? 2 * kTileM : kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
   constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
+  constexpr int kBRows = L::kBRows;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
-  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-column boxes");
+  static_assert(!B_MN || kBRows % 64 == 0, "MN-major B tiles are whole 64-column boxes");
+  static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -199,6 +198,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const int num_tiles = MODE == kModeKGrouped ? args.num_m_blk * args.num_n_blk * args.n_groups
                                               : args.num_m_blk * args.num_n_blk;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], PAIR ? 256 : 128);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -219,10 +221,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (B_DUAL || args.kb_seg0 < args.kb_total) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
@@ -232,35 +240,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+      // pair mode: every stage completes on the even CTA's barrier
+      const uint32_t full_lead = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;
+      for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
+        Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
         if (t.grp < 0) continue;
+        if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
         for (int kb = 0; kb < t.kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) { ok = false; break; }
           uint8_t* sA = smem + s * L::kStageBytes;
           uint8_t* sB = sA + L::kABytes;
-          mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+          if (!PAIR) mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+          else if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
+          auto load = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
+            if constexpr (PAIR) tma_load_2d_pair(dst, m, c0, c1, full_lead + s * 8);
+            else tma_load_2d(dst, m, c0, c1, &full[s]);
+          };
           const bool seg1 = kb >= args.kb_seg0;
           const int kk = (seg1 ? kb - args.kb_seg0 : kb) * kTileK;  // K inside the segment
           const int ka = t.a_k + (seg1 ? args.a_koff1 + kk : kk);
           if (A_MN) {
-            tma_load_2d(sA, &tmA, t.a_m, ka, &full[s]);
-            tma_load_2d(sA + 8192, &tmA, t.a_m + 64, ka, &full[s]);
+            load(sA, &tmA, t.a_m, ka);
+            load(sA + 8192, &tmA, t.a_m + 64, ka);
           } else {
-            tma_load_2d(sA, &tmA, ka, t.a_m, &full[s]);
+            load(sA, &tmA, ka, t.a_m);
           }
           const CUtensorMap* mapB = seg1 ? &tmB1 : &tmB0;
+          const int b_n = t.b_n + (PAIR && !B_DUAL ? (int)rank * kBRows : 0);
           if (B_DUAL) {
-            tma_load_2d(sB, &tmB0, t.b_k + kk, t.b_n, &full[s]);
-            tma_load_2d(sB + (BN / 2) * 128, &tmB1, t.b_k + kk, t.b_n, &full[s]);
+            if constexpr (PAIR) {
+              load(sB, rank ? &tmB1 : &tmB0, t.b_k + kk, t.b_n);  // even CTA: gate rows, odd: up
+            } else {
+              load(sB, &tmB0, t.b_k + kk, t.b_n);
+              load(sB + (BN / 2) * 128, &tmB1, t.b_k + kk, t.b_n);
+            }
           } else if (B_MN) {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sB + j * 8192, mapB, t.b_n + j * 64, t.b_k + kk, &full[s]);
+            for (int j = 0; j < kBRows / 64; ++j) load(sB + j * 8192, mapB, b_n + j * 64, t.b_k + kk);
           } else {
-            tma_load_2d(sB, mapB, t.b_k + kk, t.b_n, &full[s]);
+            load(sB, mapB, t.b_k + kk, b_n);
           }
         }
       }
@@ -275,12 +295,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       uint32_t it = 0;
       int local = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
         const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
         if (t.grp < 0) continue;
         const int buf = local & 1;
@@ -302,17 +322,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                      : smem_desc_sw128(a0 + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
                                      : smem_desc_sw128(b0 + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            else umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[s]);
+          if constexpr (PAIR) umma_commit_pair(&empty[s], 3);
+          else umma_commit(&empty[s]);
           issued = true;
         }
         if (!ok) break;
-        if (t.kb > 0) umma_commit(&tfull[buf]);
-        else mbar_arrive(&tfull[buf]);
+        if (t.kb > 0) {
+          if constexpr (PAIR) umma_commit_pair(&tfull[buf], 3);
+          else umma_commit(&tfull[buf]);
+        } else {
+          mbar_arrive(&tfull[buf]);
+          if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(smem_u32(&tfull[buf]), 1));
+        }
       }
       if (!ok && issued) {
-        umma_commit(drain);
+        if constexpr (PAIR) umma_commit_pair(drain, 1);
+        else umma_commit(drain);
         WaitCtl quick{abort_flag, args.status, 100000000ull};
         volatile int no_abort = 0;
         quick.abort = &no_abort;
@@ -323,10 +351,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue warps 2..5
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;
+    const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+    for (int tile = tile0; tile < num_tiles; tile += tile_step) {
+      Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
       if (t.grp < 0) continue;
+      if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       ++local;
@@ -446,15 +476,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 run = 0.f;
               }
             }
-          } else if constexpr (EPI == kEpiScatterAdd) {
-            const int tok = args.row_token[m];
-            if (tok >= 0) {
-              float* dst = args.acc32 + (int64_t)tok * args.ld_acc + n0;
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                if (n0 + v * 4 + 4 <= args.N)
-                  red_add_v4(dst + v * 4, acc[v * 4], acc[v * 4 + 1], acc[v * 4 + 2], acc[v * 4 + 3]);
-            }
           } else if constexpr (EPI == kEpiGroupDWgu) {
             const int G = args.group_size;
             __nv_bfloat16* op = nullptr;
@@ -479,15 +500,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      if (PAIR && rank != 0) mbar_arrive_cluster(tempty_lead + buf * 8);
+      else mbar_arrive(&tempty[buf]);
     }
   }
 
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the pair's MMAs and TMEM reads are all done
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
