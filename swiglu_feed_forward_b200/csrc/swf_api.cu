@@ -59,7 +59,7 @@ swf_status get_ctx(DevCtx* out) {
 }
 
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                      uint64_t row_elems, uint32_t box_cols, uint32_t box_rows) {
+                      uint64_t row_elems, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   std::call_once(g_encode_once, load_encode);
   if (!g_encode) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -67,7 +67,8 @@ bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

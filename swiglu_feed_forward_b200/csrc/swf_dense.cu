@@ -15,6 +15,13 @@
 
 namespace swf {
 
+namespace {
+// 32 x 32 box with 64-byte swizzle: the staging box of the TMA epilogue.
+bool epi_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t row_elems) {
+  return encode_tmap_bf16(m, base, cols, rows, row_elems, 32, 32, 64);
+}
+}  // namespace
+
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f) {
   auto t = [](int64_t m, int64_t n, int64_t bn) { return (int64_t)cdiv(m, kTileM) * cdiv(n, bn); };
   // pair-mode tiles of 256 rows
@@ -39,14 +46,14 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
   k1.aux1 = b;
   k1.ld_aux = f;
   swf_status s =
-      infer ? launch_tc_pair<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, k1, st)
-            : launch_tc_pair<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, k1, st);
+      infer ? launch_tc_pair<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, EpiMaps{}, k1, st)
+            : launch_tc_pair<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, EpiMaps{}, k1, st);
   if (s != SWF_OK) return s;
   // K2: y = h W_d^T
   TcGemmArgs k2 = base_args(M, d, 256, f, 2 * kTileM);
   k2.out0 = y;
   k2.ld_out = d;
-  return launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_DOWN, th, twd, twd, k2, st);
+  return launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_DOWN, th, twd, twd, EpiMaps{}, k2, st);
 }
 
 swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
@@ -58,14 +65,15 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     CUtensorMap tdy, twd;
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 64))
       return SWF_ERR_LAUNCH;
+    // TMA epilogue (measured: 1.05 -> 0.67 ms at 32768 x 2048 x 5504): a and b come in by TMA,
+    // dG and dU leave by TMA through two views of dGU (each [M, f], rows 2f apart)
+    EpiMaps e3{};
+    const __nv_bfloat16* dgu_b = static_cast<const __nv_bfloat16*>(dgu);
+    if (!epi_map(&e3.o[0], dgu_b, f, M, 2 * f) || !epi_map(&e3.o[1], dgu_b + f, f, M, 2 * f) ||
+        !epi_map(&e3.o[2], a, f, M, f) || !epi_map(&e3.o[3], b, f, M, f))
+      return SWF_ERR_LAUNCH;
     TcGemmArgs k3 = base_args(M, f, 256, d, 2 * kTileM);
-    k3.out0 = dgu;
-    k3.ld_out = 2 * f;
-    k3.aux0 = a;
-    k3.aux1 = b;
-    k3.ld_aux = f;
-    k3.d_ff = (int)f;
-    s = launch_tc_pair<256, false, true, false, kEpiDGate>(SWF_K_DGATE, tdy, twd, twd, k3, st);
+    s = launch_tc_pair<256, false, true, false, kEpiDGate, true>(SWF_K_DGATE, tdy, twd, twd, e3, k3, st);
     if (s != SWF_OK) return s;
   }
   {  // K4: dx = dG W_g + dU W_u: A = dGU (K-major, K = 2f), B segments W_g / W_u (MN-major)
@@ -79,7 +87,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     k4.a_koff1 = (int)f;
     k4.out0 = dx;
     k4.ld_out = d;
-    s = launch_tc_pair<256, false, true, false, kEpiStore>(SWF_K_DX, tdgu, twg, twu, k4, st);
+    s = launch_tc_pair<256, false, true, false, kEpiStore>(SWF_K_DX, tdgu, twg, twu, EpiMaps{}, k4, st);
     if (s != SWF_OK) return s;
   }
   {  // K5: [dW_g ; dW_u] = dGU^T x: A = dGU viewed [K=M rows, 2f cols] (MN-major), B = x (MN)
@@ -91,7 +99,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     k5.out1 = dwu;
     k5.row_split = (int)f;
     k5.ld_out = d;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, k5, st);
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, EpiMaps{}, k5, st);
     if (s != SWF_OK) return s;
   }
   {  // K6: dW_d = dY^T h: A = dY viewed [K=M rows, d cols] (MN), B = h [K=M rows, f cols] (MN)
@@ -101,7 +109,7 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     TcGemmArgs k6 = base_args(d, f, 256, M, 2 * kTileM);
     k6.out0 = dwd;
     k6.ld_out = f;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, k6, st);
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, EpiMaps{}, k6, st);
   }
   return s;
 }

@@ -24,20 +24,22 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE>;
-  constexpr int smem = TcSmem<BN>::kBytes;
+  constexpr int smem = TcSmem<BN, false, 0>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
   ProfScope prof(kind, st);
-  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, args);
+  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, EpiMaps{}, args);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 
 // Launches the pair-mode (cta_group::2) dense GEMM as clusters of two CTAs: min(tiles, SMs / 2)
-// clusters, each walking 256 x BN tiles.
-template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI>
+// clusters, each walking 256 x BN tiles.  TMA_EPI: the epilogue moves its tiles with TMA through
+// the maps in `em`.
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, bool TMA_EPI = false>
 swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
-                          const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
+                          const CUtensorMap& tb1, const EpiMaps& em, TcGemmArgs args,
+                          cudaStream_t st) {
   DevCtx ctx;
   swf_status s = get_ctx(&ctx);
   if (s != SWF_OK) return s;
@@ -47,8 +49,8 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   args.status = ctx.status;
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, kModeDense, true>;
-  constexpr int smem = TcSmem<BN, true>::kBytes;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, kModeDense, true, TMA_EPI>;
+  constexpr int smem = TcSmem<BN, true, epi_smem_bytes<EPI, TMA_EPI>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int clusters = (int)std::min<int64_t>(tiles, ctx.num_sms / 2);
@@ -65,7 +67,7 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ProfScope prof(kind, st);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb0, tb1, args) != cudaSuccess) return SWF_ERR_LAUNCH;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb0, tb1, em, args) != cudaSuccess) return SWF_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 

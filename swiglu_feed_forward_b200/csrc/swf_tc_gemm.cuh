@@ -84,18 +84,45 @@ struct TcGemmArgs {
   uint64_t wait_limit_ns;
 };
 
+// Epilogues that move their tiles with TMA: bf16 outputs staged per warp in shared memory
+// (32 x 32 boxes, 64-byte swizzle, double-buffered) and, for kEpiDGate, the a/b factor tiles
+// loaded by TMA into the same kind of buffers.
+template <int EPI>
+constexpr int tma_epi_outputs() {
+  return EPI == kEpiSwiGLU ? 3 : (EPI == kEpiDGate ? 2 : 1);
+}
+template <int EPI>
+constexpr int tma_epi_aux() {
+  return EPI == kEpiDGate ? 2 : 0;
+}
+constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
+template <int EPI, bool TMA_EPI>
+constexpr int epi_smem_bytes() {
+  return TMA_EPI ? 4 * (tma_epi_outputs<EPI>() + tma_epi_aux<EPI>()) * 2 * kEpiBox : 0;
+}
+
+// Tensor maps of a TMA epilogue: outputs in o[0..], kEpiDGate's a/b factors in o[2], o[3].
+struct EpiMaps {
+  CUtensorMap o[4];
+};
+
 // Shared-memory plan of one CTA.  In pair mode (cta_group::2) each CTA holds 128 rows of A and
-// BN/2 rows of B; the pair computes a 256 x BN tile.
-template <int BN, bool PAIR = false>
+// BN/2 rows of B; the pair computes a 256 x BN tile.  The stage ring takes what the epilogue
+// staging buffers and the barrier block leave of the 227 KB.
+template <int BN, bool PAIR = false, int EPI_BYTES = 0>
 struct TcSmem {
   static constexpr int kBRows = PAIR ? BN / 2 : BN;
   static constexpr int kABytes = kTileM * kTileK * 2;
   static constexpr int kBBytes = kBRows * kTileK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
+  // Without epilogue staging the ring stays at 192 KB (6 pair stages): measured on B200, a
+  // deeper ring that fills the 227 KB slowed the direct-store epilogues by 3-4%.
+  static constexpr int kBudget = EPI_BYTES == 0 ? 196608 : 232448 - 1024 - 512 - EPI_BYTES;
+  static constexpr int kStages = (kBudget / kStageBytes) < 8 ? (kBudget / kStageBytes) : 8;
   static constexpr int kTileBytes = kStages * kStageBytes;
-  static constexpr int kBarOffset = kTileBytes;
-  static constexpr int kBytes = kTileBytes + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kEpiOffset = kTileBytes;
+  static constexpr int kBarOffset = kTileBytes + EPI_BYTES;
+  static constexpr int kBytes = kBarOffset + 512 + 1024;  // barriers + alignment slack
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int raster, int& mb,
@@ -170,11 +197,12 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float* v) {
 // and runs its own epilogue.  Both CTAs' TMA loads complete on the even CTA's stage barrier,
 // and the MMA commits arrive on the stage and accumulator barriers of both CTAs.
 template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense,
-          bool PAIR = false>
+          bool PAIR = false, bool TMA_EPI = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                   const __grid_constant__ CUtensorMap tmB1, const TcGemmArgs args) {
-  using L = TcSmem<BN, PAIR>;
+                   const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ EpiMaps emaps,
+                   const TcGemmArgs args) {
+  using L = TcSmem<BN, PAIR, epi_smem_bytes<EPI, TMA_EPI>()>;
   constexpr int S = L::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(PAIR ? 2 * kTileM : kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
   constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
@@ -182,6 +210,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
   static_assert(!B_MN || kBRows % 64 == 0, "MN-major B tiles are whole 64-column boxes");
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
+  static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
+                                                    EPI == kEpiSwiGLUInf || EPI == kEpiDGate)),
+                "TMA epilogue: dense bf16 outputs");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -191,7 +222,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* auxbar = drain + 1;  // [4 epilogue warps][2 buffers]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -212,6 +244,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[b], PAIR ? 256 : 128);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&auxbar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -346,6 +379,157 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         quick.abort = &no_abort;
         mbar_wait(drain, 0, quick);
       }
+    }
+  } else if constexpr (TMA_EPI) {
+    // ------------------------------------------------------------ epilogue warps 2..5 (TMA I/O)
+    constexpr int NOUT = tma_epi_outputs<EPI>();
+    constexpr int NAUX = tma_epi_aux<EPI>();
+    constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
+    constexpr int NCH = (kGLU ? BN / 2 : BN) / 32;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int ew = warp - 2;
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (NOUT + NAUX) * 2 * kEpiBox;
+    uint8_t* abase = ebase + NOUT * 2 * kEpiBox;  // aux buffers [2][NAUX]
+    uint64_t* abar = auxbar + ew * 2;
+    const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this lane's staging row
+    uint32_t aux_issued = 0, aux_done = 0, chunks = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
+      Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+      if (t.grp < 0) continue;
+      if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
+      const int buf = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      ++local;
+      const int m_slab = t.a_m + q * 32;
+      const int n_base = t.nb * (kGLU ? BN / 2 : BN);
+      auto issue_aux = [&](int c) {
+        if constexpr (NAUX > 0) {
+          if (lane == 0) {
+            const int db = aux_issued & 1;
+            mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
+            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[2], n_base + c * 32, m_slab, &abar[db]);
+            tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
+          }
+          ++aux_issued;
+        }
+      };
+      issue_aux(0);  // the factors do not depend on the accumulator: fetch them early
+      const bool ready = mbar_wait(&tfull[buf], use & 1u, ctl);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ready)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
+      const bool have_acc = t.kb > 0;
+#pragma unroll 1
+      for (int c = 0; c < NCH; ++c) {
+        const uint8_t* aux = nullptr;
+        if constexpr (NAUX > 0) {
+          if (c + 1 < NCH) issue_aux(c + 1);
+          const int db = aux_done & 1;
+          const bool got = mbar_wait(&abar[db], (aux_done >> 1) & 1u, ctl);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          ++aux_done;
+          aux = abase + (db * NAUX) * kEpiBox;
+        }
+        float v0[32], v1[32];
+        if (have_acc) {
+          tmem_ld32(t_acc + c * 32, v0);
+          if constexpr (kGLU) tmem_ld32(t_acc + BN / 2 + c * 32, v1);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0.f;
+        }
+        uint32_t w[NOUT][16];
+        if constexpr (EPI == kEpiStore) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[0][i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+        } else if constexpr (kGLU) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float hv[2], av[2], bv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float g = v0[2 * i + e], u = v1[2 * i + e];
+              const float sg = sigmoidf_(g);
+              bv[e] = g * sg;
+              hv[e] = bv[e] * u;
+              av[e] = u * sg * (1.f + g * (1.f - sg));
+            }
+            w[0][i] = pack_bf16x2(hv[0], hv[1]);
+            if constexpr (EPI == kEpiSwiGLU) {
+              w[1][i] = pack_bf16x2(av[0], av[1]);
+              w[2][i] = pack_bf16x2(bv[0], bv[1]);
+            }
+          }
+        } else if constexpr (EPI == kEpiDGate) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int off = lane * 64 + ((c4 ^ swz) * 16);
+            const uint4 av = *reinterpret_cast<const uint4*>(aux + off);
+            const uint4 bv = *reinterpret_cast<const uint4*>(aux + kEpiBox + off);
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const float d0 = v0[c4 * 8 + p * 2], d1 = v0[c4 * 8 + p * 2 + 1];
+              w[0][c4 * 4 + p] = pack_bf16x2(d0 * bf16_lo(aw[p]), d1 * bf16_hi(aw[p]));
+              w[1][c4 * 4 + p] = pack_bf16x2(d0 * bf16_lo(bw[p]), d1 * bf16_hi(bw[p]));
+            }
+          }
+        }
+        // stage this warp's 32 x 32 box of every output, then one lane stores them with TMA
+        const int db = chunks & 1;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last used buffer db has read it
+        __syncwarp();
+#pragma unroll
+        for (int o = 0; o < NOUT; ++o) {
+          uint8_t* ob = ebase + (o * 2 + db) * kEpiBox;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(ob + lane * 64 + ((c4 ^ swz) * 16)) =
+                make_uint4(w[o][c4 * 4], w[o][c4 * 4 + 1], w[o][c4 * 4 + 2], w[o][c4 * 4 + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int n0 = n_base + c * 32;
+        // A box that starts inside its tensor is clipped by TMA at the far edges; boxes that
+        // start past the last row or column are not issued at all.
+        if (lane == 0 && m_slab < args.M && n0 < args.N) {
+          if constexpr (EPI == kEpiStore) {
+            if (m_slab < args.row_split) tma_store_2d(&emaps.o[0], n0, m_slab, ebase + db * kEpiBox);
+            else tma_store_2d(&emaps.o[1], n0, m_slab - args.row_split, ebase + db * kEpiBox);
+          } else {
+#pragma unroll
+            for (int o = 0; o < NOUT; ++o)
+              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * 2 + db) * kEpiBox);
+          }
+          bulk_commit();
+        }
+        ++chunks;
+      }
+      if (!ok) break;
+      tc_fence_before();
+      if (PAIR && rank != 0) mbar_arrive_cluster(tempty_lead + buf * 8);
+      else mbar_arrive(&tempty[buf]);
+    }
+    if (lane == 0) {
+      // factor loads still in flight after an abort land before the CTA leaves (bounded)
+      WaitCtl quick{abort_flag, args.status, 100000000ull};
+      volatile int no_abort = 0;
+      quick.abort = &no_abort;
+      for (; aux_done < aux_issued; ++aux_done) mbar_wait(&abar[aux_done & 1], (aux_done >> 1) & 1u, quick);
+      bulk_wait_all();
     }
   } else {
     // ------------------------------------------------------------ epilogue warps 2..5
