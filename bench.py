@@ -74,7 +74,7 @@ def source_sha():
 def ncu_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when absent or
     taken on other kernel sources."""
-    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
