@@ -164,9 +164,11 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """Max of a per-rank float over all ranks (a CPU tensor for gloo, a device one for NCCL)."""
     if world == 1:
         return v
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

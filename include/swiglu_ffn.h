@@ -198,6 +198,24 @@ swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const void* w_ga
                                  int32_t group_size, int32_t num_active_groups, swf_dtype dtype,
                                  void* stream);
 
+/* Group-usage frequency of one batch (eugen_sparse README, "What it does": the balancing step
+ * uses the current usage of each group): freq[c] = (number of tokens whose group_idx row holds c)
+ * / M, fp32 [num_groups].  The frequencies sum to num_active_groups.  Entries that are out of
+ * range or repeat an earlier slot of the same row are not counted. */
+swf_status swf_group_frequency(const int32_t* group_idx, int64_t M, int32_t num_active_groups,
+                               int32_t num_groups, float* freq, void* stream);
+
+/* Auxiliary-loss-free load balancing, called once per optimizer step (eugen_sparse README,
+ * update_load_balance_bias, "in the style of DeepSeek-V3"; defaults gamma 1e-3, bias_max 0.5,
+ * momentum 0.99, target_freq = num_active_groups / num_groups).  In place on the device, per
+ * group c:  freq_ema[c] = momentum * freq_ema[c] + (1 - momentum) * current_freq[c];
+ *           bias[c] = clamp(bias[c] + gamma * sign(target_freq - freq_ema[c]), -bias_max, bias_max)
+ * (the README gives no formula; this is the plainest reading of it).  All arrays fp32
+ * [num_groups]; bias and freq_ema are the caller's persistent buffers. */
+swf_status update_load_balance_bias(float* bias, float* freq_ema, const float* current_freq,
+                                    float target_freq, float gamma, float bias_max,
+                                    float momentum, int32_t num_groups, void* stream);
+
 /* ------------------------------------------------------------------ planning and queries */
 
 /* Workspace bytes `op` needs (0 if none).  group_size / num_active_groups are ignored by the
@@ -252,7 +270,8 @@ typedef enum swf_kernel_kind {
   SWF_K_SPARSE_DW = 17,    /* sparse weight-gradient GEMMs */
   SWF_K_ELEMENTWISE = 18,  /* fills */
   SWF_K_PAIR_SUM = 19,     /* per-token sum of the per-pair contributions (y, dx) */
-  SWF_K_NUM_KINDS = 20
+  SWF_K_BALANCE = 20,      /* group frequency and balancing-bias update */
+  SWF_K_NUM_KINDS = 21
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

@@ -45,7 +45,7 @@ __all__ = [
     "sparse_forward_by_groups",
     "splitmix64_stream", "make_subsample_index",
     "group_energy", "topk_groups", "topk_gap",
-    "csr_buckets", "update_load_balance_bias",
+    "csr_buckets", "group_frequency", "update_load_balance_bias",
 ]
 
 
@@ -277,6 +277,18 @@ def csr_buckets(group_idx, num_groups):
         offs[c + 1] = offs[c] + toks.size
     tokens = np.concatenate(lists) if lists else np.zeros(0, dtype=np.int64)
     return offs.astype(np.int32), tokens.astype(np.int32)
+
+
+def group_frequency(group_idx, num_groups):
+    """Fraction of the tokens whose selection holds each group: count[c] / tokens.  The
+    frequencies of a batch sum to num_active_groups, so the balanced target of every group is
+    num_active_groups / num_groups (eugen_sparse "Parameters": target_freq)."""
+    group_idx = np.asarray(group_idx)
+    counts = np.zeros(num_groups, dtype=np.float64)
+    for row in group_idx:
+        for c in set(int(v) for v in row):
+            counts[c] += 1.0
+    return counts / group_idx.shape[0]
 
 
 def update_load_balance_bias(bias, freq_ema, current_freq, target_freq,

@@ -41,6 +41,8 @@ SIGNATURES = {
     "sparse_swiglu_ffn_fwd": (I32, [P, P, P, P, P, I32, I32, P, P, SZ, P, SZ, I64, I64, I64, I32, P]),
     "sparse_swiglu_ffn_bwd": (I32, [P, P, P, P, P, P, P, SZ, P, P, P, P, P, SZ, I64, I64, I64,
                                     I32, I32, I32, P]),
+    "swf_group_frequency": (I32, [P, I64, I32, I32, P, P]),
+    "update_load_balance_bias": (I32, [P, P, P, C.c_float, C.c_float, C.c_float, C.c_float, I32, P]),
     "swf_workspace_bytes": (SZ, [I32, I64, I64, I64, I32, I32, I32]),
     "swf_sparse_saved_bytes": (SZ, [I64, I64, I64, I32, I32, I32]),
     "swf_supported": (I32, [I32, I64, I64, I64, I32, I32, I32, I32]),

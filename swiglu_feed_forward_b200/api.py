@@ -148,6 +148,24 @@ def swf_group_buckets(group_idx, num_groups, offsets=None, tokens=None, workspac
     return offsets, tokens
 
 
+def group_frequency(group_idx, num_groups, freq=None, stream=None):
+    """Fraction of tokens that selected each group (fp32 [num_groups])."""
+    M, K = group_idx.shape
+    freq = torch.empty(num_groups, device=group_idx.device, dtype=torch.float32) if freq is None else freq
+    _check("swf_group_frequency", _lib.lib().swf_group_frequency(
+        _p(group_idx), M, K, num_groups, _p(freq), _stream(stream)))
+    return freq
+
+
+def update_load_balance_bias(bias, freq_ema, current_freq, target_freq, gamma=1e-3, bias_max=0.5,
+                             momentum=0.99, stream=None):
+    """In-place balancing step on the device buffers bias and freq_ema (fp32 [num_groups])."""
+    _check("update_load_balance_bias", _lib.lib().update_load_balance_bias(
+        _p(bias), _p(freq_ema), _p(current_freq), float(target_freq), float(gamma),
+        float(bias_max), float(momentum), bias.numel(), _stream(stream)))
+    return bias, freq_ema
+
+
 def sparse_saved_bytes(M, d, f, group_size, num_active_groups, dtype=torch.bfloat16):
     return _lib.lib().swf_sparse_saved_bytes(M, d, f, group_size, num_active_groups,
                                              SWF_BF16 if dtype == torch.bfloat16 else SWF_F32)

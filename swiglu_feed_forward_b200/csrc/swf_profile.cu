@@ -40,7 +40,8 @@ const char* const kNames[SWF_K_NUM_KINDS] = {
     "gate_up_swiglu",  "gate_up_swiglu_infer", "down_proj",     "dgate",         "dx",
     "dw_gate_up",      "dw_down",              "f32_gemm",      "select_gather", "select_score",
     "select_topk",     "buckets",              "sparse_gather", "sparse_up",     "sparse_down",
-    "sparse_dgate",    "sparse_dx",            "sparse_dw",     "elementwise",   "pair_sum"};
+    "sparse_dgate",    "sparse_dx",            "sparse_dw",     "elementwise",   "pair_sum",
+    "balance"};
 
 }  // namespace
 

@@ -297,24 +297,32 @@ __global__ void fill_i32_kernel(int32_t* __restrict__ p, int64_t n, int32_t v) {
 }
 
 // out[t, :] = sum over t's valid slots k (in slot order) of rows[pair_row[t*K + k], :], fp32
-// accumulation, bf16 result: the deterministic reduction of the per-pair contributions.
+// accumulation, bf16 result: the deterministic reduction of the per-pair contributions.  One
+// warp per token; each lane issues the (up to 8) row loads of a slot chunk before summing them.
 __global__ void pair_sum_kernel(const uint4* __restrict__ rows, const int32_t* __restrict__ pair_row,
                                 int64_t M, int K, int64_t row_vecs, uint4* __restrict__ out) {
+  constexpr int kChunk = 8;
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < M; t += warps) {
     const int32_t* pr = pair_row + t * K;
     for (int64_t v = lane; v < row_vecs; v += 32) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int k = 0; k < K; ++k) {
-        const int32_t r = pr[k];
-        if (r < 0) continue;
-        const uint4 q = rows[(int64_t)r * row_vecs + v];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      for (int k0 = 0; k0 < K; k0 += kChunk) {
+        uint4 q[kChunk];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[2 * i] += bf16_lo(w[i]);
-          acc[2 * i + 1] += bf16_hi(w[i]);
+        for (int j = 0; j < kChunk; ++j) {
+          const int32_t r = (k0 + j < K) ? pr[k0 + j] : -1;
+          q[j] = r >= 0 ? rows[(int64_t)r * row_vecs + v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+          const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += bf16_lo(w[i]);
+            acc[2 * i + 1] += bf16_hi(w[i]);
+          }
         }
       }
       out[t * row_vecs + v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
@@ -660,6 +668,67 @@ extern "C" swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int
   const SparseDims d = dims_of(M, 16, (int64_t)ng * 16, 16, K);
   return run_buckets(group_idx, d, static_cast<int32_t*>(workspace), offsets, tokens, nullptr,
                      nullptr, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ load balancing
+
+namespace swf {
+namespace {
+
+// One block: integer counts of the valid slots per group (shared atomics; integers, so the
+// result does not depend on their order), then freq[c] = count[c] / M.
+__global__ void group_frequency_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
+                                       float* __restrict__ freq) {
+  extern __shared__ int32_t cnt[];
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) cnt[c] = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < M * K; i += blockDim.x) {
+    const int32_t* row = idx + (i / K) * K;
+    const int k = (int)(i % K);
+    if (valid_slot(row, k, ng)) atomicAdd(&cnt[row[k]], 1);
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) freq[c] = (float)cnt[c] / (float)M;
+}
+
+__global__ void balance_update_kernel(float* __restrict__ bias, float* __restrict__ ema,
+                                      const float* __restrict__ cur, float target, float gamma,
+                                      float bias_max, float momentum, int ng) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= ng) return;
+  const float e = momentum * ema[c] + (1.0f - momentum) * cur[c];
+  ema[c] = e;
+  const float sgn = (target > e) ? 1.0f : ((target < e) ? -1.0f : 0.0f);
+  bias[c] = fminf(fmaxf(bias[c] + gamma * sgn, -bias_max), bias_max);
+}
+
+}  // namespace
+}  // namespace swf
+
+extern "C" swf_status swf_group_frequency(const int32_t* group_idx, int64_t M, int32_t K,
+                                          int32_t ng, float* freq, void* stream) {
+  if (!group_idx || !freq) return SWF_ERR_INVALID_ARG;
+  swf_status s = swf_supported(SWF_OP_BUCKETS, M, 0, 0, ng, K, 0, SWF_BF16);
+  if (s != SWF_OK) return s;
+  if (ng > 12288) return SWF_ERR_UNSUPPORTED;
+  if (!aligned16(group_idx) || !aligned16(freq)) return SWF_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope prof(SWF_K_BALANCE, st);
+  group_frequency_kernel<<<1, 1024, ng * sizeof(int32_t), st>>>(group_idx, M, K, ng, freq);
+  return launched();
+}
+
+extern "C" swf_status update_load_balance_bias(float* bias, float* freq_ema, const float* cur,
+                                               float target, float gamma, float bias_max,
+                                               float momentum, int32_t ng, void* stream) {
+  if (!bias || !freq_ema || !cur) return SWF_ERR_INVALID_ARG;
+  if (ng <= 0 || !(bias_max >= 0.f) || !(momentum >= 0.f && momentum <= 1.f)) return SWF_ERR_INVALID_ARG;
+  if (!aligned16(bias) || !aligned16(freq_ema) || !aligned16(cur)) return SWF_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope prof(SWF_K_BALANCE, st);
+  balance_update_kernel<<<(ng + 255) / 256, 256, 0, st>>>(bias, freq_ema, cur, target, gamma,
+                                                          bias_max, momentum, ng);
+  return launched();
 }
 
 // ------------------------------------------------------------------ sparse forward

@@ -311,3 +311,12 @@ def test_load_balance_bias_update():
     np.testing.assert_allclose(nb, [-0.02, 0.02, 0.5, -0.5])
     nb2, _ = O.update_load_balance_bias(bias, ema, ema, 0.25, 0.02, 0.5, 0.9)
     np.testing.assert_allclose(nb2, bias)
+
+
+def test_group_frequency():
+    idx = np.array([[0, 2], [1, 2], [2, 3]])
+    np.testing.assert_allclose(O.group_frequency(idx, 5), [1 / 3, 1 / 3, 1.0, 1 / 3, 0.0])
+    rng = np.random.default_rng(3)
+    big = np.sort(np.stack([rng.choice(16, size=4, replace=False) for _ in range(500)]), axis=1)
+    f = O.group_frequency(big, 16)
+    assert abs(f.sum() - 4.0) < 1e-12  # frequencies sum to K: the balanced target is K / groups

@@ -171,3 +171,27 @@ def test_sparse_all_groups_matches_dense_gpu():
     torch.cuda.synchronize()
     for k, v in zip(("y", "dx", "dw_gate", "dw_up", "dw_down"), (y,) + tuple(dn)):
         assert rel_err(f64(sp[k]), f64(v)) <= 1e-2, k
+
+
+def test_group_frequency_and_balance_update():
+    M, K, ng = 5000, 4, 32
+    rng = np.random.default_rng(11)
+    idx = np.sort(np.stack([rng.choice(ng, size=K, replace=False) for _ in range(M)]), axis=1).astype(np.int32)
+    freq = api.group_frequency(torch.from_numpy(idx).cuda(), ng)
+    torch.cuda.synchronize()
+    ref_f = O.group_frequency(idx, ng)
+    np.testing.assert_allclose(freq.cpu().numpy(), ref_f, rtol=1e-6, atol=1e-7)
+    bias0 = rng.uniform(-0.5, 0.5, ng).astype(np.float32)
+    bias0[:3] = [0.4995, -0.4995, 0.0]
+    ema0 = rng.uniform(0.0, 0.3, ng).astype(np.float32)
+    target, gamma, bias_max, momentum = K / ng, 1e-3, 0.5, 0.99
+    bias, ema = torch.from_numpy(bias0).cuda(), torch.from_numpy(ema0).cuda()
+    api.update_load_balance_bias(bias, ema, freq, target, gamma, bias_max, momentum)
+    torch.cuda.synchronize()
+    ref_b, ref_e = O.update_load_balance_bias(bias0.astype(np.float64), ema0.astype(np.float64),
+                                              ref_f, target, gamma, bias_max, momentum)
+    np.testing.assert_allclose(ema.cpu().numpy(), ref_e, rtol=1e-5, atol=1e-7)
+    # the sign decision is exact except where the new EMA sits at the target
+    decided = np.abs(target - ref_e) > 1e-5
+    np.testing.assert_allclose(bias.cpu().numpy()[decided], ref_b[decided], atol=1e-6)
+    assert np.all(np.abs(bias.cpu().numpy()) <= bias_max + 1e-7)
