@@ -41,6 +41,7 @@ import numpy as np
 __all__ = [
     "sigmoid", "silu", "silu_prime",
     "dense_forward", "dense_backward",
+    "leaky_relu_sq_forward", "leaky_relu_sq_backward",
     "group_mask", "sparse_forward", "sparse_backward",
     "sparse_forward_by_groups",
     "splitmix64_stream", "make_subsample_index",
@@ -114,6 +115,31 @@ def dense_backward(x, w_gate, w_up, w_down, dy):
         "dw_down": dy.T @ fw["h"],
         "dh": dh, "dg": dg, "du": du,
     }
+
+
+# --------------------------------------------------------------------------
+# LeakyReLU(0.5)^2 MLP (parameter-golf PR 1105, "Fused MLP Kernels")
+# --------------------------------------------------------------------------
+def leaky_relu_sq_forward(x, w_up, w_down):
+    """pre = x W_up^T; post = LeakyReLU(0.5)(pre)^2; y = post W_down^T, with the
+    activation gradient the forward stores instead of the pre-activation:
+    act_grad = 2 pre where pre > 0, 0.5 pre elsewhere (d post / d pre).
+    w_up [hidden, d_model], w_down [d_model, hidden] (nn.Linear layout)."""
+    x, w_up, w_down = map(_f64, (x, w_up, w_down))
+    pre = x @ w_up.T
+    leaky = np.where(pre > 0, pre, 0.5 * pre)
+    post = leaky * leaky
+    act_grad = np.where(pre > 0, 2.0 * pre, 0.5 * pre)
+    return {"pre": pre, "post": post, "act_grad": act_grad, "y": post @ w_down.T}
+
+
+def leaky_relu_sq_backward(x, w_up, w_down, dy):
+    """Chain rule of L = sum(dy * y): dpre = (dy W_down) * act_grad;
+    dx = dpre W_up; dW_up = dpre^T x; dW_down = dy^T post."""
+    x, w_up, w_down, dy = map(_f64, (x, w_up, w_down, dy))
+    fw = leaky_relu_sq_forward(x, w_up, w_down)
+    dpre = (dy @ w_down) * fw["act_grad"]
+    return {"dx": dpre @ w_up, "dw_up": dpre.T @ x, "dw_down": dy.T @ fw["post"], "dpre": dpre}
 
 
 # --------------------------------------------------------------------------

@@ -320,3 +320,38 @@ def test_group_frequency():
     big = np.sort(np.stack([rng.choice(16, size=4, replace=False) for _ in range(500)]), axis=1)
     f = O.group_frequency(big, 16)
     assert abs(f.sum() - 4.0) < 1e-12  # frequencies sum to K: the balanced target is K / groups
+
+
+
+# ---------------------------------------------------------------- LeakyReLU(0.5)^2 MLP
+def test_leaky_relu_sq_page_identity_both_signs():
+    # the fused-MLP page's derivation: post = 0.5 * act_grad * pre for pre > 0 (pre^2) and
+    # pre <= 0 ((0.5 pre)^2), with act_grad = 2 pre or 0.5 pre
+    x, wu, wd = rnd((6, 8), 61), rnd((12, 8), 62, 8 ** -0.5), rnd((8, 12), 63, 12 ** -0.5)
+    fw = O.leaky_relu_sq_forward(x, wu, wd)
+    pre = fw["pre"]
+    assert np.any(pre > 0) and np.any(pre < 0)
+    np.testing.assert_allclose(fw["post"], 0.5 * fw["act_grad"] * pre, rtol=1e-14)
+    np.testing.assert_allclose(fw["post"][pre > 0], pre[pre > 0] ** 2, rtol=1e-14)
+    np.testing.assert_allclose(fw["post"][pre <= 0], (0.5 * pre[pre <= 0]) ** 2, rtol=1e-14)
+    # act_grad is d post / d pre
+    eps = 1e-6
+    lk = lambda z: np.where(z > 0, z, 0.5 * z) ** 2
+    np.testing.assert_allclose(fw["act_grad"], (lk(pre + eps) - lk(pre - eps)) / (2 * eps), atol=1e-8)
+
+
+def test_leaky_relu_sq_matches_torch_autograd_and_fd():
+    x, wu, wd, dy = rnd((16, 32), 71), rnd((56, 32), 72, 32 ** -0.5), rnd((32, 56), 73, 56 ** -0.5), rnd((16, 32), 74, 0.1)
+    ts = [torch.from_numpy(a).requires_grad_(True) for a in (x, wu, wd)]
+    F = torch.nn.functional
+    y = F.linear(F.leaky_relu(F.linear(ts[0], ts[1]), 0.5) ** 2, ts[2])
+    y.backward(torch.from_numpy(dy))
+    fw = O.leaky_relu_sq_forward(x, wu, wd)
+    np.testing.assert_allclose(fw["y"], y.detach().numpy(), rtol=1e-12, atol=1e-13)
+    bw = O.leaky_relu_sq_backward(x, wu, wd, dy)
+    for name, t in zip(("dx", "dw_up", "dw_down"), ts):
+        np.testing.assert_allclose(bw[name], t.grad.numpy(), rtol=1e-11, atol=1e-12)
+    xs, wus, wds, dys = x[:3, :4].copy(), wu[:6, :4].copy(), wd[:4, :6].copy(), dy[:3, :4].copy()
+    loss = lambda: float(np.sum(dys * O.leaky_relu_sq_forward(xs, wus, wds)["y"]))
+    b2 = O.leaky_relu_sq_backward(xs, wus, wds, dys)
+    _fd_check(loss, [xs, wus, wds], [b2["dx"], b2["dw_up"], b2["dw_down"]])
