@@ -332,6 +332,29 @@ def secondary_sparse(api, steps, warmup, world, peak):
             "steps": steps, "useful_flops_per_step": useful}
 
 
+def secondary_mlp2(api, steps, warmup, world, peak):
+    """parameter-golf PR 1105's LeakyReLU(0.5)^2 MLP: fwd + bwd, 12 * M * d * hidden FLOPs."""
+    w = synth.WORKLOADS[5]
+    M, d, f = w["M"], w["d_model"], w["d_ff"]
+    dev = torch.device("cuda")
+    inp = synth.workload_inputs(5)
+    t = {k: v.to(dev) for k, v in inp.items()}
+    e = lambda *sh: torch.empty(*sh, device=dev, dtype=torch.bfloat16)
+    y, post, ag, dx, dwu, dwd = e(M, d), e(M, f), e(M, f), e(M, d), e(f, d), e(d, f)
+    ws = torch.empty(api.workspace_bytes("mlp2_bwd", M, d, f), device=dev, dtype=torch.uint8)
+
+    def fn():
+        api.leaky_relu_sq_mlp_fwd(t["x"], t["w_up"], t["w_down"], y, post, ag)
+        api.leaky_relu_sq_mlp_bwd(t["dy"], t["x"], t["w_up"], t["w_down"], post, ag, dx, dwu, dwd, ws)
+    for _ in range(warmup):
+        fn()
+    ms = timed(fn, steps, world)
+    flops = 12.0 * M * d * f
+    tf = flops * steps / (ms / 1e3) / 1e12
+    return {"workload": w["name"], "tflops": round(tf * world, 2), "pct_of_peak": round(100 * tf / peak, 2),
+            "ms_per_step": round(ms / steps, 3), "steps": steps}
+
+
 def run_ours(args, world, rank, local):
     from swiglu_feed_forward_b200 import api
     w = synth.WORKLOADS[WORKLOAD]
@@ -417,6 +440,11 @@ def run_ours(args, world, rank, local):
             secondary["group_sparse_step"] = secondary_sparse(api, max(3, args.steps // 2), 3, world, peak_sus)
         except Exception as exc:
             secondary["group_sparse_step"] = {"error": str(exc)[:200]}
+        torch.cuda.empty_cache()
+        try:
+            secondary["leaky_relu_sq_mlp_step"] = secondary_mlp2(api, max(3, args.steps // 2), 3, world, peak_sus)
+        except Exception as exc:
+            secondary["leaky_relu_sq_mlp_step"] = {"error": str(exc)[:200]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

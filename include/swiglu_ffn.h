@@ -66,7 +66,9 @@ typedef enum swf_op {
   SWF_OP_SELECT = 3,      /* grouped_topk_select */
   SWF_OP_SPARSE_FWD = 4,  /* sparse_swiglu_ffn_fwd */
   SWF_OP_SPARSE_BWD = 5,  /* sparse_swiglu_ffn_bwd */
-  SWF_OP_BUCKETS = 6      /* swf_group_buckets */
+  SWF_OP_BUCKETS = 6,     /* swf_group_buckets */
+  SWF_OP_MLP2_FWD = 7,    /* leaky_relu_sq_mlp_fwd (d_ff = hidden) */
+  SWF_OP_MLP2_BWD = 8     /* leaky_relu_sq_mlp_bwd (d_ff = hidden) */
 } swf_op;
 
 /* How an operation will run (eugen_sparse README: plan() reports how the work is split,
@@ -138,6 +140,31 @@ swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate, con
 swf_status swiglu_ffn_fwd_infer_noalloc(const void* x, const void* w_gate, const void* w_up,
                                         const void* w_down, void* y, int64_t M, int64_t d_model,
                                         int64_t d_ff, swf_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------ LeakyReLU(0.5)^2 MLP */
+
+/* The MLP of parameter-golf PR 1105 ("Fused MLP Kernels"): an up projection, LeakyReLU with
+ * slope 0.5, a square, and a down projection, with the activation gradient stored in the
+ * forward pass instead of the pre-activation:
+ *   pre = x W_up^T (fp32 accumulation, never written to memory),
+ *   saved_post = LeakyReLU(0.5)(pre)^2,  saved_act_grad = 2 pre if pre > 0 else 0.5 pre,
+ *   y = saved_post W_down^T.
+ * w_up [hidden, d_model], w_down [d_model, hidden] (nn.Linear layout); saved_* [M, hidden] are
+ * outputs the caller keeps for the backward.  Same dtype and shape rules as the dense SwiGLU
+ * entry points (hidden in place of d_ff).  No workspace. */
+swf_status leaky_relu_sq_mlp_fwd(const void* x, const void* w_up, const void* w_down, void* y,
+                                 void* saved_post, void* saved_act_grad, int64_t M,
+                                 int64_t d_model, int64_t hidden, swf_dtype dtype, void* stream);
+
+/* Backward of the MLP above (the page's branch-free backward: the multiply by the stored
+ * activation gradient happens in the GEMM epilogue):
+ *   dpre = (dy W_down) * saved_act_grad      (workspace, [M, hidden])
+ *   dx = dpre W_up;  dw_up = dpre^T x;  dw_down = dy^T saved_post   (overwritten). */
+swf_status leaky_relu_sq_mlp_bwd(const void* dy, const void* x, const void* w_up,
+                                 const void* w_down, const void* saved_post,
+                                 const void* saved_act_grad, void* dx, void* dw_up, void* dw_down,
+                                 void* workspace, size_t workspace_bytes, int64_t M,
+                                 int64_t d_model, int64_t hidden, swf_dtype dtype, void* stream);
 
 /* ------------------------------------------------------------------ group-sparse variant */
 
@@ -271,7 +298,11 @@ typedef enum swf_kernel_kind {
   SWF_K_ELEMENTWISE = 18,  /* fills */
   SWF_K_PAIR_SUM = 19,     /* per-token sum of the per-pair contributions (y, dx) */
   SWF_K_BALANCE = 20,      /* group frequency and balancing-bias update */
-  SWF_K_NUM_KINDS = 21
+  SWF_K_MLP2_UP = 21,      /* LeakyReLU^2 MLP: x W_up^T with the post / act_grad epilogue */
+  SWF_K_MLP2_DPRE = 22,    /* LeakyReLU^2 MLP: (dY W_down) * act_grad */
+  SWF_K_MLP2_DX = 23,      /* LeakyReLU^2 MLP: dpre W_up */
+  SWF_K_MLP2_DW_UP = 24,   /* LeakyReLU^2 MLP: dpre^T x */
+  SWF_K_NUM_KINDS = 25
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

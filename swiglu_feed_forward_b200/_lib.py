@@ -16,7 +16,7 @@ STATUS_NAMES = {0: "SWF_OK", 1: "SWF_ERR_INVALID_ARG", 2: "SWF_ERR_UNSUPPORTED",
                 6: "SWF_ERR_TIMEOUT"}
 SWF_F32, SWF_BF16 = 0, 1
 OPS = {"fwd": 0, "fwd_infer": 1, "bwd": 2, "select": 3, "sparse_fwd": 4, "sparse_bwd": 5,
-       "buckets": 6}
+       "buckets": 6, "mlp2_fwd": 7, "mlp2_bwd": 8}
 
 
 class swf_plan_info(C.Structure):
@@ -35,6 +35,8 @@ SIGNATURES = {
     "swiglu_ffn_fwd_infer": (I32, [P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swiglu_ffn_fwd_infer_noalloc": (I32, [P, P, P, P, P, I64, I64, I64, I32, P]),
     "swiglu_ffn_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
+    "leaky_relu_sq_mlp_fwd": (I32, [P, P, P, P, P, P, I64, I64, I64, I32, P]),
+    "leaky_relu_sq_mlp_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swf_make_subsample_index": (I32, [I64, I32, I32, U64, P]),
     "grouped_topk_select": (I32, [P, P, P, I32, P, I32, I32, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swf_group_buckets": (I32, [P, I64, I32, I32, P, P, P, SZ, P]),

@@ -102,6 +102,35 @@ def swiglu_ffn_bwd(dy, x, w_gate, w_up, w_down, saved_h, saved_a, saved_b, dx=No
     return dx, dw_gate, dw_up, dw_down
 
 
+# ------------------------------------------------------------------ LeakyReLU(0.5)^2 MLP
+def leaky_relu_sq_mlp_fwd(x, w_up, w_down, y=None, saved_post=None, saved_act_grad=None, stream=None):
+    """Returns (y, saved_post, saved_act_grad)."""
+    M, d = x.shape
+    f = w_up.shape[0]
+    y = _empty((M, d), x) if y is None else y
+    saved_post = _empty((M, f), x) if saved_post is None else saved_post
+    saved_act_grad = _empty((M, f), x) if saved_act_grad is None else saved_act_grad
+    _check("leaky_relu_sq_mlp_fwd", _lib.lib().leaky_relu_sq_mlp_fwd(
+        _p(x), _p(w_up), _p(w_down), _p(y), _p(saved_post), _p(saved_act_grad), M, d, f, _dt(x),
+        _stream(stream)))
+    return y, saved_post, saved_act_grad
+
+
+def leaky_relu_sq_mlp_bwd(dy, x, w_up, w_down, saved_post, saved_act_grad, dx=None, dw_up=None,
+                          dw_down=None, workspace=None, stream=None):
+    """Returns (dx, dw_up, dw_down)."""
+    M, d = x.shape
+    f = w_up.shape[0]
+    dx = _empty((M, d), x) if dx is None else dx
+    dw_up = _empty((f, d), x) if dw_up is None else dw_up
+    dw_down = _empty((d, f), x) if dw_down is None else dw_down
+    ws, nb = _workspace("mlp2_bwd", M, d, f, 0, 0, _dt(x), x, workspace)
+    _check("leaky_relu_sq_mlp_bwd", _lib.lib().leaky_relu_sq_mlp_bwd(
+        _p(dy), _p(x), _p(w_up), _p(w_down), _p(saved_post), _p(saved_act_grad), _p(dx), _p(dw_up),
+        _p(dw_down), _p(ws), nb, M, d, f, _dt(x), _stream(stream)))
+    return dx, dw_up, dw_down
+
+
 # ------------------------------------------------------------------ group-sparse
 def make_subsample_index(d_ff, group_size, samples_per_group, seed):
     """Host call: returns (int32 CPU tensor [d_ff // group_size, spg], spg)."""

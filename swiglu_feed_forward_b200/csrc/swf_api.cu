@@ -145,6 +145,9 @@ extern "C" swf_status swf_supported(swf_op op, int64_t M, int64_t d, int64_t f, 
     case SWF_OP_SPARSE_FWD:
     case SWF_OP_SPARSE_BWD:
       return check_sparse_shape(M, d, f, G, K, dt);
+    case SWF_OP_MLP2_FWD:
+    case SWF_OP_MLP2_BWD:
+      return check_dense(M, d, f, dt);
     case SWF_OP_BUCKETS:
       if (M <= 0 || K <= 0 || G <= 0) return SWF_ERR_INVALID_ARG;
       if (K > G || M * (int64_t)K >= (int64_t(1) << 31)) return SWF_ERR_UNSUPPORTED;
@@ -165,6 +168,8 @@ extern "C" size_t swf_workspace_bytes(swf_op op, int64_t M, int64_t d, int64_t f
     case SWF_OP_SPARSE_FWD: return sparse_fwd_workspace_bytes(M, d, f, G, K);
     case SWF_OP_SPARSE_BWD: return sparse_bwd_workspace_bytes(M, d, f, G, K);
     case SWF_OP_BUCKETS: return buckets_workspace_bytes(M, K, G);
+    case SWF_OP_MLP2_FWD: return 0;
+    case SWF_OP_MLP2_BWD: return round_up((size_t)M * f * esize(dt), 256);
   }
   return 0;
 }
@@ -200,6 +205,14 @@ extern "C" swf_status swf_plan(swf_op op, int64_t M, int64_t d, int64_t f, int32
       p.num_kernels = 4;
       p.flops = 12 * M * d * f;
       p.gemm_tiles = dense_gemm_tiles(op, M, d, f);
+      break;
+    case SWF_OP_MLP2_FWD:
+      p.num_kernels = 2;
+      p.flops = 4 * M * d * f;
+      break;
+    case SWF_OP_MLP2_BWD:
+      p.num_kernels = 4;
+      p.flops = 8 * M * d * f;
       break;
     default:
       sparse_plan(op, M, d, f, G, K, spg, &p);
@@ -264,6 +277,41 @@ extern "C" swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* 
                        (const float*)w_down, (const float*)saved_h, (const float*)saved_a,
                        (const float*)saved_b, (float*)dx, (float*)dw_gate, (float*)dw_up,
                        (float*)dw_down, (float*)workspace, M, d, f, st);
+}
+
+// ------------------------------------------------------------------ LeakyReLU(0.5)^2 MLP
+extern "C" swf_status leaky_relu_sq_mlp_fwd(const void* x, const void* w_up, const void* w_down,
+                                            void* y, void* post, void* act_grad, int64_t M,
+                                            int64_t d, int64_t f, swf_dtype dt, void* stream) {
+  if (any_null({x, w_up, w_down, y, post, act_grad})) return SWF_ERR_INVALID_ARG;
+  swf_status s = check_dense(M, d, f, dt);
+  if (s != SWF_OK) return s;
+  if (!all_aligned({x, w_up, w_down, y, post, act_grad})) return SWF_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == SWF_BF16) return mlp2_fwd_bf16(x, w_up, w_down, y, post, act_grad, M, d, f, st);
+  return mlp2_fwd_f32((const float*)x, (const float*)w_up, (const float*)w_down, (float*)y,
+                      (float*)post, (float*)act_grad, M, d, f, st);
+}
+
+extern "C" swf_status leaky_relu_sq_mlp_bwd(const void* dy, const void* x, const void* w_up,
+                                            const void* w_down, const void* post,
+                                            const void* act_grad, void* dx, void* dw_up,
+                                            void* dw_down, void* workspace, size_t ws_bytes,
+                                            int64_t M, int64_t d, int64_t f, swf_dtype dt,
+                                            void* stream) {
+  if (any_null({dy, x, w_up, w_down, post, act_grad, dx, dw_up, dw_down, workspace}))
+    return SWF_ERR_INVALID_ARG;
+  swf_status s = check_dense(M, d, f, dt);
+  if (s != SWF_OK) return s;
+  if (!all_aligned({dy, x, w_up, w_down, post, act_grad, dx, dw_up, dw_down, workspace}))
+    return SWF_ERR_ALIGNMENT;
+  if (ws_bytes < swf_workspace_bytes(SWF_OP_MLP2_BWD, M, d, f, 0, 0, dt)) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == SWF_BF16)
+    return mlp2_bwd_bf16(dy, x, w_up, w_down, post, act_grad, dx, dw_up, dw_down, workspace, M, d, f, st);
+  return mlp2_bwd_f32((const float*)dy, (const float*)x, (const float*)w_up, (const float*)w_down,
+                      (const float*)post, (const float*)act_grad, (float*)dx, (float*)dw_up,
+                      (float*)dw_down, (float*)workspace, M, d, f, st);
 }
 
 // ------------------------------------------------------------------ status and self test

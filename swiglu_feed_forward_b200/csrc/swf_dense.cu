@@ -180,3 +180,120 @@ swf_status dense_bwd_f32(const float* dy, const float* x, const float* wg, const
 }
 
 }  // namespace swf
+
+// ------------------------------------------------------------------ LeakyReLU(0.5)^2 MLP
+// parameter-golf PR 1105, "Fused MLP Kernels":
+//   U1  pre = x W_up^T, epilogue post = LeakyReLU(0.5)(pre)^2, act_grad    (K = d_model)
+//   U2  y = post W_down^T                                                   (K = hidden)
+//   U3  dpre = (dY W_down) * act_grad, the multiply in the epilogue         (K = d_model)
+//   U4  dx = dpre W_up                                                      (K = hidden)
+//   U5  dW_up = dpre^T x;  U6  dW_down = dY^T post                          (K = M)
+namespace swf {
+
+swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y, void* post,
+                         void* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
+  CUtensorMap tx, twu, tpost, twd;
+  if (!encode_tmap_bf16(&tx, x, d, M, d, 64, 128) || !encode_tmap_bf16(&twu, wu, d, f, d, 64, 128) ||
+      !encode_tmap_bf16(&tpost, post, f, M, f, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 128))
+    return SWF_ERR_LAUNCH;
+  TcGemmArgs u1 = base_args(M, f, 256, d, 2 * kTileM);
+  u1.out0 = post;
+  u1.ld_out = f;
+  u1.aux0 = act_grad;
+  u1.ld_aux = f;
+  swf_status s = launch_tc_pair<256, false, false, false, kEpiLeakySq>(SWF_K_MLP2_UP, tx, twu, twu, EpiMaps{}, u1, st);
+  if (s != SWF_OK) return s;
+  TcGemmArgs u2 = base_args(M, d, 256, f, 2 * kTileM);
+  u2.out0 = y;
+  u2.ld_out = d;
+  return launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_DOWN, tpost, twd, twd, EpiMaps{}, u2, st);
+}
+
+swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const void* wd,
+                         const void* post, const void* act_grad, void* dx, void* dwu, void* dwd,
+                         void* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
+  swf_status s;
+  {  // U3: dpost = dY W_down (B = W_down viewed [K=d rows, N=hidden cols]); * act_grad by TMA epilogue
+    CUtensorMap tdy, twd;
+    EpiMaps e{};
+    if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 64) ||
+        !epi_map(&e.o[0], dpre, f, M, f) || !epi_map(&e.o[2], act_grad, f, M, f))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs u3 = base_args(M, f, 256, d, 2 * kTileM);
+    s = launch_tc_pair<256, false, true, false, kEpiScale, true>(SWF_K_MLP2_DPRE, tdy, twd, twd, e, u3, st);
+    if (s != SWF_OK) return s;
+  }
+  {  // U4: dx = dpre W_up (B = W_up viewed [K=hidden rows, N=d cols], MN-major)
+    CUtensorMap tdp, twu;
+    if (!encode_tmap_bf16(&tdp, dpre, f, M, f, 64, 128) || !encode_tmap_bf16(&twu, wu, d, f, d, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs u4 = base_args(M, d, 256, f, 2 * kTileM);
+    u4.out0 = dx;
+    u4.ld_out = d;
+    s = launch_tc_pair<256, false, true, false, kEpiStore>(SWF_K_MLP2_DX, tdp, twu, twu, EpiMaps{}, u4, st);
+    if (s != SWF_OK) return s;
+  }
+  {  // U5: dW_up = dpre^T x (both MN-major)
+    CUtensorMap tdp, tx;
+    if (!encode_tmap_bf16(&tdp, dpre, f, M, f, 64, 64) || !encode_tmap_bf16(&tx, x, d, M, d, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs u5 = base_args(f, d, 256, M, 2 * kTileM);
+    u5.out0 = dwu;
+    u5.ld_out = d;
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_MLP2_DW_UP, tdp, tx, tx, EpiMaps{}, u5, st);
+    if (s != SWF_OK) return s;
+  }
+  {  // U6: dW_down = dY^T post
+    CUtensorMap tdy, tpost;
+    if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 64) || !encode_tmap_bf16(&tpost, post, f, M, f, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs u6 = base_args(d, f, 256, M, 2 * kTileM);
+    u6.out0 = dwd;
+    u6.ld_out = f;
+    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, tpost, tpost, EpiMaps{}, u6, st);
+  }
+  return s;
+}
+
+swf_status mlp2_fwd_f32(const float* x, const float* wu, const float* wd, float* y, float* post,
+                        float* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
+  SimtArgs u1 = simt_base(M, f, d);
+  u1.A = x, u1.sam = d, u1.sak = 1;
+  u1.B0 = wu, u1.B1 = wu, u1.sbn = d, u1.sbk = 1;
+  u1.out0 = post, u1.ld_out = f, u1.aux0 = act_grad, u1.ld_aux = f;
+  swf_status s = launch_simt<kSimtLeakySq, false>(u1, st);
+  if (s != SWF_OK) return s;
+  SimtArgs u2 = simt_base(M, d, f);
+  u2.A = post, u2.sam = f, u2.sak = 1;
+  u2.B0 = wd, u2.B1 = wd, u2.sbn = f, u2.sbk = 1;
+  u2.out0 = y, u2.ld_out = d;
+  return launch_simt<kSimtStore, false>(u2, st);
+}
+
+swf_status mlp2_bwd_f32(const float* dy, const float* x, const float* wu, const float* wd,
+                        const float* post, const float* act_grad, float* dx, float* dwu,
+                        float* dwd, float* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
+  SimtArgs u3 = simt_base(M, f, d);  // dpre[m, n] = sum_k dY[m, k] W_d[k, n] * act_grad[m, n]
+  u3.A = dy, u3.sam = d, u3.sak = 1;
+  u3.B0 = wd, u3.B1 = wd, u3.sbn = 1, u3.sbk = f;
+  u3.out0 = dpre, u3.ld_out = f, u3.aux0 = const_cast<float*>(act_grad), u3.ld_aux = f;
+  swf_status s = launch_simt<kSimtScale, false>(u3, st);
+  if (s != SWF_OK) return s;
+  SimtArgs u4 = simt_base(M, d, f);  // dx[m, n] = sum_k dpre[m, k] W_u[k, n]
+  u4.A = dpre, u4.sam = f, u4.sak = 1;
+  u4.B0 = wu, u4.B1 = wu, u4.sbn = 1, u4.sbk = d;
+  u4.out0 = dx, u4.ld_out = d;
+  if ((s = launch_simt<kSimtStore, false>(u4, st)) != SWF_OK) return s;
+  SimtArgs u5 = simt_base(f, d, M);  // dW_u[i, n] = sum_m dpre[m, i] x[m, n]
+  u5.A = dpre, u5.sam = 1, u5.sak = f;
+  u5.B0 = x, u5.B1 = x, u5.sbn = 1, u5.sbk = d;
+  u5.out0 = dwu, u5.ld_out = d;
+  if ((s = launch_simt<kSimtStore, false>(u5, st)) != SWF_OK) return s;
+  SimtArgs u6 = simt_base(d, f, M);  // dW_d[i, n] = sum_m dY[m, i] post[m, n]
+  u6.A = dy, u6.sam = 1, u6.sak = d;
+  u6.B0 = post, u6.B1 = post, u6.sbn = 1, u6.sbk = f;
+  u6.out0 = dwd, u6.ld_out = f;
+  return launch_simt<kSimtStore, false>(u6, st);
+}
+
+}  // namespace swf

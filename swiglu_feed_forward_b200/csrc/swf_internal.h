@@ -60,6 +60,18 @@ swf_status dense_bwd_f32(const float* dy, const float* x, const float* wg, const
                          float* dx, float* dwg, float* dwu, float* dwd, float* dgu, int64_t M,
                          int64_t d, int64_t f, cudaStream_t st);
 
+// ---- LeakyReLU(0.5)^2 MLP (swf_dense.cu) ----
+swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y, void* post,
+                         void* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const void* wd,
+                         const void* post, const void* act_grad, void* dx, void* dwu, void* dwd,
+                         void* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+swf_status mlp2_fwd_f32(const float* x, const float* wu, const float* wd, float* y, float* post,
+                        float* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+swf_status mlp2_bwd_f32(const float* dy, const float* x, const float* wu, const float* wd,
+                        const float* post, const float* act_grad, float* dx, float* dwu,
+                        float* dwd, float* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+
 // Tile count and launch shape of the dense bf16 GEMMs (for swf_plan).
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f);
 

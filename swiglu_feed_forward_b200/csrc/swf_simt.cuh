@@ -10,7 +10,14 @@
 
 namespace swf {
 
-enum : int { kSimtStore = 0, kSimtSwiGLU = 1, kSimtSwiGLUInf = 2, kSimtDGate = 3 };
+enum : int {
+  kSimtStore = 0,
+  kSimtSwiGLU = 1,
+  kSimtSwiGLUInf = 2,
+  kSimtDGate = 3,
+  kSimtLeakySq = 4,  // out0 = LeakyReLU(0.5)(C)^2, aux0 = its derivative (2 C or 0.5 C)
+  kSimtScale = 5     // out0 = C * aux0
+};
 
 struct SimtArgs {
   int M, N, K;
@@ -100,6 +107,12 @@ __global__ void __launch_bounds__(256) simt_gemm_f32(const SimtArgs a) {
           a.aux0[m * a.ld_aux + n] = u * s * (1.0f + g * (1.0f - s));
           a.aux1[m * a.ld_aux + n] = g * s;
         }
+      } else if constexpr (EPI == kSimtLeakySq) {
+        const float lk = c > 0.f ? c : 0.5f * c;
+        a.out0[m * a.ld_out + n] = lk * lk;
+        a.aux0[m * a.ld_aux + n] = c > 0.f ? 2.f * c : 0.5f * c;
+      } else if constexpr (EPI == kSimtScale) {
+        a.out0[m * a.ld_out + n] = c * a.aux0[m * a.ld_aux + n];
       } else if constexpr (EPI == kSimtDGate) {
         a.out0[m * a.ld_out + n] = c * a.aux0[m * a.ld_aux + n];
         a.out0[m * a.ld_out + a.d_ff + n] = c * a.aux1[m * a.ld_aux + n];

@@ -28,6 +28,9 @@
 //   kEpiEnergy     per group of energy_p columns: sum |SiLU(C)| (+ bias[g]) -> fp32 out0
 //   kEpiGroupDWgu  per-group [dG|dU]^T X: rows [0,G) -> out0 rows g*G.., [64,64+G) -> out1
 //   kEpiGroupDWd   per-group dY^T h: columns [0,G) -> out0[:, g*G ..]
+//   kEpiLeakySq    C = pre: post = LeakyReLU(0.5)(pre)^2 -> out0, act_grad (2 pre or 0.5 pre)
+//                  -> aux0 (parameter-golf PR 1105, "Fused MLP Kernels")
+//   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,7 +47,9 @@ enum : int {
   kEpiDGate = 3,
   kEpiEnergy = 4,
   kEpiGroupDWgu = 5,
-  kEpiGroupDWd = 6
+  kEpiGroupDWd = 6,
+  kEpiLeakySq = 7,
+  kEpiScale = 8
 };
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
 
@@ -93,7 +98,7 @@ constexpr int tma_epi_outputs() {
 }
 template <int EPI>
 constexpr int tma_epi_aux() {
-  return EPI == kEpiDGate ? 2 : 0;
+  return EPI == kEpiDGate ? 2 : (EPI == kEpiScale ? 1 : 0);
 }
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <int EPI, bool TMA_EPI>
@@ -211,7 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(!B_MN || kBRows % 64 == 0, "MN-major B tiles are whole 64-column boxes");
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
-                                                    EPI == kEpiSwiGLUInf || EPI == kEpiDGate)),
+                                                    EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
+                                                    EPI == kEpiScale)),
                 "TMA epilogue: dense bf16 outputs");
 
   extern __shared__ uint8_t smem_raw[];
@@ -411,7 +417,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int db = aux_issued & 1;
             mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
             tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[2], n_base + c * 32, m_slab, &abar[db]);
-            tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
+            if constexpr (NAUX > 1)
+              tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
           }
           ++aux_issued;
         }
@@ -471,6 +478,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               w[1][i] = pack_bf16x2(av[0], av[1]);
               w[2][i] = pack_bf16x2(bv[0], bv[1]);
             }
+          }
+        } else if constexpr (EPI == kEpiScale) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 av = *reinterpret_cast<const uint4*>(aux + lane * 64 + ((c4 ^ swz) * 16));
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              w[0][c4 * 4 + p] = pack_bf16x2(v0[c4 * 8 + p * 2] * bf16_lo(aw[p]),
+                                             v0[c4 * 8 + p * 2 + 1] * bf16_hi(aw[p]));
           }
         } else if constexpr (EPI == kEpiDGate) {
 #pragma unroll
@@ -609,7 +626,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int n0 = t.nb * BN + c;
           if (!row_ok) continue;
-          if constexpr (EPI == kEpiStore) {
+          if constexpr (EPI == kEpiLeakySq) {
+            __nv_bfloat16* pp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
+            __nv_bfloat16* gp = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux0)) +
+                                (int64_t)m * args.ld_aux + n0;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (n0 + v * 8 + 8 <= args.N) {
+                float post[8], ag[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float pre = acc[v * 8 + e];
+                  const float lk = pre > 0.f ? pre : 0.5f * pre;
+                  post[e] = lk * lk;
+                  ag[e] = pre > 0.f ? 2.f * pre : 0.5f * pre;
+                }
+                store_bf16x8(pp + v * 8, post);
+                store_bf16x8(gp + v * 8, ag);
+              }
+            }
+          } else if constexpr (EPI == kEpiStore) {
             __nv_bfloat16* op =
                 m < args.row_split
                     ? static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0

@@ -20,7 +20,7 @@ from . import api, synth
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", default="step",
-                    choices=["fwd", "fwd_infer", "bwd", "step", "select", "sparse_step"])
+                    choices=["fwd", "fwd_infer", "bwd", "step", "select", "sparse_step", "mlp2_step"])
     ap.add_argument("--M", type=int, default=32768)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--f", type=int, default=5504)
@@ -46,6 +46,10 @@ def main():
     ops["bwd"] = lambda: api.swiglu_ffn_bwd(t["dy"], t["x"], t["w_gate"], t["w_up"], t["w_down"], h, ga, gb,
                                             dx, dwg, dwu, dwd, ws)
     ops["step"] = lambda: (ops["fwd"](), ops["bwd"]())
+    ws2 = torch.empty(max(16, api.workspace_bytes("mlp2_bwd", M, d, f)), device=dev, dtype=torch.uint8)
+    ops["mlp2_step"] = lambda: (
+        api.leaky_relu_sq_mlp_fwd(t["x"], t["w_up"], t["w_down"], y, h, ga),
+        api.leaky_relu_sq_mlp_bwd(t["dy"], t["x"], t["w_up"], t["w_down"], h, ga, dx, dwu, dwd, ws2))
     if a.op in ("select", "sparse_step"):
         ng = f // G
         sub, _ = api.make_subsample_index(f, G, a.spg, a.seed)

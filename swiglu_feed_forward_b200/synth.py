@@ -27,6 +27,10 @@ WORKLOADS = {
             num_active_groups=8, samples_per_group=8, seed=3),
     4: dict(name="infer_bf16_m262144_d2048_f5504", kind="infer", dtype="bf16",
             M=262144, d_model=2048, d_ff=5504, seed=4),
+    # parameter-golf PR 1105's MLP: d_model 512, hidden 1792 (3.5x), LeakyReLU(0.5)^2; its
+    # "302 MB intermediate" of [tokens, 1792] bf16 is about 86K tokens
+    5: dict(name="leaky_relu_sq_mlp_bf16_m86016_d512_f1792", kind="mlp2", dtype="bf16",
+            M=86016, d_model=512, d_ff=1792, seed=5),
 }
 
 _TENSOR_IDS = {"x": 1, "w_gate": 2, "w_up": 3, "w_down": 4, "dy": 5, "bias": 6}
