@@ -112,7 +112,10 @@ swf_status swiglu_ffn_fwd_infer(const void* x, const void* w_gate, const void* w
  * multiplied by the stored activation-gradient factor inside the GEMM epilogue):
  *   dH = dy W_down;  dG = dH * saved_a;  dU = dH * saved_b        (workspace, [M, 2 d_ff])
  *   dx = dG W_gate + dU W_up;  dw_gate = dG^T x;  dw_up = dU^T x;  dw_down = dy^T saved_h.
- * dx [M, d_model]; dw_gate, dw_up [d_ff, d_model]; dw_down [d_model, d_ff] (overwritten). */
+ * dx [M, d_model]; dw_gate, dw_up [d_ff, d_model]; dw_down [d_model, d_ff] (overwritten).  When
+ * a weight gradient has too few output tiles to fill the GPU, its sum over the tokens is split
+ * into fp32 partial sums (in the workspace) that are added in a fixed order, so the result stays
+ * deterministic. */
 swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate, const void* w_up,
                           const void* w_down, const void* saved_h, const void* saved_a,
                           const void* saved_b, void* dx, void* dw_gate, void* dw_up,
@@ -302,7 +305,8 @@ typedef enum swf_kernel_kind {
   SWF_K_MLP2_DPRE = 22,    /* LeakyReLU^2 MLP: (dY W_down) * act_grad */
   SWF_K_MLP2_DX = 23,      /* LeakyReLU^2 MLP: dpre W_up */
   SWF_K_MLP2_DW_UP = 24,   /* LeakyReLU^2 MLP: dpre^T x */
-  SWF_K_NUM_KINDS = 25
+  SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
+  SWF_K_NUM_KINDS = 26
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

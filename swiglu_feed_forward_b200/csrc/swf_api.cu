@@ -163,13 +163,17 @@ extern "C" size_t swf_workspace_bytes(swf_op op, int64_t M, int64_t d, int64_t f
   switch (op) {
     case SWF_OP_FWD: return 0;
     case SWF_OP_FWD_INFER: return round_up((size_t)M * f * esize(dt), 256);
-    case SWF_OP_BWD: return round_up((size_t)M * 2 * f * esize(dt), 256);
+    case SWF_OP_BWD:  // [dG | dU], then the split-K partial planes of the weight gradients
+      return round_up((size_t)M * 2 * f * esize(dt), 256) +
+             (dt == SWF_BF16 ? round_up((size_t)dense_bwd_part_elems(M, d, f) * 4, 256) : 0);
     case SWF_OP_SELECT: return select_workspace_bytes(M, d, f, G, K);
     case SWF_OP_SPARSE_FWD: return sparse_fwd_workspace_bytes(M, d, f, G, K);
     case SWF_OP_SPARSE_BWD: return sparse_bwd_workspace_bytes(M, d, f, G, K);
     case SWF_OP_BUCKETS: return buckets_workspace_bytes(M, K, G);
     case SWF_OP_MLP2_FWD: return 0;
-    case SWF_OP_MLP2_BWD: return round_up((size_t)M * f * esize(dt), 256);
+    case SWF_OP_MLP2_BWD:  // dpre, then the split-K partial planes
+      return round_up((size_t)M * f * esize(dt), 256) +
+             (dt == SWF_BF16 ? round_up((size_t)mlp2_bwd_part_elems(M, d, f) * 4, 256) : 0);
   }
   return 0;
 }
@@ -272,7 +276,10 @@ extern "C" swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == SWF_BF16)
     return dense_bwd_bf16(dy, x, w_gate, w_up, w_down, saved_h, saved_a, saved_b, dx, dw_gate, dw_up,
-                          dw_down, workspace, M, d, f, st);
+                          dw_down, workspace,
+                          reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                   round_up((size_t)M * 2 * f * 2, 256)),
+                          M, d, f, st);
   return dense_bwd_f32((const float*)dy, (const float*)x, (const float*)w_gate, (const float*)w_up,
                        (const float*)w_down, (const float*)saved_h, (const float*)saved_a,
                        (const float*)saved_b, (float*)dx, (float*)dw_gate, (float*)dw_up,
@@ -308,7 +315,10 @@ extern "C" swf_status leaky_relu_sq_mlp_bwd(const void* dy, const void* x, const
   if (ws_bytes < swf_workspace_bytes(SWF_OP_MLP2_BWD, M, d, f, 0, 0, dt)) return SWF_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == SWF_BF16)
-    return mlp2_bwd_bf16(dy, x, w_up, w_down, post, act_grad, dx, dw_up, dw_down, workspace, M, d, f, st);
+    return mlp2_bwd_bf16(dy, x, w_up, w_down, post, act_grad, dx, dw_up, dw_down, workspace,
+                         reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                  round_up((size_t)M * f * 2, 256)),
+                         M, d, f, st);
   return mlp2_bwd_f32((const float*)dy, (const float*)x, (const float*)w_up, (const float*)w_down,
                       (const float*)post, (const float*)act_grad, (float*)dx, (float*)dw_up,
                       (float*)dw_down, (float*)workspace, M, d, f, st);

@@ -9,6 +9,8 @@
 //   K4  dx = dGU [W_g ; W_u]                               (K = 2 d_ff, two B segments)
 //   K5  [dW_g ; dW_u] = dGU^T x                            (K = M)
 //   K6  dW_d = dY^T h                                      (K = M)
+#include <algorithm>
+
 #include "swf_internal.h"
 #include "swf_launch.cuh"
 #include "swf_simt.cuh"
@@ -20,7 +22,80 @@ namespace {
 bool epi_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t row_elems) {
   return encode_tmap_bf16(m, base, cols, rows, row_elems, 32, 32, 64);
 }
+
+// out[m, n] = bf16(sum over splits s = 0, 1, ... of part[s][m][n]) in that fixed order; rows at
+// or past row_split go to out1 (row - row_split).  8 elements per thread.
+__global__ void splitk_reduce_kernel(const float4* __restrict__ part, int64_t plane4, int ks,
+                                     int64_t rows, int64_t cols, int64_t row_split,
+                                     __nv_bfloat16* __restrict__ out0,
+                                     __nv_bfloat16* __restrict__ out1) {
+  const int64_t n8 = rows * cols / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < ks; ++s) {
+      const float4 a = part[s * plane4 + 2 * i], b = part[s * plane4 + 2 * i + 1];
+      acc[0] += a.x, acc[1] += a.y, acc[2] += a.z, acc[3] += a.w;
+      acc[4] += b.x, acc[5] += b.y, acc[6] += b.z, acc[7] += b.w;
+    }
+    const int64_t e = 8 * i, m = e / cols, n = e - m * cols;
+    __nv_bfloat16* dst = m < row_split ? out0 + m * cols + n : out1 + (m - row_split) * cols + n;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+// K splits the planner gives a weight-gradient GEMM of rows x cols over K (pair tiles 256 x 256).
+int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
+  const int64_t tiles = (int64_t)cdiv(rows, 2 * kTileM) * cdiv(cols, 256);
+  const int kb = cdiv(K, kTileK);
+  const int ks = choose_ksplit(tiles, kb, rows * cols);
+  return ks > 1 ? cdiv(kb, cdiv(kb, ks)) : 1;  // no empty trailing split
+}
+
+// Weight-gradient GEMM (both operands MN-major, K = tokens): split-K into fp32 partial planes
+// plus a fixed-order reduction when the planner finds too few output tiles, else direct stores.
+swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
+                     int64_t cols, int64_t K, void* out0, void* out1, int64_t row_split,
+                     float* part, cudaStream_t st) {
+  TcGemmArgs a = base_args(rows, cols, 256, K, 2 * kTileM);
+  const int ks = dw_ksplit(rows, cols, K);
+  if (ks <= 1) {
+    a.out0 = out0;
+    a.out1 = out1;
+    a.row_split = (int)row_split;
+    a.ld_out = cols;
+    return launch_tc_pair<256, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st);
+  }
+  a.ksplit = ks;
+  a.kb_per_split = cdiv(a.kb_total, ks);
+  a.part = part;
+  a.part_plane = rows * cols;
+  swf_status s = launch_tc_pair<256, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st);
+  if (s != SWF_OK) return s;
+  ProfScope prof(SWF_K_SPLITK_REDUCE, st);
+  const int64_t n8 = rows * cols / 8;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 148 * 16));
+  splitk_reduce_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(part), rows * cols / 4,
+                                             ks, rows, cols, row_split,
+                                             static_cast<__nv_bfloat16*>(out0),
+                                             static_cast<__nv_bfloat16*>(out1));
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
+int64_t part_elems(int64_t rows, int64_t cols, int64_t K) {
+  const int ks = dw_ksplit(rows, cols, K);
+  return ks > 1 ? ks * rows * cols : 0;
+}
 }  // namespace
+
+int64_t dense_bwd_part_elems(int64_t M, int64_t d, int64_t f) {
+  return std::max(part_elems(2 * f, d, M), part_elems(d, f, M));
+}
+
+int64_t mlp2_bwd_part_elems(int64_t M, int64_t d, int64_t f) {
+  return std::max(part_elems(f, d, M), part_elems(d, f, M));
+}
 
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f) {
   auto t = [](int64_t m, int64_t n, int64_t bn) { return (int64_t)cdiv(m, kTileM) * cdiv(n, bn); };
@@ -58,8 +133,8 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
 
 swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
                           const void* wd, const void* h, const void* a, const void* b, void* dx,
-                          void* dwg, void* dwu, void* dwd, void* dgu, int64_t M, int64_t d,
-                          int64_t f, cudaStream_t st) {
+                          void* dwg, void* dwu, void* dwd, void* dgu, float* part, int64_t M,
+                          int64_t d, int64_t f, cudaStream_t st) {
   swf_status s;
   {  // K3: dH = dY W_d (B = W_d viewed [K=d rows, N=f cols], MN-major), epilogue * a, * b
     CUtensorMap tdy, twd;
@@ -94,22 +169,14 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     CUtensorMap tdgu, tx;
     if (!encode_tmap_bf16(&tdgu, dgu, 2 * f, M, 2 * f, 64, 64) || !encode_tmap_bf16(&tx, x, d, M, d, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k5 = base_args(2 * f, d, 256, M, 2 * kTileM);
-    k5.out0 = dwg;
-    k5.out1 = dwu;
-    k5.row_split = (int)f;
-    k5.ld_out = d;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_GATE_UP, tdgu, tx, tx, EpiMaps{}, k5, st);
+    s = launch_dw(SWF_K_DW_GATE_UP, tdgu, tx, 2 * f, d, M, dwg, dwu, f, part, st);
     if (s != SWF_OK) return s;
   }
   {  // K6: dW_d = dY^T h: A = dY viewed [K=M rows, d cols] (MN), B = h [K=M rows, f cols] (MN)
     CUtensorMap tdy, th;
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 64) || !encode_tmap_bf16(&th, h, f, M, f, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs k6 = base_args(d, f, 256, M, 2 * kTileM);
-    k6.out0 = dwd;
-    k6.ld_out = f;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, th, th, EpiMaps{}, k6, st);
+    s = launch_dw(SWF_K_DW_DOWN, tdy, th, d, f, M, dwd, dwd, d, part, st);
   }
   return s;
 }
@@ -211,7 +278,7 @@ swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y,
 
 swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const void* wd,
                          const void* post, const void* act_grad, void* dx, void* dwu, void* dwd,
-                         void* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
+                         void* dpre, float* part, int64_t M, int64_t d, int64_t f, cudaStream_t st) {
   swf_status s;
   {  // U3: dpost = dY W_down (B = W_down viewed [K=d rows, N=hidden cols]); * act_grad by TMA epilogue
     CUtensorMap tdy, twd;
@@ -237,20 +304,14 @@ swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const vo
     CUtensorMap tdp, tx;
     if (!encode_tmap_bf16(&tdp, dpre, f, M, f, 64, 64) || !encode_tmap_bf16(&tx, x, d, M, d, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs u5 = base_args(f, d, 256, M, 2 * kTileM);
-    u5.out0 = dwu;
-    u5.ld_out = d;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_MLP2_DW_UP, tdp, tx, tx, EpiMaps{}, u5, st);
+    s = launch_dw(SWF_K_MLP2_DW_UP, tdp, tx, f, d, M, dwu, dwu, f, part, st);
     if (s != SWF_OK) return s;
   }
   {  // U6: dW_down = dY^T post
     CUtensorMap tdy, tpost;
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 64) || !encode_tmap_bf16(&tpost, post, f, M, f, 64, 64))
       return SWF_ERR_LAUNCH;
-    TcGemmArgs u6 = base_args(d, f, 256, M, 2 * kTileM);
-    u6.out0 = dwd;
-    u6.ld_out = f;
-    s = launch_tc_pair<256, true, true, false, kEpiStore>(SWF_K_DW_DOWN, tdy, tpost, tpost, EpiMaps{}, u6, st);
+    s = launch_dw(SWF_K_DW_DOWN, tdy, tpost, d, f, M, dwd, dwd, d, part, st);
   }
   return s;
 }

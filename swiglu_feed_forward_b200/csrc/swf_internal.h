@@ -50,8 +50,8 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
                           cudaStream_t st);
 swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const void* wu,
                           const void* wd, const void* h, const void* a, const void* b, void* dx,
-                          void* dwg, void* dwu, void* dwd, void* dgu, int64_t M, int64_t d,
-                          int64_t f, cudaStream_t st);
+                          void* dwg, void* dwu, void* dwd, void* dgu, float* part, int64_t M,
+                          int64_t d, int64_t f, cudaStream_t st);
 swf_status dense_fwd_f32(const float* x, const float* wg, const float* wu, const float* wd,
                          float* y, float* h, float* a, float* b, int64_t M, int64_t d, int64_t f,
                          bool infer, cudaStream_t st);
@@ -65,12 +65,16 @@ swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y,
                          void* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st);
 swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const void* wd,
                          const void* post, const void* act_grad, void* dx, void* dwu, void* dwd,
-                         void* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+                         void* dpre, float* part, int64_t M, int64_t d, int64_t f, cudaStream_t st);
 swf_status mlp2_fwd_f32(const float* x, const float* wu, const float* wd, float* y, float* post,
                         float* act_grad, int64_t M, int64_t d, int64_t f, cudaStream_t st);
 swf_status mlp2_bwd_f32(const float* dy, const float* x, const float* wu, const float* wd,
                         const float* post, const float* act_grad, float* dx, float* dwu,
                         float* dwd, float* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st);
+
+// fp32 elements of the split-K partial planes the bf16 backward passes need (0: no split).
+int64_t dense_bwd_part_elems(int64_t M, int64_t d, int64_t f);
+int64_t mlp2_bwd_part_elems(int64_t M, int64_t d, int64_t f);
 
 // Tile count and launch shape of the dense bf16 GEMMs (for swf_plan).
 int64_t dense_gemm_tiles(int op, int64_t M, int64_t d, int64_t f);

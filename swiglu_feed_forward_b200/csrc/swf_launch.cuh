@@ -1,6 +1,7 @@
 // Host launcher of the tcgen05 GEMM template, shared by the dense and group-sparse paths.
 #pragma once
 #include <algorithm>
+#include <cmath>
 
 #include "swf_internal.h"
 #include "swf_tc_gemm.cuh"
@@ -43,7 +44,7 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   DevCtx ctx;
   swf_status s = get_ctx(&ctx);
   if (s != SWF_OK) return s;
-  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk;
+  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk * std::max(1, args.ksplit);
   if (tiles == 0) return SWF_OK;
   if (tiles > INT32_MAX) return SWF_ERR_UNSUPPORTED;
   args.status = ctx.status;
@@ -69,6 +70,26 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   ProfScope prof(kind, st);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb0, tb1, em, args) != cudaSuccess) return SWF_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
+// K splits of a pair-mode GEMM with `tiles` output tiles of kb_total k-blocks whose fp32 partial
+// planes hold out_elems elements each: the split that minimises (waves x k-blocks per split) of
+// the GEMM plus the partials' extra HBM traffic, on the 74 clusters of a 148-SM B200 (a host
+// planning constant: the launch itself uses the device's SM count).
+inline int choose_ksplit(int64_t tiles, int kb_total, int64_t out_elems) {
+  constexpr double kClusters = 74.0, kKblockUs = 0.27, kBytesPerUs = 5.0e6;
+  int best = 1;
+  double best_us = std::ceil(tiles / kClusters) * kb_total * kKblockUs;
+  for (int ks = 2; ks <= 16 && kb_total / ks >= 8; ++ks) {
+    const double per = std::ceil((double)kb_total / ks);
+    const double us = std::ceil(tiles * ks / kClusters) * per * kKblockUs +
+                      (8.0 * ks * out_elems + 2.0 * out_elems) / kBytesPerUs;
+    if (us < best_us) {
+      best_us = us;
+      best = ks;
+    }
+  }
+  return best;
 }
 
 // Arguments of a dense GEMM of M x N (N-blocks of n_blk_cols columns) over K, with M-blocks of

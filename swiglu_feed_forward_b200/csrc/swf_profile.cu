@@ -41,7 +41,8 @@ const char* const kNames[SWF_K_NUM_KINDS] = {
     "dw_gate_up",      "dw_down",              "f32_gemm",      "select_gather", "select_score",
     "select_topk",     "buckets",              "sparse_gather", "sparse_up",     "sparse_down",
     "sparse_dgate",    "sparse_dx",            "sparse_dw",     "elementwise",   "pair_sum",
-    "balance",         "mlp2_up",              "mlp2_dpre",     "mlp2_dx",       "mlp2_dw_up"};
+    "balance",         "mlp2_up",              "mlp2_dpre",     "mlp2_dx",       "mlp2_dw_up",
+    "splitk_reduce"};
 
 }  // namespace
 

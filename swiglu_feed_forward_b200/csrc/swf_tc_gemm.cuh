@@ -31,6 +31,8 @@
 //   kEpiLeakySq    C = pre: post = LeakyReLU(0.5)(pre)^2 -> out0, act_grad (2 pre or 0.5 pre)
 //                  -> aux0 (parameter-golf PR 1105, "Fused MLP Kernels")
 //   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
+//   kEpiPartialF32 fp32 C of K-split ks -> part[ks][m][n] (split-K weight gradients; a separate
+//                  kernel sums the splits in a fixed order)
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,7 +51,8 @@ enum : int {
   kEpiGroupDWgu = 5,
   kEpiGroupDWd = 6,
   kEpiLeakySq = 7,
-  kEpiScale = 8
+  kEpiScale = 8,
+  kEpiPartialF32 = 9
 };
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
 
@@ -85,6 +88,10 @@ struct TcGemmArgs {
   const float* bias;      // kEpiEnergy (nullable)
   int energy_p;           // kEpiEnergy: columns per group
   int n_groups;           // kEpiEnergy: groups (columns of out0)
+  int ksplit;             // kModeDense: K splits per output tile (1: none)
+  int kb_per_split;       //   k-blocks of each split (the last may be shorter)
+  float* part;            // kEpiPartialF32: [ksplit][M][N] fp32 partial sums
+  int64_t part_plane;     //   elements per split (M * N)
   int* status;            // device status word
   uint64_t wait_limit_ns;
 };
@@ -147,6 +154,7 @@ struct Tile {
   int mb, nb, grp;
   int a_m, a_k, b_n, b_k;
   int kb;
+  int ks;  // K split (split-K GEMMs)
 };
 
 template <int BN, bool B_DUAL, int MODE>
@@ -165,14 +173,20 @@ __device__ __forceinline__ Tile decode_tile(int tile, const TcGemmArgs& a) {
     t.b_k = s0;
     t.kb = a.seg_rows[t.grp] / kTileK;
   } else {
+    t.ks = 0;
+    if (MODE == kModeDense && a.ksplit > 1) {  // consecutive tiles are the splits of one block
+      t.ks = tile % a.ksplit;
+      tile /= a.ksplit;
+    }
     tile_coords(tile, a.num_m_blk, a.num_n_blk, a.raster, t.mb, t.nb);
     t.grp = MODE == kModeRowGrouped ? a.tile_group[t.mb] : 0;
     const int g = t.grp < 0 ? 0 : t.grp;
+    const int k0 = t.ks * a.kb_per_split * kTileK;
     t.a_m = t.mb * kTileM;
-    t.a_k = 0;
+    t.a_k = k0;
     t.b_n = t.nb * (B_DUAL ? BN / 2 : BN) + g * a.grp_b_n;
-    t.b_k = g * a.grp_b_k;
-    t.kb = a.kb_total;
+    t.b_k = g * a.grp_b_k + k0;
+    t.kb = a.ksplit > 1 ? min(a.kb_per_split, a.kb_total - t.ks * a.kb_per_split) : a.kb_total;
   }
   return t;
 }
@@ -234,8 +248,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_tiles = MODE == kModeKGrouped ? args.num_m_blk * args.num_n_blk * args.n_groups
-                                              : args.num_m_blk * args.num_n_blk;
+  const int num_tiles = MODE == kModeKGrouped
+                            ? args.num_m_blk * args.num_n_blk * args.n_groups
+                            : args.num_m_blk * args.num_n_blk * (args.ksplit > 1 ? args.ksplit : 1);
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
@@ -626,7 +641,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int n0 = t.nb * BN + c;
           if (!row_ok) continue;
-          if constexpr (EPI == kEpiLeakySq) {
+          if constexpr (EPI == kEpiPartialF32) {
+            float* pp = args.part + (int64_t)t.ks * args.part_plane + (int64_t)m * args.N + n0;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              if (n0 + v * 4 + 4 <= args.N)
+                *reinterpret_cast<float4*>(pp + v * 4) =
+                    make_float4(acc[v * 4], acc[v * 4 + 1], acc[v * 4 + 2], acc[v * 4 + 3]);
+          } else if constexpr (EPI == kEpiLeakySq) {
             __nv_bfloat16* pp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
             __nv_bfloat16* gp = static_cast<__nv_bfloat16*>(const_cast<void*>(args.aux0)) +
                                 (int64_t)m * args.ld_aux + n0;
