@@ -263,12 +263,11 @@ swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y,
   if (!encode_tmap_bf16(&tx, x, d, M, d, 64, 128) || !encode_tmap_bf16(&twu, wu, d, f, d, 64, 128) ||
       !encode_tmap_bf16(&tpost, post, f, M, f, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 128))
     return SWF_ERR_LAUNCH;
+  // post and act_grad leave through TMA stores (K = d_model is short, the epilogue dominates)
+  EpiMaps e1{};
+  if (!epi_map(&e1.o[0], post, f, M, f) || !epi_map(&e1.o[1], act_grad, f, M, f)) return SWF_ERR_LAUNCH;
   TcGemmArgs u1 = base_args(M, f, 256, d, 2 * kTileM);
-  u1.out0 = post;
-  u1.ld_out = f;
-  u1.aux0 = act_grad;
-  u1.ld_aux = f;
-  swf_status s = launch_tc_pair<256, false, false, false, kEpiLeakySq>(SWF_K_MLP2_UP, tx, twu, twu, EpiMaps{}, u1, st);
+  swf_status s = launch_tc_pair<256, false, false, false, kEpiLeakySq, true>(SWF_K_MLP2_UP, tx, twu, twu, e1, u1, st);
   if (s != SWF_OK) return s;
   TcGemmArgs u2 = base_args(M, d, 256, f, 2 * kTileM);
   u2.out0 = y;

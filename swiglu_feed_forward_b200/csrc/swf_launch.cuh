@@ -11,9 +11,11 @@ namespace swf {
 inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 
 // Launches tc_gemm_kernel on min(tiles, SMs) persistent CTAs, bracketed for profiling as `kind`.
-template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense>
+template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense,
+          bool TMA_EPI = false>
 swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
-                     const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st) {
+                     const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st,
+                     const EpiMaps& em = EpiMaps{}) {
   DevCtx ctx;
   swf_status s = get_ctx(&ctx);
   if (s != SWF_OK) return s;
@@ -24,13 +26,13 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   args.status = ctx.status;
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE>;
-  constexpr int smem = TcSmem<BN, false, 0>::kBytes;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE, false, TMA_EPI>;
+  constexpr int smem = TcSmem<BN, false, epi_smem_bytes<EPI, TMA_EPI>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
   ProfScope prof(kind, st);
-  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, EpiMaps{}, args);
+  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, em, args);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 

@@ -788,12 +788,12 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     CUtensorMap th, twd;
     if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 256))
       return SWF_ERR_LAUNCH;
+    EpiMaps em{};
+    if (!encode_tmap_bf16(&em.o[0], w.yc, d, sd.rmax, d, 32, 32, 64)) return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, d, 256, G);
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
-    a.out0 = w.yc;
-    a.ld_out = d;
-    s = launch_tc<256, false, false, false, kEpiStore, kModeRowGrouped>(SWF_K_SPARSE_DOWN, th, twd, twd, a, st);
+    s = launch_tc<256, false, false, false, kEpiStore, kModeRowGrouped, true>(SWF_K_SPARSE_DOWN, th, twd, twd, a, st, em);
     if (s != SWF_OK) return s;
   }
   return run_pair_sum(w.yc, v.pair_row, sd, y, st);
@@ -851,9 +851,9 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.a_koff1 = 64;
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
-    a.out0 = w.dxc;
-    a.ld_out = d;
-    s = launch_tc<256, false, true, false, kEpiStore, kModeRowGrouped>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st);
+    EpiMaps em{};
+    if (!encode_tmap_bf16(&em.o[0], w.dxc, d, sd.rmax, d, 32, 32, 64)) return SWF_ERR_LAUNCH;
+    s = launch_tc<256, false, true, false, kEpiStore, kModeRowGrouped, true>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st, em);
     if (s != SWF_OK) return s;
   }
   if ((s = run_pair_sum(w.dxc, v.pair_row, sd, dx, st)) != SWF_OK) return s;

@@ -101,7 +101,7 @@ struct TcGemmArgs {
 // loaded by TMA into the same kind of buffers.
 template <int EPI>
 constexpr int tma_epi_outputs() {
-  return EPI == kEpiSwiGLU ? 3 : (EPI == kEpiDGate ? 2 : 1);
+  return EPI == kEpiSwiGLU ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
 }
 template <int EPI>
 constexpr int tma_epi_aux() {
@@ -231,8 +231,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
                                                     EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
-                                                    EPI == kEpiScale)),
-                "TMA epilogue: dense bf16 outputs");
+                                                    EPI == kEpiScale || EPI == kEpiLeakySq)) ||
+                    (MODE == kModeRowGrouped && EPI == kEpiStore),
+                "TMA epilogue: dense bf16 outputs, or row-grouped plain stores");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -493,6 +494,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               w[1][i] = pack_bf16x2(av[0], av[1]);
               w[2][i] = pack_bf16x2(bv[0], bv[1]);
             }
+          }
+        } else if constexpr (EPI == kEpiLeakySq) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float post[2], ag[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float pre = v0[2 * i + e];
+              const float lk = pre > 0.f ? pre : 0.5f * pre;
+              post[e] = lk * lk;
+              ag[e] = pre > 0.f ? 2.f * pre : 0.5f * pre;
+            }
+            w[0][i] = pack_bf16x2(post[0], post[1]);
+            w[1][i] = pack_bf16x2(ag[0], ag[1]);
           }
         } else if constexpr (EPI == kEpiScale) {
 #pragma unroll
