@@ -30,7 +30,8 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   constexpr int smem = TcSmem<BN, false, epi_smem_bytes<EPI, TMA_EPI>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
-  const int grid = (int)std::min<int64_t>(tiles, ctx.num_sms);
+  const int64_t units = args.unit > 1 ? (tiles + args.unit - 1) / args.unit : tiles;
+  const int grid = (int)std::min<int64_t>(units, ctx.num_sms);
   ProfScope prof(kind, st);
   kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, em, args);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;

@@ -83,6 +83,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// ------------------------------------------------------------------ predicated global access
+// A guarded load or store as one predicated instruction instead of a branch around it (guards in
+// unrolled epilogue loops otherwise become a chain of branches).  A false guard touches no memory.
+__device__ __forceinline__ float ld_global_if(const float* p, bool pred, float otherwise) {
+  float r;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "mov.f32 %0, %3;\n\t"
+      "@q ld.global.f32 %0, [%1];\n\t}"
+      : "=f"(r)
+      : "l"(p), "r"((int)pred), "f"(otherwise)
+      : "memory");
+  return r;
+}
+__device__ __forceinline__ void st_global_if(float* p, float v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "@q st.global.f32 [%0], %1;\n\t}" ::"l"(p),
+      "f"(v), "r"((int)pred)
+      : "memory");
+}
+__device__ __forceinline__ void st_global_if(int32_t* p, int32_t v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "@q st.global.b32 [%0], %1;\n\t}" ::"l"(p),
+      "r"(v), "r"((int)pred)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -191,6 +223,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// tcgen05.wait::ld that also ties the 32 registers of an earlier tmem_ld32 to the wait, so no
+// read of them can be scheduled before the load has completed.
+__device__ __forceinline__ void tmem_ld_wait_regs(float (&v)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+        "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
+        "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]),
+        "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]),
+        "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+      :
+      : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

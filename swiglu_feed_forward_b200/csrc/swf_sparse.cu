@@ -376,20 +376,25 @@ __global__ void select_gather_kernel(const uint4* __restrict__ w, const int32_t*
   }
 }
 
-// One warp per token: K rounds of a warp-wide argmax over the group scores (larger score first,
-// lower group index among equal scores), then the chosen groups written in ascending order.
+// One warp per token: the bias (if any) added to the group scores and written back, then K rounds
+// of a warp-wide argmax over them (larger score first, lower group index among equal scores), then
+// the chosen groups written in ascending order.
 template <int VPL>
-__global__ void topk_kernel(const float* __restrict__ E, int64_t M, int ng, int K,
-                            int32_t* __restrict__ idx) {
+__global__ void topk_kernel(float* __restrict__ E, const float* __restrict__ bias, int64_t M,
+                            int ng, int K, int32_t* __restrict__ idx) {
   const int lane = threadIdx.x & 31;
   const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (m >= M) return;  // uniform per warp
-  const float* row = E + m * ng;
+  float* row = E + m * ng;
   float v[VPL];
 #pragma unroll
   for (int j = 0; j < VPL; ++j) {
     const int c = lane + 32 * j;
     v[j] = c < ng ? row[c] : -INFINITY;
+    if (bias && c < ng) {
+      v[j] += bias[c];
+      row[c] = v[j];
+    }
   }
   uint64_t taken = 0;
   int chosen = 0;
@@ -485,9 +490,10 @@ swf_status run_pair_sum(const void* rows, const int32_t* pair_row, const SparseD
 }
 
 template <int VPL>
-swf_status launch_topk(const float* E, int64_t M, int ng, int K, int32_t* idx, cudaStream_t st) {
+swf_status launch_topk(float* E, const float* bias, int64_t M, int ng, int K, int32_t* idx,
+                       cudaStream_t st) {
   ProfScope prof(SWF_K_SELECT_TOPK, st);
-  topk_kernel<VPL><<<(unsigned)((M + 7) / 8), 256, 0, st>>>(E, M, ng, K, idx);
+  topk_kernel<VPL><<<(unsigned)((M + 7) / 8), 256, 0, st>>>(E, bias, M, ng, K, idx);
   return launched();
 }
 
@@ -632,7 +638,8 @@ extern "C" swf_status grouped_topk_select(const void* x, const void* w_gate,
     if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
     wrows = w.wsub;
   }
-  // scoring GEMM: E[m, c] = sum over the group's P columns of |SiLU(x . w_row)| (+ bias)
+  // scoring GEMM: E[m, c] = sum over the group's P columns of |SiLU(x . w_row)|, then + bias[c]
+  // in the top-k step
   CUtensorMap tx, tw;
   const int64_t ncols = (int64_t)ng * P;
   if (!encode_tmap_bf16(&tx, x, d, M, d, 64, 128) || !encode_tmap_bf16(&tw, wrows, d, ncols, d, 64, 256))
@@ -643,15 +650,29 @@ extern "C" swf_status grouped_topk_select(const void* x, const void* w_gate,
   a.energy_p = P;
   a.n_groups = ng;
   a.bias = bias;
+  if (ng <= kTopKMaxGroups) {
+    // one CTA scores all groups of its 128 tokens, then each epilogue thread selects its token's
+    // groups from the energies it just wrote
+    a.raster = 1;
+    a.unit = a.num_n_blk;
+    if (!energies) {  // energies stay internal: group-major, so a warp's 32 tokens store together
+      a.ld_out = 1;
+      a.ld_grp = M;
+    }
+    a.sel_idx = group_idx;
+    a.sel_k = K;
+    a.energies_out = energies != nullptr;
+    return launch_tc<256, false, false, false, kEpiEnergyTopK>(SWF_K_SELECT_SCORE, tx, tw, tw, a, st);
+  }
   s = launch_tc<256, false, false, false, kEpiEnergy>(SWF_K_SELECT_SCORE, tx, tw, tw, a, st);
   if (s != SWF_OK) return s;
-  if (ng <= 32) return launch_topk<1>(E, M, ng, K, group_idx, st);
-  if (ng <= 64) return launch_topk<2>(E, M, ng, K, group_idx, st);
-  if (ng <= 128) return launch_topk<4>(E, M, ng, K, group_idx, st);
-  if (ng <= 256) return launch_topk<8>(E, M, ng, K, group_idx, st);
-  if (ng <= 512) return launch_topk<16>(E, M, ng, K, group_idx, st);
-  if (ng <= 1024) return launch_topk<32>(E, M, ng, K, group_idx, st);
-  return launch_topk<64>(E, M, ng, K, group_idx, st);
+  if (ng <= 32) return launch_topk<1>(E, bias, M, ng, K, group_idx, st);
+  if (ng <= 64) return launch_topk<2>(E, bias, M, ng, K, group_idx, st);
+  if (ng <= 128) return launch_topk<4>(E, bias, M, ng, K, group_idx, st);
+  if (ng <= 256) return launch_topk<8>(E, bias, M, ng, K, group_idx, st);
+  if (ng <= 512) return launch_topk<16>(E, bias, M, ng, K, group_idx, st);
+  if (ng <= 1024) return launch_topk<32>(E, bias, M, ng, K, group_idx, st);
+  return launch_topk<64>(E, bias, M, ng, K, group_idx, st);
 }
 
 // ------------------------------------------------------------------ bucketing

@@ -25,7 +25,8 @@
 //   kEpiSwiGLUInf  same, h only
 //   kEpiDGate      C = dH: dG = dH*a -> out0[:, n], dU = dH*b -> out0[:, d_ff + n]; columns
 //                  [N, pad_cols) of both halves are written as zeros
-//   kEpiEnergy     per group of energy_p columns: sum |SiLU(C)| (+ bias[g]) -> fp32 out0
+//   kEpiEnergy     per group of energy_p columns: sum |SiLU(C)| -> fp32 out0 (no bias: the top-k
+//                  step adds it)
 //   kEpiGroupDWgu  per-group [dG|dU]^T X: rows [0,G) -> out0 rows g*G.., [64,64+G) -> out1
 //   kEpiGroupDWd   per-group dY^T h: columns [0,G) -> out0[:, g*G ..]
 //   kEpiLeakySq    C = pre: post = LeakyReLU(0.5)(pre)^2 -> out0, act_grad (2 pre or 0.5 pre)
@@ -33,6 +34,10 @@
 //   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
 //   kEpiPartialF32 fp32 C of K-split ks -> part[ks][m][n] (split-K weight gradients; a separate
 //                  kernel sums the splits in a fixed order)
+//   kEpiEnergyTopK kEpiEnergy, and once a CTA has scored every group of its 128 tokens (it owns
+//                  all N-blocks of an M-block, `unit` = num_n_blk) each epilogue thread adds the
+//                  bias to its token's energies and picks the top-k groups -> sel_idx (ascending; larger energy first, lower group
+//                  index among equal energies; NaN never chosen, -1 fills what cannot be chosen)
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -52,8 +57,10 @@ enum : int {
   kEpiGroupDWd = 6,
   kEpiLeakySq = 7,
   kEpiScale = 8,
-  kEpiPartialF32 = 9
+  kEpiPartialF32 = 9,
+  kEpiEnergyTopK = 10
 };
+constexpr int kTopKMaxGroups = 64;  // kEpiEnergyTopK: groups held in registers per token
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
 
 constexpr int kTileM = 128;
@@ -88,6 +95,12 @@ struct TcGemmArgs {
   const float* bias;      // kEpiEnergy (nullable)
   int energy_p;           // kEpiEnergy: columns per group
   int n_groups;           // kEpiEnergy: groups (columns of out0)
+  int64_t ld_grp;         // kEpiEnergy*: stride of out0 between groups (0: 1); ld_out is the
+                          //   stride between tokens (1 with ld_grp = M: group-major energies)
+  int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
+  int sel_k;
+  bool energies_out;      // kEpiEnergyTopK: out0 is returned (gets the bias added in place)
+  int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
   int ksplit;             // kModeDense: K splits per output tile (1: none)
   int kb_per_split;       //   k-blocks of each split (the last may be shorter)
   float* part;            // kEpiPartialF32: [ksplit][M][N] fp32 partial sums
@@ -148,6 +161,13 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
   nb = r / gm;
 }
 
+// The i-th tile of a persistent CTA: units of `unit` consecutive tile ids, dealt out round robin.
+__device__ __forceinline__ int sched_tile(int i, int tile0, int step, int unit) {
+  if (unit <= 1) return tile0 + i * step;
+  const int u = i / unit;
+  return (tile0 + u * step) * unit + (i - u * unit);
+}
+
 // What one tile computes: output block (mb, nb), group (-1: skip), TMA coordinates of its first
 // k-block, and its number of k-blocks.
 struct Tile {
@@ -189,6 +209,72 @@ __device__ __forceinline__ Tile decode_tile(int tile, const TcGemmArgs& a) {
     t.kb = a.ksplit > 1 ? min(a.kb_per_split, a.kb_total - t.ks * a.kb_per_split) : a.kb_total;
   }
   return t;
+}
+
+// Adds the bias (if any) to one token's n_groups (<= kTopKMaxGroups) energies e_row[g * stride]
+// (writing them back if write_back), then selects the top k of them as k rounds of
+// an argmax that prefers the larger energy and, among equal energies, the lower group; NaN is
+// never chosen.  Each round is a pairwise tree over the 64 slots (left = lower groups; the right
+// side wins only with a strictly larger energy or a NaN on the left), so its compares are
+// independent.  The chosen groups go out in ascending order, then -1 for rounds that found nothing.
+__device__ __forceinline__ void topk_row(float* e_row, int64_t stride, int n_groups,
+                                         const float* bias, bool write_back, int k,
+                                         int32_t* out) {
+  const float kNaN = __int_as_float(0x7fc00000);
+  float e[kTopKMaxGroups];
+#pragma unroll
+  for (int j = 0; j < kTopKMaxGroups; ++j) e[j] = ld_global_if(e_row + j * stride, j < n_groups, kNaN);
+  if (bias) {
+#pragma unroll
+    for (int j = 0; j < kTopKMaxGroups; ++j) e[j] += ld_global_if(bias + j, j < n_groups, 0.f);
+    if (write_back) {
+#pragma unroll
+      for (int j = 0; j < kTopKMaxGroups; ++j) st_global_if(e_row + j * stride, e[j], j < n_groups);
+    }
+  }
+  uint64_t taken = 0;
+  for (int r = 0; r < k; ++r) {
+    float v[kTopKMaxGroups / 2];
+    int ix[kTopKMaxGroups / 2];
+#pragma unroll
+    for (int i = 0; i < kTopKMaxGroups / 2; ++i) {
+      const float a = e[2 * i], b = e[2 * i + 1];
+      const bool right = b > a || a != a;
+      v[i] = right ? b : a;
+      ix[i] = right ? 2 * i + 1 : 2 * i;
+    }
+#pragma unroll
+    for (int w = kTopKMaxGroups / 4; w >= 1; w >>= 1) {
+#pragma unroll
+      for (int i = 0; i < w; ++i) {
+        const float a = v[2 * i], b = v[2 * i + 1];
+        const bool right = b > a || a != a;
+        v[i] = right ? b : a;
+        ix[i] = right ? ix[2 * i + 1] : ix[2 * i];
+      }
+    }
+    if (v[0] != v[0]) break;  // only NaN (taken, absent or NaN energies) is left
+    const int win = ix[0];
+    taken |= 1ull << win;
+#pragma unroll
+    for (int j = 0; j < kTopKMaxGroups; ++j) e[j] = j == win ? kNaN : e[j];
+  }
+  int p = 0;
+#pragma unroll
+  for (int j = 0; j < kTopKMaxGroups; ++j) {
+    const bool bit = (taken >> j) & 1ull;
+    st_global_if(out + p, j, bit);
+    p += bit;
+  }
+  for (; p < k; ++p) out[p] = -1;
+}
+
+// ep[(g0 + q) * lg] = v[q] for the NG group sums of a chunk that exist (g0 + q < n_groups).
+template <int NG>
+__device__ __forceinline__ void store_group_sums(float* ep, int64_t lg, int g0, int n_groups,
+                                                 const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < NG; ++q) st_global_if(ep + (g0 + q) * lg, v[q], g0 + q < n_groups);
 }
 
 // 16-byte vector store of 8 bf16 values held as 4 packed words.
@@ -255,6 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int unit_ = args.unit > 1 ? args.unit : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -297,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       // pair mode: every stage completes on the even CTA's barrier
       const uint32_t full_lead = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;
-      for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
+      for (int i_ = 0, tile = tile0 * unit_; ok && tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
         Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
         if (t.grp < 0) continue;
         if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
@@ -355,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int local = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
+      for (int i_ = 0, tile = tile0 * unit_; ok && tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
         const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
         if (t.grp < 0) continue;
         const int buf = local & 1;
@@ -418,7 +505,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t aux_issued = 0, aux_done = 0, chunks = 0;
     int local = 0;
     bool ok = true;
-    for (int tile = tile0; ok && tile < num_tiles; tile += tile_step) {
+    for (int i_ = 0, tile = tile0 * unit_; ok && tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
       Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
       if (t.grp < 0) continue;
       if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
@@ -584,7 +671,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = q * 32 + lane;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     int local = 0;
-    for (int tile = tile0; tile < num_tiles; tile += tile_step) {
+    for (int i_ = 0, tile = tile0 * unit_; tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
       Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
       if (t.grp < 0) continue;
       if (PAIR) t.a_m = t.mb * 2 * kTileM + (int)rank * kTileM;
@@ -641,8 +728,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
+      } else if constexpr (EPI == kEpiEnergy || EPI == kEpiEnergyTopK) {
+        // |SiLU| of each column, summed over aligned runs of P = energy_p = 2^lp columns (lp <= 6),
+        // stored at ep[g * lg] (the bias is added by the top-k step, which reads every energy).  Columns arrive 32 at a time from TMEM (the
+        // next 32 load while these are reduced); pairwise sums pack a chunk's group sums into
+        // v[0 .. 32/P); a 64-column group spans two chunks.
+        float* ep = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
+        const int64_t lg = args.ld_grp ? args.ld_grp : 1;
+        const int lp = __ffs(args.energy_p) - 1;
+        const int lv = lp < 5 ? lp : 5;
+        float run = 0.f;
+        float nxt[32];
+        if (have_acc) tmem_ld32(t_acc, nxt);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          if (have_acc) {
+            tmem_ld_wait_regs(nxt);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = nxt[j];
+            if (c + 32 < BN) tmem_ld32(t_acc + c + 32, nxt);  // warp-uniform: before any row test
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+          if (!row_ok) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fabsf(v[j] * sigmoidf_(v[j]));
+#pragma unroll
+          for (int l = 1, w = 16; l <= 5; ++l, w >>= 1) {
+            if (l <= lv) {
+#pragma unroll
+              for (int j = 0; j < w; ++j) v[j] = v[2 * j] + v[2 * j + 1];
+            }
+          }
+          const int n0 = t.nb * BN + c;
+          const int g0 = n0 >> lp;
+          if (lp == 6) {
+            if ((n0 & 32) == 0) {
+              run = v[0];
+            } else if (g0 < args.n_groups) {
+              ep[g0 * lg] = run + v[0];
+            }
+          } else {
+            switch (lv) {  // a fixed number of group sums per chunk for each group width
+              case 0: store_group_sums<32>(ep, lg, g0, args.n_groups, v); break;
+              case 1: store_group_sums<16>(ep, lg, g0, args.n_groups, v); break;
+              case 2: store_group_sums<8>(ep, lg, g0, args.n_groups, v); break;
+              case 3: store_group_sums<4>(ep, lg, g0, args.n_groups, v); break;
+              case 4: store_group_sums<2>(ep, lg, g0, args.n_groups, v); break;
+              default: store_group_sums<1>(ep, lg, g0, args.n_groups, v); break;
+            }
+          }
+        }
       } else {
-        float run = 0.f;  // kEpiEnergy: running sum of the current group
         static_assert(EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf || BN % 32 == 0, "chunking");
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -719,20 +858,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 st_v4(up + v * 8, 0u, 0u, 0u, 0u);
               }
             }
-          } else if constexpr (EPI == kEpiEnergy) {
-            float* ep = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
-            const int pm = args.energy_p - 1;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float z = acc[j];
-              run += fabsf(z * sigmoidf_(z));
-              const int n = n0 + j;
-              if ((n & pm) == pm) {
-                const int grp = n / args.energy_p;
-                if (grp < args.n_groups) ep[grp] = run + (args.bias ? args.bias[grp] : 0.f);
-                run = 0.f;
-              }
-            }
           } else if constexpr (EPI == kEpiGroupDWgu) {
             const int G = args.group_size;
             __nv_bfloat16* op = nullptr;
@@ -759,6 +884,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       if (PAIR && rank != 0) mbar_arrive_cluster(tempty_lead + buf * 8);
       else mbar_arrive(&tempty[buf]);
+      if constexpr (EPI == kEpiEnergyTopK) {
+        // this thread wrote its token's whole energy row (all N-blocks of the unit): select
+        if (row_ok && t.nb == args.num_n_blk - 1)
+          topk_row(static_cast<float*>(args.out0) + (int64_t)m * args.ld_out,
+                   args.ld_grp ? args.ld_grp : 1, args.n_groups, args.bias, args.energies_out, args.sel_k,
+                   args.sel_idx + (int64_t)m * args.sel_k);
+      }
     }
   }
 

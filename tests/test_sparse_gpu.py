@@ -64,6 +64,10 @@ def test_selection_workload3_full_size():
     (333, 256, 1024, 64, 1, 5, True),      # K = 1, spg not a power of two
     (129, 64, 256, 16, 16, 16, True),      # K = all groups, G = 16
     (64, 48, 4096, 16, 7, 3, False),       # 256 groups, d below one k-block
+    (19244, 128, 1024, 16, 4, None, True),  # 151 token blocks of 4 N-blocks: CTAs take two
+    (300, 64, 768, 16, 5, 2, True),        # 48 groups, P = 2
+    (500, 128, 2048, 64, 4, None, True),   # P = 64: a group spans two 32-column chunks
+    (260, 64, 1024, 32, 3, 1, False),      # P = 1: one sampled column per group
 ])
 def test_selection_small(M, d, f, G, K, spg, use_bias):
     inp = synth.dense_inputs(M, d, f, seed=M + K, dtype=torch.bfloat16, with_dy=False)
@@ -81,6 +85,21 @@ def test_bias_forces_selection():
     bias[[2, 7, 11]] = 1000.0
     idx, _ = select(inp["x"].cuda(), inp["w_gate"].cuda(), G, K, None, bias.cuda())
     assert np.all(idx == np.array([2, 7, 11]))
+
+
+@pytest.mark.parametrize("f,G", [(512, 32), (8192, 64)])  # 16 and 128 groups
+def test_minus_inf_bias_chosen_last(f, G):
+    """Groups whose bias is -inf score -inf: they are taken only when nothing else is left."""
+    M, d = 130, 64
+    ng = f // G
+    K = ng - 2
+    inp = synth.dense_inputs(M, d, f, seed=3, dtype=torch.bfloat16, with_dy=False)
+    bias = torch.zeros(ng)
+    bias[[1, 5, 9]] = -float("inf")
+    idx, E = select(inp["x"].cuda(), inp["w_gate"].cuda(), G, K, None, bias.cuda())
+    np.testing.assert_array_equal(idx, O.topk_groups(E, K))
+    # K = ng - 2 leaves two groups out: two of the three -inf ones (the lower index is kept)
+    assert np.all(idx == np.array([g for g in range(ng) if g not in (5, 9)]))
 
 
 @pytest.mark.parametrize("M,K,ng", [(16384, 8, 64), (1000, 3, 7), (5000, 1, 300), (77, 20, 20)])
