@@ -83,34 +83,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// ------------------------------------------------------------------ predicated global access
-// A guarded load or store as one predicated instruction instead of a branch around it (guards in
-// unrolled epilogue loops otherwise become a chain of branches).  A false guard touches no memory.
-__device__ __forceinline__ float ld_global_if(const float* p, bool pred, float otherwise) {
+// ------------------------------------------------------------------ predicated access
+// A guarded load or store (generic address: global or shared) as one predicated instruction
+// instead of a branch around it (guards in unrolled epilogue loops otherwise become a chain of
+// branches).  A false guard touches no memory.
+__device__ __forceinline__ float ld_if(const float* p, bool pred, float otherwise) {
   float r;
   asm volatile(
       "{\n\t.reg .pred q;\n\t"
       "setp.ne.b32 q, %2, 0;\n\t"
       "mov.f32 %0, %3;\n\t"
-      "@q ld.global.f32 %0, [%1];\n\t}"
+      "@q ld.f32 %0, [%1];\n\t}"
       : "=f"(r)
       : "l"(p), "r"((int)pred), "f"(otherwise)
       : "memory");
   return r;
 }
-__device__ __forceinline__ void st_global_if(float* p, float v, bool pred) {
+__device__ __forceinline__ void st_if(float* p, float v, bool pred) {
   asm volatile(
       "{\n\t.reg .pred q;\n\t"
       "setp.ne.b32 q, %2, 0;\n\t"
-      "@q st.global.f32 [%0], %1;\n\t}" ::"l"(p),
+      "@q st.f32 [%0], %1;\n\t}" ::"l"(p),
       "f"(v), "r"((int)pred)
       : "memory");
 }
-__device__ __forceinline__ void st_global_if(int32_t* p, int32_t v, bool pred) {
+__device__ __forceinline__ void st_if(int32_t* p, int32_t v, bool pred) {
   asm volatile(
       "{\n\t.reg .pred q;\n\t"
       "setp.ne.b32 q, %2, 0;\n\t"
-      "@q st.global.b32 [%0], %1;\n\t}" ::"l"(p),
+      "@q st.b32 [%0], %1;\n\t}" ::"l"(p),
       "r"(v), "r"((int)pred)
       : "memory");
 }

@@ -651,17 +651,14 @@ extern "C" swf_status grouped_topk_select(const void* x, const void* w_gate,
   a.n_groups = ng;
   a.bias = bias;
   if (ng <= kTopKMaxGroups) {
-    // one CTA scores all groups of its 128 tokens, then each epilogue thread selects its token's
-    // groups from the energies it just wrote
+    // one CTA scores all groups of its 128 tokens (energies held in shared memory), then each
+    // epilogue thread selects its token's groups
     a.raster = 1;
     a.unit = a.num_n_blk;
-    if (!energies) {  // energies stay internal: group-major, so a warp's 32 tokens store together
-      a.ld_out = 1;
-      a.ld_grp = M;
-    }
     a.sel_idx = group_idx;
     a.sel_k = K;
-    a.energies_out = energies != nullptr;
+    a.out0 = energies;  // [M][ng] with the bias, only if asked for
+    a.ld_grp = 1;
     return launch_tc<256, false, false, false, kEpiEnergyTopK>(SWF_K_SELECT_SCORE, tx, tw, tw, a, st);
   }
   s = launch_tc<256, false, false, false, kEpiEnergy>(SWF_K_SELECT_SCORE, tx, tw, tw, a, st);

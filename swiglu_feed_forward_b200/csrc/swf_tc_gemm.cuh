@@ -34,10 +34,12 @@
 //   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
 //   kEpiPartialF32 fp32 C of K-split ks -> part[ks][m][n] (split-K weight gradients; a separate
 //                  kernel sums the splits in a fixed order)
-//   kEpiEnergyTopK kEpiEnergy, and once a CTA has scored every group of its 128 tokens (it owns
-//                  all N-blocks of an M-block, `unit` = num_n_blk) each epilogue thread adds the
-//                  bias to its token's energies and picks the top-k groups -> sel_idx (ascending; larger energy first, lower group
-//                  index among equal energies; NaN never chosen, -1 fills what cannot be chosen)
+//   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
+//                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
+//                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
+//                  if not null) and picks the top-k groups -> sel_idx (ascending; larger energy
+//                  first, lower group index among equal energies; NaN never chosen, -1 fills
+//                  what cannot be chosen)
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -99,7 +101,6 @@ struct TcGemmArgs {
                           //   stride between tokens (1 with ld_grp = M: group-major energies)
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
   int sel_k;
-  bool energies_out;      // kEpiEnergyTopK: out0 is returned (gets the bias added in place)
   int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
   int ksplit;             // kModeDense: K splits per output tile (1: none)
   int kb_per_split;       //   k-blocks of each split (the last may be shorter)
@@ -123,7 +124,8 @@ constexpr int tma_epi_aux() {
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <int EPI, bool TMA_EPI>
 constexpr int epi_smem_bytes() {
-  return TMA_EPI ? 4 * (tma_epi_outputs<EPI>() + tma_epi_aux<EPI>()) * 2 * kEpiBox : 0;
+  return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
+                               : (TMA_EPI ? 4 * (tma_epi_outputs<EPI>() + tma_epi_aux<EPI>()) * 2 * kEpiBox : 0);
 }
 
 // Tensor maps of a TMA epilogue: outputs in o[0..], kEpiDGate's a/b factors in o[2], o[3].
@@ -212,58 +214,63 @@ __device__ __forceinline__ Tile decode_tile(int tile, const TcGemmArgs& a) {
 }
 
 // Adds the bias (if any) to one token's n_groups (<= kTopKMaxGroups) energies e_row[g * stride]
-// (writing them back if write_back), then selects the top k of them as k rounds of
-// an argmax that prefers the larger energy and, among equal energies, the lower group; NaN is
-// never chosen.  Each round is a pairwise tree over the 64 slots (left = lower groups; the right
-// side wins only with a strictly larger energy or a NaN on the left), so its compares are
-// independent.  The chosen groups go out in ascending order, then -1 for rounds that found nothing.
-__device__ __forceinline__ void topk_row(float* e_row, int64_t stride, int n_groups,
-                                         const float* bias, bool write_back, int k,
-                                         int32_t* out) {
+// (writing the sums to e_out[g * out_stride] if e_out), then selects the top k of them as k rounds of an argmax that
+// prefers the larger energy and, among equal energies, the lower group; NaN is never chosen.  The
+// energies become order-preserving int keys (NaN, chosen and absent slots: INT_MIN, below -inf),
+// and each round is a pairwise tree over the 64 slots (left = lower groups; the right side wins
+// only with a strictly larger key), so its compares are independent.  The chosen groups go out in
+// ascending order, then -1 for rounds that found nothing.
+__device__ __forceinline__ void topk_row(const float* e_row, int64_t stride, int n_groups,
+                                         const float* bias, float* e_out, int64_t out_stride,
+                                         int k, int32_t* out) {
   const float kNaN = __int_as_float(0x7fc00000);
   float e[kTopKMaxGroups];
 #pragma unroll
-  for (int j = 0; j < kTopKMaxGroups; ++j) e[j] = ld_global_if(e_row + j * stride, j < n_groups, kNaN);
+  for (int j = 0; j < kTopKMaxGroups; ++j) e[j] = ld_if(e_row + j * stride, j < n_groups, kNaN);
   if (bias) {
 #pragma unroll
-    for (int j = 0; j < kTopKMaxGroups; ++j) e[j] += ld_global_if(bias + j, j < n_groups, 0.f);
-    if (write_back) {
+    for (int j = 0; j < kTopKMaxGroups; ++j) e[j] += ld_if(bias + j, j < n_groups, 0.f);
+  }
+  if (e_out) {
 #pragma unroll
-      for (int j = 0; j < kTopKMaxGroups; ++j) st_global_if(e_row + j * stride, e[j], j < n_groups);
-    }
+    for (int j = 0; j < kTopKMaxGroups; ++j) st_if(e_out + j * out_stride, e[j], j < n_groups);
+  }
+  int key[kTopKMaxGroups];
+#pragma unroll
+  for (int j = 0; j < kTopKMaxGroups; ++j) {
+    const int b = __float_as_int(e[j] + 0.0f);  // -0 -> +0: equal energies get equal keys
+    key[j] = e[j] != e[j] ? INT32_MIN : (b >= 0 ? b : b ^ 0x7fffffff);
   }
   uint64_t taken = 0;
   for (int r = 0; r < k; ++r) {
-    float v[kTopKMaxGroups / 2];
+    int v[kTopKMaxGroups / 2];
     int ix[kTopKMaxGroups / 2];
 #pragma unroll
     for (int i = 0; i < kTopKMaxGroups / 2; ++i) {
-      const float a = e[2 * i], b = e[2 * i + 1];
-      const bool right = b > a || a != a;
-      v[i] = right ? b : a;
+      const bool right = key[2 * i + 1] > key[2 * i];
+      v[i] = right ? key[2 * i + 1] : key[2 * i];
       ix[i] = right ? 2 * i + 1 : 2 * i;
     }
 #pragma unroll
     for (int w = kTopKMaxGroups / 4; w >= 1; w >>= 1) {
 #pragma unroll
       for (int i = 0; i < w; ++i) {
-        const float a = v[2 * i], b = v[2 * i + 1];
-        const bool right = b > a || a != a;
-        v[i] = right ? b : a;
+        const bool right = v[2 * i + 1] > v[2 * i];
+        v[i] = right ? v[2 * i + 1] : v[2 * i];
         ix[i] = right ? ix[2 * i + 1] : ix[2 * i];
       }
     }
-    if (v[0] != v[0]) break;  // only NaN (taken, absent or NaN energies) is left
+    if (v[0] == INT32_MIN) break;  // only NaN, chosen or absent slots are left
     const int win = ix[0];
     taken |= 1ull << win;
 #pragma unroll
-    for (int j = 0; j < kTopKMaxGroups; ++j) e[j] = j == win ? kNaN : e[j];
+    for (int j = 0; j < kTopKMaxGroups; ++j) key[j] = j == win ? INT32_MIN : key[j];
   }
   int p = 0;
 #pragma unroll
   for (int j = 0; j < kTopKMaxGroups; ++j) {
     const bool bit = (taken >> j) & 1ull;
-    st_global_if(out + p, j, bit);
+    st_if(out + p, j, bit);
     p += bit;
   }
   for (; p < k; ++p) out[p] = -1;
@@ -274,7 +281,7 @@ template <int NG>
 __device__ __forceinline__ void store_group_sums(float* ep, int64_t lg, int g0, int n_groups,
                                                  const float (&v)[32]) {
 #pragma unroll
-  for (int q = 0; q < NG; ++q) st_global_if(ep + (g0 + q) * lg, v[q], g0 + q < n_groups);
+  for (int q = 0; q < NG; ++q) st_if(ep + (g0 + q) * lg, v[q], g0 + q < n_groups);
 }
 
 // 16-byte vector store of 8 bf16 values held as 4 packed words.
@@ -733,8 +740,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // stored at ep[g * lg] (the bias is added by the top-k step, which reads every energy).  Columns arrive 32 at a time from TMEM (the
         // next 32 load while these are reduced); pairwise sums pack a chunk's group sums into
         // v[0 .. 32/P); a 64-column group spans two chunks.
-        float* ep = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
-        const int64_t lg = args.ld_grp ? args.ld_grp : 1;
+        // kEpiEnergyTopK keeps the energies of its 128 tokens in shared memory, group-major
+        float* ep = EPI == kEpiEnergyTopK
+                        ? reinterpret_cast<float*>(smem + L::kEpiOffset) + row
+                        : static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
+        const int64_t lg = EPI == kEpiEnergyTopK ? kTileM : (args.ld_grp ? args.ld_grp : 1);
         const int lp = __ffs(args.energy_p) - 1;
         const int lv = lp < 5 ? lp : 5;
         float run = 0.f;
@@ -887,9 +897,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if constexpr (EPI == kEpiEnergyTopK) {
         // this thread wrote its token's whole energy row (all N-blocks of the unit): select
         if (row_ok && t.nb == args.num_n_blk - 1)
-          topk_row(static_cast<float*>(args.out0) + (int64_t)m * args.ld_out,
-                   args.ld_grp ? args.ld_grp : 1, args.n_groups, args.bias, args.energies_out, args.sel_k,
-                   args.sel_idx + (int64_t)m * args.sel_k);
+          topk_row(reinterpret_cast<const float*>(smem + L::kEpiOffset) + row, kTileM,
+                   args.n_groups, args.bias,
+                   args.out0 ? static_cast<float*>(args.out0) + (int64_t)m * args.ld_out : nullptr,
+                   args.ld_grp ? args.ld_grp : 1, args.sel_k, args.sel_idx + (int64_t)m * args.sel_k);
       }
     }
   }
