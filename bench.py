@@ -293,7 +293,7 @@ def secondary_infer(api, steps, warmup, world):
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
-def secondary_sparse(api, steps, warmup, world, peak):
+def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     w = synth.WORKLOADS[3]
     M, d, f, G, K, spg = (w[k] for k in ("M", "d_model", "d_ff", "group_size", "num_active_groups",
                                           "samples_per_group"))
@@ -305,7 +305,7 @@ def secondary_sparse(api, steps, warmup, world, peak):
     ng = f // G
     sub, _ = api.make_subsample_index(f, G, spg, w["seed"])
     sub = sub.to(dev)
-    bias = synth.balance_bias(ng, w["seed"]).to(dev)
+    bias = (synth.skewed_balance_bias if skewed else synth.balance_bias)(ng, w["seed"]).to(dev)
     idx = torch.empty(M, K, device=dev, dtype=torch.int32)
     ws_sel = torch.empty(max(16, api.workspace_bytes("select", M, d, f, G, K)), device=dev, dtype=torch.uint8)
     ws_f = torch.empty(max(16, api.workspace_bytes("sparse_fwd", M, d, f, G, K)), device=dev, dtype=torch.uint8)
@@ -327,9 +327,13 @@ def secondary_sparse(api, steps, warmup, world, peak):
     ms = timed(fn, steps, world)
     useful = 2.0 * M * d * ng * spg + 18.0 * M * d * K * G
     tf = useful * steps / (ms / 1e3) / 1e12
-    return {"workload": w["name"], "useful_tflops": round(tf * world, 3),
+    per_group = torch.bincount(idx.flatten().long(), minlength=ng)
+    return {"workload": w["name"] + (" (skewed bias: +0.5 on 2 groups, -0.5 on 2)" if skewed else ""),
+            "useful_tflops": round(tf * world, 3),
             "pct_of_peak": round(100 * tf / peak, 2), "ms_per_step": round(ms / steps, 3),
-            "steps": steps, "useful_flops_per_step": useful}
+            "steps": steps, "useful_flops_per_step": useful,
+            "tokens_per_group": {"max": int(per_group.max()), "mean": round(M * K / ng, 1),
+                                 "min": int(per_group.min())}}
 
 
 def secondary_mlp2(api, steps, warmup, world, peak):
@@ -440,6 +444,11 @@ def run_ours(args, world, rank, local):
             secondary["group_sparse_step"] = secondary_sparse(api, max(3, args.steps // 2), 3, world, peak_sus)
         except Exception as exc:
             secondary["group_sparse_step"] = {"error": str(exc)[:200]}
+        try:
+            secondary["group_sparse_step_skewed"] = secondary_sparse(api, max(3, args.steps // 2), 3, world,
+                                                                     peak_sus, skewed=True)
+        except Exception as exc:  # reported, not fatal
+            secondary["group_sparse_step_skewed"] = {"error": str(exc)[:200]}
         torch.cuda.empty_cache()
         try:
             secondary["leaky_relu_sq_mlp_step"] = secondary_mlp2(api, max(3, args.steps // 2), 3, world, peak_sus)

@@ -76,6 +76,15 @@ def balance_bias(num_groups, seed, lo=-0.1, hi=0.1):
     return u * (hi - lo) + lo
 
 
+def skewed_balance_bias(num_groups, seed):
+    """The load-imbalance variant of the group-sparse workload: the U(-0.1, 0.1) bias with groups
+    0 and 1 raised to +0.5 and groups 2 and 3 lowered to -0.5."""
+    b = balance_bias(num_groups, seed)
+    b[:2] = 0.5
+    b[2:4] = -0.5
+    return b
+
+
 def workload_inputs(cfg_id: int, with_dy=True):
     w = WORKLOADS[cfg_id]
     return dense_inputs(w["M"], w["d_model"], w["d_ff"], w["seed"],

@@ -179,6 +179,22 @@ def test_sparse_small(M, d, f, G, K):
     check_sparse(inp, idx, out, G)
 
 
+def test_sparse_skewed_bias_selection_to_gradients():
+    """The load-imbalance variant: two groups favoured by +0.5, two held back by -0.5."""
+    M, d, f, G, K, spg = 2304, 256, 1024, 64, 4, 8
+    inp = synth.dense_inputs(M, d, f, seed=13, dtype=torch.bfloat16)
+    sub = torch.from_numpy(O.make_subsample_index(f, G, spg, 13)).cuda()
+    bias = synth.skewed_balance_bias(f // G, 13).cuda()
+    idx_dev = api.grouped_topk_select(inp["x"].cuda(), inp["w_gate"].cuda(), G, K, subsample_idx=sub,
+                                      samples_per_group=spg, load_balance_bias=bias)
+    idx = idx_dev.cpu().numpy()
+    counts = np.bincount(idx.ravel(), minlength=f // G)
+    mean = M * K / (f // G)
+    assert min(counts[0], counts[1]) > 1.2 * mean and max(counts[2], counts[3]) < 0.8 * mean
+    out = run_sparse(inp, idx_dev, G)
+    check_sparse(inp, idx, out, G)
+
+
 def test_sparse_all_groups_matches_dense_gpu():
     M, d, f, G = 640, 256, 512, 32
     inp = synth.dense_inputs(M, d, f, seed=5, dtype=torch.bfloat16)
