@@ -355,3 +355,74 @@ def test_leaky_relu_sq_matches_torch_autograd_and_fd():
     loss = lambda: float(np.sum(dys * O.leaky_relu_sq_forward(xs, wus, wds)["y"]))
     b2 = O.leaky_relu_sq_backward(xs, wus, wds, dys)
     _fd_check(loss, [xs, wus, wds], [b2["dx"], b2["dw_up"], b2["dw_down"]])
+
+
+# ---------------------------------------------------------------- FlashFFN multi-head FFN
+def mh_inputs(T=5, H=2, E=3, de=4, dh=6, seed=80):
+    return (rnd((T, H, dh), seed), rnd((H, E, de, dh), seed + 1, dh ** -0.5),
+            rnd((H, E, de, dh), seed + 2, dh ** -0.5), rnd((H, E, de, dh), seed + 3, de ** -0.5),
+            np.random.default_rng(seed + 4).uniform(0.1, 1.0, (T, H, E)), rnd((T, H, dh), seed + 5, 0.1))
+
+
+def test_mhffn_one_head_one_subnetwork_is_dense_swiglu():
+    # H = E = 1, R = 1: the block is a SwiGLU FFN with W_gate = K, W_up = U, W_down = V^T
+    q, k, u, v, _, _ = mh_inputs(T=7, H=1, E=1, de=10, dh=6, seed=81)
+    o = O.mhffn_forward(q, k, u, v, np.ones((7, 1, 1)))["o"]
+    y = O.dense_forward(q[:, 0], k[0, 0], u[0, 0], v[0, 0].T)["y"]
+    np.testing.assert_allclose(o[:, 0], y, rtol=1e-13, atol=1e-14)
+
+
+def test_mhffn_brute_force_scalar_loops():
+    q, k, u, v, r, _ = mh_inputs(T=2, H=2, E=2, de=3, dh=2, seed=82)
+    sil = lambda z: z / (1.0 + math.exp(-z))
+    o = np.zeros_like(q)
+    for t, h, e, j, c in itertools.product(range(2), range(2), range(2), range(3), range(2)):
+        g = sum(q[t, h, i] * k[h, e, j, i] for i in range(2))
+        w = sum(q[t, h, i] * u[h, e, j, i] for i in range(2))
+        o[t, h, c] += r[t, h, e] * sil(g) * w * v[h, e, j, c]
+    np.testing.assert_allclose(O.mhffn_forward(q, k, u, v, r)["o"], o, rtol=1e-13, atol=1e-15)
+
+
+def test_mhffn_additive_over_subnetworks_heads_independent_linear_in_r():
+    q, k, u, v, r, _ = mh_inputs(seed=83)
+    o = O.mhffn_forward(q, k, u, v, r)["o"]
+    parts = sum(O.mhffn_forward(q, k[:, e:e + 1], u[:, e:e + 1], v[:, e:e + 1], r[:, :, e:e + 1])["o"]
+                for e in range(k.shape[1]))
+    np.testing.assert_allclose(o, parts, rtol=1e-12, atol=1e-14)
+    o1 = O.mhffn_forward(q[:, 1:], k[1:], u[1:], v[1:], r[:, 1:])["o"]
+    np.testing.assert_allclose(o[:, 1:], o1, rtol=1e-13)
+    np.testing.assert_allclose(O.mhffn_forward(q, k, u, v, 2.5 * r)["o"], 2.5 * o, rtol=1e-12)
+
+
+def test_mhffn_backward_matches_torch_autograd_and_fd():
+    q, k, u, v, r, do = mh_inputs(T=6, H=2, E=3, de=5, dh=4, seed=84)
+    ts = [torch.from_numpy(a.copy()).requires_grad_(True) for a in (q, k, u, v, r)]
+    F = torch.nn.functional
+    tq, tk, tu, tv, tr = ts
+    act = F.silu(torch.einsum("thd,hefd->thef", tq, tk)) * torch.einsum("thd,hefd->thef", tq, tu)
+    o = torch.einsum("thef,hefd->thd", act * tr[..., None], tv)
+    o.backward(torch.from_numpy(do))
+    np.testing.assert_allclose(O.mhffn_forward(q, k, u, v, r)["o"], o.detach().numpy(), rtol=1e-12, atol=1e-14)
+    bw = O.mhffn_backward(q, k, u, v, r, do)
+    for name, t in zip(("dq", "dk", "du", "dv", "dr"), ts):
+        np.testing.assert_allclose(bw[name], t.grad.numpy(), rtol=1e-11, atol=1e-13)
+    qs, ks, us, vs, rs, dos = (a.copy() for a in mh_inputs(T=2, H=1, E=2, de=2, dh=3, seed=85))
+    loss = lambda: float(np.sum(dos * O.mhffn_forward(qs, ks, us, vs, rs)["o"]))
+    b2 = O.mhffn_backward(qs, ks, us, vs, rs, dos)
+    _fd_check(loss, [qs, ks, us, vs, rs], [b2["dq"], b2["dk"], b2["du"], b2["dv"], b2["dr"]])
+
+
+def test_head_rmsnorm_and_router_weights():
+    z = rnd((4, 3 * 8), 86, 3.0)
+    n = O.head_rmsnorm(z, 3, eps=0.0)
+    np.testing.assert_allclose(np.mean(n * n, axis=-1), 1.0, rtol=1e-12)   # unit RMS per head
+    np.testing.assert_allclose(n * np.sqrt(np.mean(z.reshape(4, 3, 8) ** 2, -1, keepdims=True)),
+                               z.reshape(4, 3, 8), rtol=1e-12)
+    lg = rnd((4, 3, 5), 87)
+    w = O.router_weights(lg)
+    np.testing.assert_allclose(w.sum(-1), 1.0, rtol=1e-13)
+    assert np.all(w > 0)
+    np.testing.assert_allclose(O.router_weights(np.zeros((1, 1, 4))), 0.25)
+    # order follows the logits; sigmoid(0) = 1/2 against sigmoid(large) ~ 1
+    w2 = O.router_weights(np.array([[[0.0, 50.0]]]))
+    np.testing.assert_allclose(w2[0, 0], [1 / 3, 2 / 3], rtol=1e-12)
