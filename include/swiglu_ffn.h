@@ -169,6 +169,26 @@ swf_status leaky_relu_sq_mlp_bwd(const void* dy, const void* x, const void* w_up
                                  void* workspace, size_t workspace_bytes, int64_t M,
                                  int64_t d_model, int64_t hidden, swf_dtype dtype, void* stream);
 
+/* ------------------------------------------------------------------ FlashFFN multi-head FFN */
+
+/* Multi-head FFN forward ("FlashFFN: Multi-Head Decomposition Enables I/O-Aware Feed-Forward
+ * Networks", section "Overview"): for every token t and head h,
+ *   o[t,h,:] = sum_e router[t,h,e] * (SiLU(q[t,h,:] K_{h,e}^T) (.) (q[t,h,:] U_{h,e}^T)) V_{h,e}
+ * with K_{h,e}, U_{h,e}, V_{h,e} the [sub_dim, head_dim] blocks of w_k, w_u, w_v.
+ *   q        [T, num_heads * head_dim]   the heads' normalised input projections (head-minor)
+ *   w_k/u/v  [num_heads * num_sub * sub_dim, head_dim], rows ordered (head, sub-network, row)
+ *   router   [T, num_heads, num_sub] fp32 sub-network weights
+ *   o        [T, num_heads * head_dim]   (overwritten)
+ * One fused kernel: the [T, num_sub * sub_dim] activations of a head stay on chip (TMEM and
+ * shared memory) and never reach HBM.  Device pointers, caller-owned, 16-byte aligned (else
+ * SWF_ERR_ALIGNMENT); asynchronous on `stream`; nothing allocates.  Supported: dtype SWF_BF16
+ * (fp32 accumulation), head_dim 128 (the page's d_h), sub_dim a multiple of 64; anything else
+ * returns SWF_ERR_UNSUPPORTED (there is no fallback). */
+swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void* w_u, const void* w_v,
+                           const float* router, void* o, int64_t T, int32_t num_heads,
+                           int32_t head_dim, int32_t num_sub, int32_t sub_dim, swf_dtype dtype,
+                           void* stream);
+
 /* ------------------------------------------------------------------ group-sparse variant */
 
 /* Subsample index (eugen_sparse README, make_subsample_index; drawn once per layer).  HOST
@@ -306,7 +326,8 @@ typedef enum swf_kernel_kind {
   SWF_K_MLP2_DX = 23,      /* LeakyReLU^2 MLP: dpre W_up */
   SWF_K_MLP2_DW_UP = 24,   /* LeakyReLU^2 MLP: dpre^T x */
   SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
-  SWF_K_NUM_KINDS = 26
+  SWF_K_MHFFN_FWD = 26,    /* FlashFFN multi-head FFN forward (fused, one kernel) */
+  SWF_K_NUM_KINDS = 27
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

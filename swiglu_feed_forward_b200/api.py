@@ -131,6 +131,24 @@ def leaky_relu_sq_mlp_bwd(dy, x, w_up, w_down, saved_post, saved_act_grad, dx=No
     return dx, dw_up, dw_down
 
 
+# ------------------------------------------------------------------ FlashFFN multi-head FFN
+def flash_mhffn_fwd(q, w_k, w_u, w_v, router, o=None, stream=None):
+    """q [T, H, d_h]; w_k, w_u, w_v [H, E, d_e, d_h]; router [T, H, E] fp32.
+    Returns o [T, H, d_h]."""
+    T, H, dh = q.shape
+    E, de = w_k.shape[1], w_k.shape[2]
+    for t in (q, w_k, w_u, w_v, router):
+        if not t.is_contiguous():
+            raise ValueError("flash_mhffn_fwd: tensors must be contiguous")
+    if router.dtype != torch.float32 or tuple(router.shape) != (T, H, E):
+        raise ValueError("flash_mhffn_fwd: router must be fp32 [T, H, E]")
+    o = _empty((T, H, dh), q) if o is None else o
+    _check("flash_mhffn_fwd", _lib.lib().flash_mhffn_fwd(
+        _p(q), _p(w_k), _p(w_u), _p(w_v), _p(router), _p(o), T, H, dh, E, de, _dt(q),
+        _stream(stream)))
+    return o
+
+
 # ------------------------------------------------------------------ group-sparse
 def make_subsample_index(d_ff, group_size, samples_per_group, seed):
     """Host call: returns (int32 CPU tensor [d_ff // group_size, spg], spg)."""

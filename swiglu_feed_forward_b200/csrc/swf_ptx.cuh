@@ -239,6 +239,13 @@ __device__ __forceinline__ void tmem_ld_wait_regs(float (&v)[32]) {
       : "memory");
 }
 
+// Ties 32 registers to this point of the program: reads after it cannot be hoisted above an
+// earlier wait (for the second array of a pair of tcgen05 loads waited on by tmem_ld_wait_regs).
+__device__ __forceinline__ void pin_regs(float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) asm volatile("" : "+f"(v[j])::"memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

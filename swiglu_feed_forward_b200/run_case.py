@@ -20,7 +20,8 @@ from . import api, synth
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", default="step",
-                    choices=["fwd", "fwd_infer", "bwd", "step", "select", "sparse_step", "mlp2_step"])
+                    choices=["fwd", "fwd_infer", "bwd", "step", "select", "sparse_step", "mlp2_step",
+                             "mhffn_fwd"])
     ap.add_argument("--M", type=int, default=32768)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--f", type=int, default=5504)
@@ -28,10 +29,16 @@ def main():
     ap.add_argument("--K", type=int, default=8)
     ap.add_argument("--spg", type=int, default=8)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--T", type=int, default=32768)   # mhffn_fwd: tokens, heads, sub-networks, width
+    ap.add_argument("--H", type=int, default=16)
+    ap.add_argument("--E", type=int, default=15)
+    ap.add_argument("--de", type=int, default=384)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--reps", type=int, default=5)
     a = ap.parse_args()
     dev = torch.device("cuda")
+    if a.op == "mhffn_fwd":
+        return run_mhffn(a, dev)
     M, d, f, G, K = a.M, a.d, a.f, a.G, a.K
     inp = synth.dense_inputs(M, d, f, a.seed, torch.bfloat16)
     t = {k: v.to(dev) for k, v in inp.items()}
@@ -91,6 +98,37 @@ def main():
            "kernels": {k: {"launches": n, "avg_ms": round(v / n, 4), "share": round(v / max(1e-9, sum(x for _, x in kern.values())), 4)}
                        for k, (n, v) in sorted(kern.items(), key=lambda kv: -kv[1][1])}}
     print(json.dumps(out))
+    return 0 if status == 0 else 1
+
+
+def timed_reps(fn, a):
+    for _ in range(a.warmup):
+        fn()
+    torch.cuda.synchronize()
+    api.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    kern = api.profile_read()
+    api.profile_enable(False)
+    return e0.elapsed_time(e1) / a.reps, kern
+
+
+def run_mhffn(a, dev):
+    inp = synth.mhffn_inputs(a.T, a.H, 128, a.E, a.de, a.seed, with_do=False)
+    t = {k: v.to(dev) for k, v in inp.items()}
+    o = torch.empty_like(t["q"])
+    ms, kern = timed_reps(lambda: api.flash_mhffn_fwd(t["q"], t["w_k"], t["w_u"], t["w_v"],
+                                                      t["router"], o), a)
+    flops = 6.0 * a.T * a.H * 128 * a.E * a.de
+    status = api.device_status()
+    print(json.dumps({"op": "mhffn_fwd", "T": a.T, "H": a.H, "E": a.E, "de": a.de,
+                      "ms_per_rep": round(ms, 4), "tflops": round(flops / (ms / 1e3) / 1e12, 1),
+                      "status": status,
+                      "kernels": {k: {"launches": n, "avg_ms": round(v / n, 4)} for k, (n, v) in kern.items()}}))
     return 0 if status == 0 else 1
 
 

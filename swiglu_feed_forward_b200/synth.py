@@ -31,9 +31,14 @@ WORKLOADS = {
     # "302 MB intermediate" of [tokens, 1792] bf16 is about 86K tokens
     5: dict(name="leaky_relu_sq_mlp_bf16_m86016_d512_f1792", kind="mlp2", dtype="bf16",
             M=86016, d_model=512, d_ff=1792, seed=5),
+    # FlashFFN's 1.3B configuration (d_model 2048 = 16 heads x d_h 128, E = 15 sub-networks,
+    # intermediate size 5760 = 15 x 384 per head) at batch 8 x 4096 tokens
+    6: dict(name="flashffn_bf16_t32768_h16_dh128_e15_de384", kind="mhffn", dtype="bf16",
+            T=32768, H=16, d_h=128, E=15, d_e=384, seed=6),
 }
 
-_TENSOR_IDS = {"x": 1, "w_gate": 2, "w_up": 3, "w_down": 4, "dy": 5, "bias": 6}
+_TENSOR_IDS = {"x": 1, "w_gate": 2, "w_up": 3, "w_down": 4, "dy": 5, "bias": 6,
+               "q": 7, "w_k": 8, "w_u": 9, "w_v": 10, "router": 11, "do": 12}
 
 DY_STD = 0.1  # N(0, 1e-2) as a variance
 
@@ -74,6 +79,24 @@ def balance_bias(num_groups, seed, lo=-0.1, hi=0.1):
     """Per-group load-balance bias ~ U(lo, hi), fp32."""
     u = torch.rand(num_groups, generator=_gen(seed, "bias"), dtype=torch.float32)
     return u * (hi - lo) + lo
+
+
+def mhffn_inputs(T, H, d_h, E, d_e, seed, dtype=torch.bfloat16, with_do=True):
+    """Multi-head FFN inputs: q [T, H, d_h] ~ N(0, 1) (unit RMS, as after the per-head norm);
+    w_k, w_u [H, E, d_e, d_h] ~ N(0, 1/d_h); w_v [H, E, d_e, d_h] ~ N(0, 1/d_e); router
+    [T, H, E] fp32, positive and summing to one over E (U(0.05, 1) draws divided by their sum);
+    do [T, H, d_h] ~ N(0, 1e-2).  CPU tensors."""
+    u = torch.rand(T, H, E, generator=_gen(seed, "router"), dtype=torch.float32) * 0.95 + 0.05
+    out = {
+        "q": normal((T, H, d_h), 1.0, seed, "q", dtype),
+        "w_k": normal((H, E, d_e, d_h), d_h ** -0.5, seed, "w_k", dtype),
+        "w_u": normal((H, E, d_e, d_h), d_h ** -0.5, seed, "w_u", dtype),
+        "w_v": normal((H, E, d_e, d_h), d_e ** -0.5, seed, "w_v", dtype),
+        "router": u / u.sum(-1, keepdim=True),
+    }
+    if with_do:
+        out["do"] = normal((T, H, d_h), DY_STD, seed, "do", dtype)
+    return out
 
 
 def skewed_balance_bias(num_groups, seed):

@@ -94,6 +94,19 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.swf_selftest_wait_timeout(0, None) == 1
 
 
+def test_mhffn_argument_errors(lib):
+    BF, F32 = _lib.SWF_BF16, _lib.SWF_F32
+    p, q = C.c_void_p(0x10000), C.c_void_p(0x10008)
+    f = lib.flash_mhffn_fwd
+    assert f(None, p, p, p, p, p, 256, 16, 128, 15, 384, BF, None) == 1   # null pointer
+    assert f(p, p, p, p, p, p, 0, 16, 128, 15, 384, BF, None) == 1        # no tokens
+    assert f(p, p, p, p, p, p, 256, 16, 64, 15, 384, BF, None) == 2       # d_h other than 128
+    assert f(p, p, p, p, p, p, 256, 16, 128, 15, 96, BF, None) == 2       # d_e not a multiple of 64
+    assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, F32, None) == 2     # fp32
+    assert f(p, p, p, p, q, p, 256, 16, 128, 15, 384, BF, None) == 3      # unaligned router
+    assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, 9, None) == 1       # bad dtype
+
+
 @pytest.mark.parametrize("d_ff,G,spg,seed", [(4096, 64, 8, 3), (512, 32, 8, 0), (256, 16, 16, 7),
                                              (3200, 32, 1, 2 ** 63 + 5)])
 def test_subsample_index_matches_oracle(lib, d_ff, G, spg, seed):

@@ -1,0 +1,71 @@
+"""GPU parity of the FlashFFN multi-head FFN forward (one fused kernel) against the fp64
+oracle, through the C ABI: small and ragged token counts, several heads and sub-network widths,
+and sampled token rows of the full 1.3B-configuration workload."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from swiglu_feed_forward_b200 import api, synth
+from tests._util import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run(inp):
+    t = {k: v.cuda() for k, v in inp.items() if k != "do"}
+    o = api.flash_mhffn_fwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    return o
+
+
+def reference(inp, tokens=None):
+    q, k, u, v, r = (f64(inp[n]) for n in ("q", "w_k", "w_u", "w_v", "router"))
+    if tokens is not None:
+        q, r = q[tokens], r[tokens]
+    return O.mhffn_forward(q, k, u, v, r)["o"]
+
+
+@pytest.mark.parametrize("T,H,E,de", [
+    (200, 2, 3, 64),     # ragged token tile, 3 sub-networks of one chunk
+    (1, 1, 1, 64),       # one token, one chunk
+    (128, 1, 2, 128),    # exactly one tile, two chunks per sub-network
+    (300, 3, 2, 192),    # three heads, ragged
+    (700, 2, 5, 384),    # the 1.3B sub-network width, several tiles per head
+])
+def test_small_and_ragged(T, H, E, de):
+    inp = synth.mhffn_inputs(T, H, 128, E, de, seed=T + E, with_do=False)
+    o = run(inp)
+    assert o.shape == (T, H, 128)
+    assert_close("o", f64(o), reference(inp), torch.bfloat16)
+
+
+def test_router_weight_scales_its_subnetwork_only():
+    """A sub-network whose router weight is zero for a token contributes nothing to it."""
+    inp = synth.mhffn_inputs(256, 2, 128, 3, 128, seed=5, with_do=False)
+    inp["router"][:, :, 1] = 0.0
+    o = run(inp)
+    assert_close("o", f64(o), reference(inp), torch.bfloat16)
+    sub = {k: (v[:, [0, 2]].contiguous() if k in ("w_k", "w_u", "w_v") else v) for k, v in inp.items()}
+    sub["router"] = inp["router"][:, :, [0, 2]].contiguous()
+    o2 = run(sub)
+    # exact zeros added to the fp32 accumulator change nothing: bitwise equal
+    assert torch.equal(o.view(torch.int16), o2.view(torch.int16))
+
+
+def test_deterministic():
+    inp = synth.mhffn_inputs(384, 2, 128, 2, 128, seed=9, with_do=False)
+    a, b = run(inp), run(inp)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_full_size_sampled_tokens():
+    """32768 tokens x 16 heads x 15 sub-networks of 384 (the bench's launch configuration):
+    sampled token rows, every head, against the oracle."""
+    w = synth.WORKLOADS[6]
+    inp = synth.mhffn_inputs(w["T"], w["H"], w["d_h"], w["E"], w["d_e"], w["seed"], with_do=False)
+    o = run(inp)
+    rng = np.random.default_rng(0)
+    tokens = np.sort(np.concatenate([rng.choice(w["T"] - 128, 24, replace=False), [w["T"] - 1]]))
+    assert_close("o[tokens]", f64(o)[tokens], reference(inp, tokens), torch.bfloat16)
