@@ -10,13 +10,15 @@
 //
 //   per work unit (head h, 128-token tile), for each 64-column chunk c of the head's E*d_e
 //   sub-network columns:
-//     S_g = Q K_c^T, S_u = Q U_c^T      (tcgen05, M=128 N=64 K=128, fp32 in TMEM, two buffers)
+//     [S_g | S_u] = Q [K_c ; U_c]^T     (tcgen05, M=128 N=128 K=128, fp32 in TMEM, two buffers)
 //     P   = SiLU(S_g) * S_u * R_e       (epilogue warps, bf16 into shared memory, two buffers)
 //     O  += P V_c                       (tcgen05, M=128 N=128 K=64, A from shared memory)
 //   then O (128 TMEM columns) -> bf16 -> HBM.
 //
 // Warp roles: warp 0 lane 0 issues TMA loads (Q once per unit, then a ring of K|U|V chunk
-// stages); warp 1 owns TMEM and lane 0 issues every MMA; warps 2..5 turn S into P and drain O.
+// stages); warp 1 owns TMEM and lane 0 issues every MMA, running the S products two chunks ahead
+// of the PV products; warps 2..9 turn S into P and drain O as two sets of four warps (one per
+// TMEM lane quadrant) that take alternate chunks, so two chunks' epilogues are in flight.
 // Every wait is bounded (status word + abort flag, as in the GEMM template).
 #include <algorithm>
 #include <initializer_list>
@@ -30,16 +32,22 @@ namespace {
 constexpr int kMhTile = 128;     // tokens per unit
 constexpr int kMhDh = 128;       // head width d_h
 constexpr int kMhChunk = 64;     // sub-network columns per chunk
-constexpr int kMhStages = 3;     // K|U|V chunk stages
-constexpr int kMhThreads = 192;
+constexpr int kMhKuStages = 3;   // K|U chunk stages (free once the chunk's S products are done)
+constexpr int kMhVStages = 4;    // V chunk stages (free once its PV product is done)
+constexpr int kMhEpiWarps = 8;  // two sets of four (one warp per TMEM lane quadrant each)
+constexpr int kMhThreads = 64 + 32 * kMhEpiWarps;
+constexpr int kMhEpiThreads = 32 * kMhEpiWarps;
 constexpr int kMhBox = 64 * 64 * 2;                 // one 64 x 64 bf16 TMA box (8 KB)
 constexpr int kMhQBytes = 2 * kMhTile * 64 * 2;     // Q tile: two 128 x 64 boxes
-constexpr int kMhStageBytes = 6 * kMhBox;           // K, U, V chunks: two boxes each
+constexpr int kMhKuBytes = 4 * kMhBox;              // K and U chunks: two boxes each
+constexpr int kMhVBytes = 2 * kMhBox;               // V chunk: two boxes
 constexpr int kMhPBytes = kMhTile * kMhChunk * 2;   // one P buffer (128 x 64 bf16)
-constexpr int kMhStageOff = kMhQBytes;
-constexpr int kMhPOff = kMhStageOff + kMhStages * kMhStageBytes;
+constexpr int kMhKuOff = kMhQBytes;
+constexpr int kMhVOff = kMhKuOff + kMhKuStages * kMhKuBytes;
+constexpr int kMhPOff = kMhVOff + kMhVStages * kMhVBytes;
 constexpr int kMhBarOff = kMhPOff + 2 * kMhPBytes;
 constexpr int kMhSmemBytes = kMhBarOff + 256 + 1024;  // barriers + alignment slack
+static_assert(kMhSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kMhTmemCols = 512;                      // O [0,128); S buffers at 128, 256
 
 struct MhArgs {
@@ -77,9 +85,11 @@ __global__ void __launch_bounds__(kMhThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kMhBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* full = bars + 2;             // [kMhStages]
-  uint64_t* empty = full + kMhStages;    // [kMhStages]
-  uint64_t* s_full = empty + kMhStages;  // [2]
+  uint64_t* ku_full = bars + 2;               // [kMhKuStages]
+  uint64_t* ku_empty = ku_full + kMhKuStages;  // [kMhKuStages]
+  uint64_t* v_full = ku_empty + kMhKuStages;   // [kMhVStages]
+  uint64_t* v_empty = v_full + kMhVStages;     // [kMhVStages]
+  uint64_t* s_full = v_empty + kMhVStages;     // [2]
   uint64_t* s_empty = s_full + 2;        // [2]
   uint64_t* p_full = s_empty + 2;        // [2]
   uint64_t* p_empty = p_full + 2;        // [2]
@@ -94,18 +104,22 @@ __global__ void __launch_bounds__(kMhThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < kMhStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kMhKuStages; ++s) {
+      mbar_init(&ku_full[s], 1);
+      mbar_init(&ku_empty[s], 1);
+    }
+    for (int s = 0; s < kMhVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);
+      mbar_init(&s_empty[b], 128);  // one epilogue set per buffer
       mbar_init(&p_full[b], 128);
       mbar_init(&p_empty[b], 1);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, kMhEpiThreads);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -139,28 +153,34 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         tma_load_2d(smem, &tmQ, h * kMhDh, tt * kMhTile, q_full);
         tma_load_2d(smem + kMhQBytes / 2, &tmQ, h * kMhDh + 64, tt * kMhTile, q_full);
         for (int c = 0; c < args.nch; ++c, ++gc) {
-          const int s = gc % kMhStages;
-          if (!mbar_wait(&empty[s], ((gc / kMhStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
-          uint8_t* st = smem + kMhStageOff + s * kMhStageBytes;
-          mbar_arrive_expect_tx(&full[s], kMhStageBytes);
           const int row = h * rows_per_head + c * kMhChunk;
-          tma_load_2d(st + 0 * kMhBox, &tmK, 0, row, &full[s]);
-          tma_load_2d(st + 1 * kMhBox, &tmK, 64, row, &full[s]);
-          tma_load_2d(st + 2 * kMhBox, &tmU, 0, row, &full[s]);
-          tma_load_2d(st + 3 * kMhBox, &tmU, 64, row, &full[s]);
-          tma_load_2d(st + 4 * kMhBox, &tmV, 0, row, &full[s]);
-          tma_load_2d(st + 5 * kMhBox, &tmV, 64, row, &full[s]);
+          const int s = gc % kMhKuStages;
+          if (!mbar_wait(&ku_empty[s], ((gc / kMhKuStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* ku = smem + kMhKuOff + s * kMhKuBytes;
+          mbar_arrive_expect_tx(&ku_full[s], kMhKuBytes);
+          // [K | U] rows of the chunk per 64-wide d_h half: one N = 128 B operand for both
+          tma_load_2d(ku + 0 * kMhBox, &tmK, 0, row, &ku_full[s]);
+          tma_load_2d(ku + 1 * kMhBox, &tmU, 0, row, &ku_full[s]);
+          tma_load_2d(ku + 2 * kMhBox, &tmK, 64, row, &ku_full[s]);
+          tma_load_2d(ku + 3 * kMhBox, &tmU, 64, row, &ku_full[s]);
+          const int sv = gc % kMhVStages;
+          if (!mbar_wait(&v_empty[sv], ((gc / kMhVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* vs = smem + kMhVOff + sv * kMhVBytes;
+          mbar_arrive_expect_tx(&v_full[sv], kMhVBytes);
+          tma_load_2d(vs, &tmV, 0, row, &v_full[sv]);
+          tma_load_2d(vs + kMhBox, &tmV, 64, row, &v_full[sv]);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16(kMhTile, kMhChunk, 0, 0);
+      constexpr uint32_t kIdescS = idesc_bf16(kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
       constexpr uint32_t kIdescPV = idesc_bf16(kMhTile, kMhDh, 0, 1);
       const uint32_t q_addr = smem_u32(smem);
       const uint32_t p_addr = smem_u32(smem + kMhPOff);
-      const uint32_t st_addr = smem_u32(smem + kMhStageOff);
+      const uint32_t ku_addr = smem_u32(smem + kMhKuOff);
+      const uint32_t v_addr = smem_u32(smem + kMhVOff);
       uint32_t gc = 0;
       int lu = 0;
       bool ok = true, issued = false;
@@ -169,15 +189,17 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         const uint32_t pb = g & 1u;
         if (!mbar_wait(&p_full[pb], (g >> 1) & 1u, ctl)) return false;
         if (first && !mbar_wait(o_empty, (unit_local & 1) ^ 1u, ctl)) return false;
+        const uint32_t sv = g % kMhVStages;
+        if (!mbar_wait(&v_full[sv], (g / kMhVStages) & 1u, ctl)) return false;
         tc_fence_after();
-        const uint32_t vst = st_addr + (g % kMhStages) * kMhStageBytes + 4 * kMhBox;
+        const uint32_t vst = v_addr + sv * kMhVBytes;
 #pragma unroll
         for (int k = 0; k < kMhChunk / 16; ++k)
           umma_bf16(tmem_base, smem_desc_sw128(p_addr + pb * kMhPBytes + k * 32, 16, 1024),
                     smem_desc_sw128(vst + k * 2048, kMhBox, 1024), kIdescPV,
                     (!first || k != 0) ? 1u : 0u);
         umma_commit(&p_empty[pb]);
-        umma_commit(&empty[g % kMhStages]);
+        umma_commit(&v_empty[sv]);
         return true;
       };
       for (int unit = blockIdx.x; ok && unit < args.n_units; unit += gridDim.x, ++lu) {
@@ -185,31 +207,32 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         tc_fence_after();
         const uint32_t gcb = gc;
         for (int c = 0; c < args.nch; ++c, ++gc) {
-          const uint32_t s = gc % kMhStages;
-          if (!mbar_wait(&full[s], (gc / kMhStages) & 1u, ctl)) { ok = false; break; }
+          const uint32_t s = gc % kMhKuStages;
+          if (!mbar_wait(&ku_full[s], (gc / kMhKuStages) & 1u, ctl)) { ok = false; break; }
           const uint32_t sb = gc & 1u;
           if (!mbar_wait(&s_empty[sb], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kst = st_addr + s * kMhStageBytes;
+          const uint32_t kst = ku_addr + s * kMhKuBytes;
           const uint32_t d_s = tmem_base + 128 + sb * 128;
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint64_t qd = smem_desc_sw128(q_addr + kb * (kMhQBytes / 2) + k * 32, 16, 1024);
-              const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
-              umma_bf16(d_s, qd, smem_desc_sw128(kst + kb * kMhBox + k * 32, 16, 1024), kIdescS, acc);
-              umma_bf16(d_s + kMhChunk, qd,
-                        smem_desc_sw128(kst + (2 + kb) * kMhBox + k * 32, 16, 1024), kIdescS, acc);
+              umma_bf16(d_s, qd, smem_desc_sw128(kst + kb * 2 * kMhBox + k * 32, 16, 1024), kIdescS,
+                        (kb | k) != 0 ? 1u : 0u);
             }
           }
           umma_commit(&s_full[sb]);
+          umma_commit(&ku_empty[s]);
           if (c == args.nch - 1) umma_commit(q_empty);  // Q no longer read in this unit
           issued = true;
-          if (c >= 1 && !pv(gc - 1, c == 1, lu)) { ok = false; break; }
+          if (c >= 2 && !pv(gc - 2, c == 2, lu)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!pv(gcb + args.nch - 1, args.nch == 1, lu)) { ok = false; break; }
+        for (int c = args.nch >= 2 ? args.nch - 2 : 0; c < args.nch; ++c)
+          if (!pv(gcb + c, c == 0, lu)) { ok = false; break; }
+        if (!ok) break;
         umma_commit(o_full);
       }
       if (!ok && issued) {
@@ -221,11 +244,12 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue warps 2..5
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // ------------------------------------------------------------ epilogue warps 2..9
+    const int q = warp & 3;            // TMEM lane quadrant this warp may access
+    const int set = (warp - 2) >> 2;   // chunks with (global chunk index & 1) == set; O columns
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t p_addr = smem_u32(smem + kMhPOff);
+    const uint32_t pbuf = smem_u32(smem + kMhPOff) + set * kMhPBytes;
     const int64_t o_ld = (int64_t)args.H * kMhDh;
     uint32_t gc = 0;
     int lu = 0;
@@ -235,48 +259,39 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       const int token = tt * kMhTile + row;
       const bool tok_ok = token < args.T;
       const float* rrow = args.r + ((int64_t)(tok_ok ? token : 0) * args.H + h) * args.E;
-      float rv = 0.f;
-      int e_cur = -1;
       for (int c = 0; c < args.nch; ++c, ++gc) {
-        const uint32_t sb = gc & 1u;
-        const bool ready = mbar_wait(&s_full[sb], (gc >> 1) & 1u, ctl);
+        if ((int)(gc & 1u) != set) continue;
+        const uint32_t use = gc >> 1;
+        const bool ready = mbar_wait(&s_full[set], use & 1u, ctl);
         __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
         if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
         tc_fence_after();
-        const int e = c / args.ch_per_sub;
-        if (e != e_cur) {
-          rv = tok_ok ? rrow[e] : 0.f;
-          e_cur = e;
-        }
-        const uint32_t ts = t_lane + 128 + sb * 128;
+        const uint32_t ts = t_lane + 128 + set * 128;
+        const float rv = tok_ok ? rrow[c / args.ch_per_sub] : 0.f;
         uint32_t w[32];  // this row's 64 P values as bf16 pairs
         float g[32], u[32];
-        tmem_ld32(ts, g);
-        tmem_ld32(ts + kMhChunk, u);
-        tmem_ld_wait_regs(g);
-        pin_regs(u);
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          w[j] = pack_bf16x2(g[2 * j] * sigmoidf_(g[2 * j]) * u[2 * j] * rv,
-                             g[2 * j + 1] * sigmoidf_(g[2 * j + 1]) * u[2 * j + 1] * rv);
-        tmem_ld32(ts + 32, g);
-        tmem_ld32(ts + kMhChunk + 32, u);
-        tmem_ld_wait_regs(g);
-        pin_regs(u);
-        tc_fence_before();
-        mbar_arrive(&s_empty[sb]);  // both halves are in registers: the S buffer is free
+        for (int hh = 0; hh < 2; ++hh) {
+          tmem_ld32(ts + hh * 32, g);
+          tmem_ld32(ts + kMhChunk + hh * 32, u);
+          tmem_ld_wait_regs(g);
+          pin_regs(u);
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(&s_empty[set]);  // the whole S buffer is in registers or P
+          }
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          w[16 + j] = pack_bf16x2(g[2 * j] * sigmoidf_(g[2 * j]) * u[2 * j] * rv,
-                                  g[2 * j + 1] * sigmoidf_(g[2 * j + 1]) * u[2 * j + 1] * rv);
-        if (!mbar_wait(&p_empty[sb], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
-        const uint32_t pbuf = p_addr + sb * kMhPBytes;
+          for (int j = 0; j < 16; ++j)
+            w[hh * 16 + j] = pack_bf16x2(g[2 * j] * sigmoidf_(g[2 * j]) * u[2 * j] * rv,
+                                         g[2 * j + 1] * sigmoidf_(g[2 * j + 1]) * u[2 * j + 1] * rv);
+        }
+        if (!mbar_wait(&p_empty[set], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
           st_shared_v4(pbuf + p_offset(row, c16), w[4 * c16], w[4 * c16 + 1], w[4 * c16 + 2],
                        w[4 * c16 + 3]);
         fence_proxy_async_smem();  // make P visible to the tensor core's reads
-        mbar_arrive(&p_full[sb]);
+        mbar_arrive(&p_full[set]);
       }
       if (!ok) break;
       const bool ready = mbar_wait(o_full, lu & 1, ctl);
@@ -285,7 +300,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       tc_fence_after();
       __nv_bfloat16* orow = args.o + (int64_t)token * o_ld + h * kMhDh;
 #pragma unroll 1
-      for (int cc = 0; cc < kMhDh; cc += 32) {
+      for (int cc = set * 64; cc < set * 64 + 64; cc += 32) {
         float ov[32];
         tmem_ld32(t_lane + cc, ov);
         tmem_ld_wait_regs(ov);
