@@ -68,6 +68,16 @@ __device__ __forceinline__ uint32_t p_offset(int row, int c16) {
   return static_cast<uint32_t>(row * 128 + ((c16 ^ (row & 7)) << 4));
 }
 
+// SiLU(z) = z * sigmoid(z) with sigmoid(z) = (1 + tanh(z / 2)) / 2: one MUFU operation
+// (tanh.approx.f32, relative error about 2^-11) instead of an exponential and a reciprocal.  The
+// epilogue is bound by the MUFU pipe, and P is rounded to bf16 (2^-9) right after.
+__device__ __forceinline__ float silu_tanh(float z) {
+  const float hz = 0.5f * z;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hz));
+  return fmaf(hz, t, hz);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -282,8 +292,8 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           }
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            w[hh * 16 + j] = pack_bf16x2(g[2 * j] * sigmoidf_(g[2 * j]) * u[2 * j] * rv,
-                                         g[2 * j + 1] * sigmoidf_(g[2 * j + 1]) * u[2 * j + 1] * rv);
+            w[hh * 16 + j] = pack_bf16x2(silu_tanh(g[2 * j]) * u[2 * j] * rv,
+                                         silu_tanh(g[2 * j + 1]) * u[2 * j + 1] * rv);
         }
         if (!mbar_wait(&p_empty[set], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
 #pragma unroll
