@@ -8,18 +8,22 @@
 // on chip, so the [tokens, E*d_e] intermediate never reaches HBM.  On B200 it lives in TMEM and
 // shared memory:
 //
-//   per work unit (head h, 128-token tile), for each 64-column chunk c of the head's E*d_e
-//   sub-network columns:
-//     [S_g | S_u] = Q [K_c ; U_c]^T     (tcgen05, M=128 N=128 K=128, fp32 in TMEM, two buffers)
-//     P   = SiLU(S_g) * S_u * R_e       (epilogue warps, bf16 into shared memory, two buffers)
-//     O  += P V_c                       (tcgen05, M=128 N=128 K=64, A from shared memory)
-//   then O (128 TMEM columns) -> bf16 -> HBM.
+//   per work unit (head h, 256 tokens on a pair of CTAs), for each 64-column chunk c of the
+//   head's E*d_e sub-network columns:
+//     [S_g | S_u] = Q [K_c ; U_c]^T   (tcgen05 cta_group::2, M=256 N=128 K=128, fp32 in TMEM)
+//     P   = SiLU(S_g) * S_u * R_e     (epilogue warps, bf16 into shared memory, two buffers)
+//     O  += P V_c                     (tcgen05 cta_group::2, M=256 N=128 K=64, A from smem)
+//   then O (128 TMEM columns per CTA) -> bf16 -> HBM.
 //
-// Warp roles: warp 0 lane 0 issues TMA loads (Q once per unit, then a ring of K|U|V chunk
-// stages); warp 1 owns TMEM and lane 0 issues every MMA, running the S products two chunks ahead
-// of the PV products; warps 2..9 turn S into P and drain O as two sets of four warps (one per
-// TMEM lane quadrant) that take alternate chunks, so two chunks' epilogues are in flight.
-// Every wait is bounded (status word + abort flag, as in the GEMM template).
+// Pair mode: the two CTAs of a cluster each hold 128 tokens of Q and of P and half of each B
+// operand (the even CTA the K rows and V's first 64 d_h columns, the odd CTA the U rows and V's
+// other 64), so each SM stages half of the weight bytes; the even CTA issues every MMA, both
+// CTAs' TMA loads complete on its barriers, and the MMA commits arrive on both CTAs' barriers.
+// Warp roles per CTA: warp 0 lane 0 issues TMA loads (Q once per unit, then rings of K|U and V
+// chunk stages); warp 1 owns TMEM and, in the even CTA, lane 0 issues every MMA, running the S
+// products two chunks ahead of the PV products; warps 2..9 turn S into P and drain O as two sets
+// of four warps (one per TMEM lane quadrant) that take alternate chunks.  No TMA load uses
+// multicast.  Every wait is bounded (status word + abort flag, as in the GEMM template).
 #include <algorithm>
 #include <initializer_list>
 
@@ -29,31 +33,32 @@
 namespace swf {
 namespace {
 
-constexpr int kMhTile = 128;     // tokens per unit
+constexpr int kMhTile = 128;     // tokens per CTA and unit
 constexpr int kMhDh = 128;       // head width d_h
 constexpr int kMhChunk = 64;     // sub-network columns per chunk
-constexpr int kMhKuStages = 3;   // K|U chunk stages (free once the chunk's S products are done)
-constexpr int kMhVStages = 4;    // V chunk stages (free once its PV product is done)
-constexpr int kMhEpiWarps = 8;  // two sets of four (one warp per TMEM lane quadrant each)
+constexpr int kMhKuStages = 4;   // K|U chunk stages (free once the chunk's S products are done)
+constexpr int kMhVStages = 6;    // V chunk stages (free once its PV product is done)
+constexpr int kMhEpiWarps = 8;   // two sets of four (one warp per TMEM lane quadrant each)
 constexpr int kMhThreads = 64 + 32 * kMhEpiWarps;
 constexpr int kMhEpiThreads = 32 * kMhEpiWarps;
 constexpr int kMhBox = 64 * 64 * 2;                 // one 64 x 64 bf16 TMA box (8 KB)
 constexpr int kMhQBytes = 2 * kMhTile * 64 * 2;     // Q tile: two 128 x 64 boxes
-constexpr int kMhKuBytes = 4 * kMhBox;              // K and U chunks: two boxes each
-constexpr int kMhVBytes = 2 * kMhBox;               // V chunk: two boxes
+constexpr int kMhKuBytes = 2 * kMhBox;              // this CTA's half of [K; U]: two d_h boxes
+constexpr int kMhVBytes = kMhBox;                   // this CTA's 64 d_h columns of V
 constexpr int kMhPBytes = kMhTile * kMhChunk * 2;   // one P buffer (128 x 64 bf16)
 constexpr int kMhKuOff = kMhQBytes;
 constexpr int kMhVOff = kMhKuOff + kMhKuStages * kMhKuBytes;
 constexpr int kMhPOff = kMhVOff + kMhVStages * kMhVBytes;
 constexpr int kMhBarOff = kMhPOff + 2 * kMhPBytes;
-constexpr int kMhSmemBytes = kMhBarOff + 256 + 1024;  // barriers + alignment slack
+constexpr int kMhSmemBytes = kMhBarOff + 512 + 1024;  // barriers + alignment slack
 static_assert(kMhSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kMhTmemCols = 512;                      // O [0,128); S buffers at 128, 256
 
 struct MhArgs {
   int T, H, E, de;
   int n_tt;         // 128-token tiles
-  int n_units;      // n_tt * H, head-major
+  int n_pt;         // pairs of token tiles (one per cluster and unit)
+  int n_units;      // n_pt * H, head-major
   int nch;          // 64-column chunks per head (E * de / 64)
   int ch_per_sub;   // chunks per sub-network (de / 64)
   const float* r;   // [T][H][E]
@@ -85,6 +90,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// One arrival per warp on `bar` of the even CTA (locally there, remotely from the odd CTA), after
+// every lane of the warp has reached this point (its TMEM reads waited, its P stores fenced).
+__device__ __forceinline__ void warp_arrive_lead(uint64_t* bar, uint32_t rank, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    if (rank == 0) mbar_arrive(bar);
+    else mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
+  }
+}
+
+// UMMA shared-memory descriptor moved by `bytes` (a multiple of 16): the start address is the
+// low 14-bit field in 16-byte units, which stays below 2^14 for any address in the 227 KB.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 __global__ void __launch_bounds__(kMhThreads, 1)
     mhffn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
@@ -95,23 +114,27 @@ __global__ void __launch_bounds__(kMhThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kMhBarOff);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* ku_full = bars + 2;               // [kMhKuStages]
+  uint64_t* ku_full = bars + 2;                // [kMhKuStages]
   uint64_t* ku_empty = ku_full + kMhKuStages;  // [kMhKuStages]
   uint64_t* v_full = ku_empty + kMhKuStages;   // [kMhVStages]
   uint64_t* v_empty = v_full + kMhVStages;     // [kMhVStages]
   uint64_t* s_full = v_empty + kMhVStages;     // [2]
-  uint64_t* s_empty = s_full + 2;        // [2]
-  uint64_t* p_full = s_empty + 2;        // [2]
-  uint64_t* p_empty = p_full + 2;        // [2]
+  uint64_t* s_empty = s_full + 2;              // [2]
+  uint64_t* p_full = s_empty + 2;              // [2]
+  uint64_t* p_empty = p_full + 2;              // [2]
   uint64_t* o_full = p_empty + 2;
   uint64_t* o_empty = o_full + 1;
   uint64_t* drain = o_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 + 2 * kMhKuStages + 2 * kMhVStages + 11) * 8 + 8 <= 512, "barrier block");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cl = static_cast<int>(blockIdx.x >> 1), n_cl = static_cast<int>(gridDim.x >> 1);
   if (threadIdx.x == 0) {
+    // arrival counts are those of the even CTA's barriers, the only ones waited on with them
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < kMhKuStages; ++s) {
@@ -124,73 +147,75 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);  // one epilogue set per buffer
-      mbar_init(&p_full[b], 128);
+      mbar_init(&s_empty[b], 2 * 4);  // one arrival per warp of a set, in both CTAs
+      mbar_init(&p_full[b], 2 * 4);
       mbar_init(&p_empty[b], 1);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_empty, kMhEpiThreads);
+    mbar_init(o_empty, 2 * kMhEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmU);
+    tma_prefetch_desc(rank == 0 ? &tmK : &tmU);
     tma_prefetch_desc(&tmV);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kMhTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kMhTmemCols);
+    tmem_relinquish_pair();
   }
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
   const int rows_per_head = args.E * args.de;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
+      const uint32_t q_full_lead = map_to_rank(smem_u32(q_full), 0);
+      const uint32_t ku_full_lead = map_to_rank(smem_u32(ku_full), 0);
+      const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
+      const CUtensorMap* tm_b = rank == 0 ? &tmK : &tmU;  // this CTA's half of [K; U]
       uint32_t gc = 0;  // chunks loaded so far (all units)
       int lu = 0;       // units so far
       bool ok = true;
-      for (int unit = blockIdx.x; ok && unit < args.n_units; unit += gridDim.x, ++lu) {
-        const int h = unit / args.n_tt, tt = unit - h * args.n_tt;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+        const int h = unit / args.n_pt, pt = unit - h * args.n_pt;
+        const int tt = 2 * pt + static_cast<int>(rank);  // may lie past the last tile: zero rows
         if (!mbar_wait(q_empty, (lu & 1) ^ 1u, ctl)) { ok = false; break; }
-        mbar_arrive_expect_tx(q_full, kMhQBytes);
-        tma_load_2d(smem, &tmQ, h * kMhDh, tt * kMhTile, q_full);
-        tma_load_2d(smem + kMhQBytes / 2, &tmQ, h * kMhDh + 64, tt * kMhTile, q_full);
+        if (rank == 0) mbar_arrive_expect_tx(q_full, 2 * kMhQBytes);
+        tma_load_2d_pair(smem, &tmQ, h * kMhDh, tt * kMhTile, q_full_lead);
+        tma_load_2d_pair(smem + kMhQBytes / 2, &tmQ, h * kMhDh + 64, tt * kMhTile, q_full_lead);
         for (int c = 0; c < args.nch; ++c, ++gc) {
           const int row = h * rows_per_head + c * kMhChunk;
           const int s = gc % kMhKuStages;
           if (!mbar_wait(&ku_empty[s], ((gc / kMhKuStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
           uint8_t* ku = smem + kMhKuOff + s * kMhKuBytes;
-          mbar_arrive_expect_tx(&ku_full[s], kMhKuBytes);
-          // [K | U] rows of the chunk per 64-wide d_h half: one N = 128 B operand for both
-          tma_load_2d(ku + 0 * kMhBox, &tmK, 0, row, &ku_full[s]);
-          tma_load_2d(ku + 1 * kMhBox, &tmU, 0, row, &ku_full[s]);
-          tma_load_2d(ku + 2 * kMhBox, &tmK, 64, row, &ku_full[s]);
-          tma_load_2d(ku + 3 * kMhBox, &tmU, 64, row, &ku_full[s]);
+          if (rank == 0) mbar_arrive_expect_tx(&ku_full[s], 2 * kMhKuBytes);
+          tma_load_2d_pair(ku, tm_b, 0, row, ku_full_lead + s * 8);
+          tma_load_2d_pair(ku + kMhBox, tm_b, 64, row, ku_full_lead + s * 8);
           const int sv = gc % kMhVStages;
           if (!mbar_wait(&v_empty[sv], ((gc / kMhVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
-          uint8_t* vs = smem + kMhVOff + sv * kMhVBytes;
-          mbar_arrive_expect_tx(&v_full[sv], kMhVBytes);
-          tma_load_2d(vs, &tmV, 0, row, &v_full[sv]);
-          tma_load_2d(vs + kMhBox, &tmV, 64, row, &v_full[sv]);
+          if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kMhVBytes);
+          tma_load_2d_pair(smem + kMhVOff + sv * kMhVBytes, &tmV, static_cast<int>(rank) * 64, row,
+                           v_full_lead + sv * 8);
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16(kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
-      constexpr uint32_t kIdescPV = idesc_bf16(kMhTile, kMhDh, 0, 1);
-      const uint32_t q_addr = smem_u32(smem);
-      const uint32_t p_addr = smem_u32(smem + kMhPOff);
-      const uint32_t ku_addr = smem_u32(smem + kMhKuOff);
-      const uint32_t v_addr = smem_u32(smem + kMhVOff);
+    // ------------------------------------------------------------ UMMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(2 * kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
+      constexpr uint32_t kIdescPV = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
+      // descriptors of the first stage of each operand; every MMA moves them by a constant
+      const uint64_t q_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t p_desc = smem_desc_sw128(smem_u32(smem + kMhPOff), 16, 1024);
+      const uint64_t ku_desc = smem_desc_sw128(smem_u32(smem + kMhKuOff), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kMhVOff), kMhBox, 1024);
       uint32_t gc = 0;
       int lu = 0;
       bool ok = true, issued = false;
@@ -202,17 +227,17 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         const uint32_t sv = g % kMhVStages;
         if (!mbar_wait(&v_full[sv], (g / kMhVStages) & 1u, ctl)) return false;
         tc_fence_after();
-        const uint32_t vst = v_addr + sv * kMhVBytes;
+        const uint64_t pd = desc_add(p_desc, pb * kMhPBytes);
+        const uint64_t vd = desc_add(v_desc, sv * kMhVBytes);
 #pragma unroll
         for (int k = 0; k < kMhChunk / 16; ++k)
-          umma_bf16(tmem_base, smem_desc_sw128(p_addr + pb * kMhPBytes + k * 32, 16, 1024),
-                    smem_desc_sw128(vst + k * 2048, kMhBox, 1024), kIdescPV,
-                    (!first || k != 0) ? 1u : 0u);
-        umma_commit(&p_empty[pb]);
-        umma_commit(&v_empty[sv]);
+          umma_bf16_pair(tmem_base, desc_add(pd, k * 32), desc_add(vd, k * 2048), kIdescPV,
+                         (!first || k != 0) ? 1u : 0u);
+        umma_commit_pair(&p_empty[pb], 3);
+        umma_commit_pair(&v_empty[sv], 3);
         return true;
       };
-      for (int unit = blockIdx.x; ok && unit < args.n_units; unit += gridDim.x, ++lu) {
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
         if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t gcb = gc;
@@ -222,20 +247,18 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           const uint32_t sb = gc & 1u;
           if (!mbar_wait(&s_empty[sb], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kst = ku_addr + s * kMhKuBytes;
+          const uint64_t kd = desc_add(ku_desc, s * kMhKuBytes);
           const uint32_t d_s = tmem_base + 128 + sb * 128;
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t qd = smem_desc_sw128(q_addr + kb * (kMhQBytes / 2) + k * 32, 16, 1024);
-              umma_bf16(d_s, qd, smem_desc_sw128(kst + kb * 2 * kMhBox + k * 32, 16, 1024), kIdescS,
-                        (kb | k) != 0 ? 1u : 0u);
-            }
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_pair(d_s, desc_add(q_desc, kb * (kMhQBytes / 2) + k * 32),
+                             desc_add(kd, kb * kMhBox + k * 32), kIdescS, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(&s_full[sb]);
-          umma_commit(&ku_empty[s]);
-          if (c == args.nch - 1) umma_commit(q_empty);  // Q no longer read in this unit
+          umma_commit_pair(&s_full[sb], 3);
+          umma_commit_pair(&ku_empty[s], 3);
+          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // Q no longer read in this unit
           issued = true;
           if (c >= 2 && !pv(gc - 2, c == 2, lu)) { ok = false; break; }
         }
@@ -243,10 +266,10 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         for (int c = args.nch >= 2 ? args.nch - 2 : 0; c < args.nch; ++c)
           if (!pv(gcb + c, c == 0, lu)) { ok = false; break; }
         if (!ok) break;
-        umma_commit(o_full);
+        umma_commit_pair(o_full, 3);
       }
       if (!ok && issued) {
-        umma_commit(drain);
+        umma_commit_pair(drain, 1);
         WaitCtl quick{abort_flag, args.status, 100000000ull};
         volatile int no_abort = 0;
         quick.abort = &no_abort;
@@ -264,9 +287,9 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     uint32_t gc = 0;
     int lu = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < args.n_units; unit += gridDim.x, ++lu) {
-      const int h = unit / args.n_tt, tt = unit - h * args.n_tt;
-      const int token = tt * kMhTile + row;
+    for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+      const int h = unit / args.n_pt, pt = unit - h * args.n_pt;
+      const int token = (2 * pt + static_cast<int>(rank)) * kMhTile + row;
       const bool tok_ok = token < args.T;
       const float* rrow = args.r + ((int64_t)(tok_ok ? token : 0) * args.H + h) * args.E;
       for (int c = 0; c < args.nch; ++c, ++gc) {
@@ -288,20 +311,21 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           pin_regs(u);
           if (hh == 1) {
             tc_fence_before();
-            mbar_arrive(&s_empty[set]);  // the whole S buffer is in registers or P
+            warp_arrive_lead(&s_empty[set], rank, lane);  // the S buffer is in registers or P
           }
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             w[hh * 16 + j] = pack_bf16x2(silu_tanh(g[2 * j]) * u[2 * j] * rv,
                                          silu_tanh(g[2 * j + 1]) * u[2 * j + 1] * rv);
         }
-        if (!mbar_wait(&p_empty[set], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
+        const bool p_free = mbar_wait(&p_empty[set], (use & 1u) ^ 1u, ctl);
+        if (!__all_sync(0xffffffffu, p_free)) { ok = false; break; }  // warp-uniform exit
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
           st_shared_v4(pbuf + p_offset(row, c16), w[4 * c16], w[4 * c16 + 1], w[4 * c16 + 2],
                        w[4 * c16 + 3]);
         fence_proxy_async_smem();  // make P visible to the tensor core's reads
-        mbar_arrive(&p_full[set]);
+        warp_arrive_lead(&p_full[set], rank, lane);
       }
       if (!ok) break;
       const bool ready = mbar_wait(o_full, lu & 1, ctl);
@@ -323,15 +347,16 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(o_empty);
+      warp_arrive_lead(o_empty, rank, lane);
     }
   }
 
   __syncthreads();
+  cluster_sync();  // the pair's MMAs and TMEM reads are all done
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kMhTmemCols);
+    tmem_dealloc_pair(tmem_base, kMhTmemCols);
   }
 }
 
@@ -373,7 +398,8 @@ extern "C" swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void
   a.E = num_sub;
   a.de = sub_dim;
   a.n_tt = (int)((T + kMhTile - 1) / kMhTile);
-  a.n_units = a.n_tt * num_heads;
+  a.n_pt = (a.n_tt + 1) / 2;
+  a.n_units = a.n_pt * num_heads;
   a.nch = num_sub * sub_dim / kMhChunk;
   a.ch_per_sub = sub_dim / kMhChunk;
   a.r = router;
@@ -383,9 +409,21 @@ extern "C" swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void
   if (cudaFuncSetAttribute(mhffn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kMhSmemBytes) != cudaSuccess)
     return SWF_ERR_LAUNCH;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int grid = std::min(a.n_units, ctx.num_sms);
-  ProfScope prof(SWF_K_MHFFN_FWD, st);
-  mhffn_fwd_kernel<<<grid, kMhThreads, kMhSmemBytes, st>>>(tq, tk, tu, tv, a);
+  const int clusters = std::min(a.n_units, ctx.num_sms / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kMhThreads, 1, 1);
+  cfg.dynamicSmemBytes = kMhSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfScope prof(SWF_K_MHFFN_FWD, cfg.stream);
+  if (cudaLaunchKernelEx(&cfg, mhffn_fwd_kernel, tq, tk, tu, tv, a) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
