@@ -19,11 +19,13 @@
 // operand (the even CTA the K rows and V's first 64 d_h columns, the odd CTA the U rows and V's
 // other 64), so each SM stages half of the weight bytes; the even CTA issues every MMA, both
 // CTAs' TMA loads complete on its barriers, and the MMA commits arrive on both CTAs' barriers.
-// Warp roles per CTA: warp 0 lane 0 issues TMA loads (Q once per unit, then rings of K|U and V
-// chunk stages); warp 1 owns TMEM and, in the even CTA, lane 0 issues every MMA, running the S
-// products two chunks ahead of the PV products; warps 2..9 turn S into P and drain O as two sets
-// of four warps (one per TMEM lane quadrant) that take alternate chunks.  No TMA load uses
-// multicast.  Every wait is bounded (status word + abort flag, as in the GEMM template).
+// Warp roles per CTA: warp 0 lane 0 issues the TMA loads of Q (once per unit) and of the K|U
+// chunk ring, warp 3 lane 0 those of the V chunk ring; warp 1 owns TMEM and, in the even CTA,
+// lane 0 issues the S products; warp 2 lane 0 (even CTA) issues the PV products; warps 4..11
+// turn S into P and drain O as two sets of four
+// warps (one per TMEM lane quadrant) that take alternate chunks.  A thread issues about one
+// tcgen05.mma per 60-90 cycles, close to the 64 tensor cycles of each product here, so the S and
+// PV products come from two threads.  No TMA load uses multicast.  Every wait is bounded (status word + abort flag, as in the GEMM template).
 #include <algorithm>
 #include <initializer_list>
 
@@ -39,7 +41,7 @@ constexpr int kMhChunk = 64;     // sub-network columns per chunk
 constexpr int kMhKuStages = 4;   // K|U chunk stages (free once the chunk's S products are done)
 constexpr int kMhVStages = 6;    // V chunk stages (free once its PV product is done)
 constexpr int kMhEpiWarps = 8;   // two sets of four (one warp per TMEM lane quadrant each)
-constexpr int kMhThreads = 64 + 32 * kMhEpiWarps;
+constexpr int kMhThreads = 128 + 32 * kMhEpiWarps;  // 2 producers, S and PV issuers, epilogue
 constexpr int kMhEpiThreads = 32 * kMhEpiWarps;
 constexpr int kMhBox = 64 * 64 * 2;                 // one 64 x 64 bf16 TMA box (8 KB)
 constexpr int kMhQBytes = 2 * kMhTile * 64 * 2;     // Q tile: two 128 x 64 boxes
@@ -49,10 +51,12 @@ constexpr int kMhPBytes = kMhTile * kMhChunk * 2;   // one P buffer (128 x 64 bf
 constexpr int kMhKuOff = kMhQBytes;
 constexpr int kMhVOff = kMhKuOff + kMhKuStages * kMhKuBytes;
 constexpr int kMhPOff = kMhVOff + kMhVStages * kMhVBytes;
-constexpr int kMhBarOff = kMhPOff + 2 * kMhPBytes;
+constexpr int kMhPBufs = 4;                         // P buffers: two per epilogue set
+constexpr int kMhBarOff = kMhPOff + kMhPBufs * kMhPBytes;
 constexpr int kMhSmemBytes = kMhBarOff + 512 + 1024;  // barriers + alignment slack
 static_assert(kMhSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kMhTmemCols = 512;                      // O [0,128); S buffers at 128, 256
+constexpr int kMhSBufs = 3;                           // S buffers (TMEM: O 128 + 3 x 128 = 512)
+constexpr int kMhTmemCols = 512;                      // O [0,128); S buffers at 128, 256, 384
 
 struct MhArgs {
   int T, H, E, de;
@@ -92,17 +96,27 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 // One arrival per warp on `bar` of the even CTA (locally there, remotely from the odd CTA), after
 // every lane of the warp has reached this point (its TMEM reads waited, its P stores fenced).
+// Every signal sent this way releases data of the arriving CTA's own SM (see mbar_arrive_remote).
 __device__ __forceinline__ void warp_arrive_lead(uint64_t* bar, uint32_t rank, int lane) {
   __syncwarp();
   if (lane == 0) {
     if (rank == 0) mbar_arrive(bar);
-    else mbar_arrive_cluster(map_to_rank(smem_u32(bar), 0));
+    else mbar_arrive_remote(map_to_rank(smem_u32(bar), 0));
   }
 }
 
 // UMMA shared-memory descriptor moved by `bytes` (a multiple of 16): the start address is the
 // low 14-bit field in 16-byte units, which stays below 2^14 for any address in the 227 KB.
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
+// After an aborted wait: lets this thread's MMAs in flight finish (bounded) before the CTA leaves.
+__device__ __forceinline__ void drain_mma(uint64_t* bar, volatile int* abort_flag, int* status) {
+  umma_commit_pair(bar, 1);
+  WaitCtl quick{abort_flag, status, 100000000ull};
+  volatile int no_abort = 0;
+  quick.abort = &no_abort;
+  mbar_wait(bar, 0, quick);
+}
 
 __global__ void __launch_bounds__(kMhThreads, 1)
     mhffn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -118,16 +132,17 @@ __global__ void __launch_bounds__(kMhThreads, 1)
   uint64_t* ku_empty = ku_full + kMhKuStages;  // [kMhKuStages]
   uint64_t* v_full = ku_empty + kMhKuStages;   // [kMhVStages]
   uint64_t* v_empty = v_full + kMhVStages;     // [kMhVStages]
-  uint64_t* s_full = v_empty + kMhVStages;     // [2]
-  uint64_t* s_empty = s_full + 2;              // [2]
-  uint64_t* p_full = s_empty + 2;              // [2]
-  uint64_t* p_empty = p_full + 2;              // [2]
-  uint64_t* o_full = p_empty + 2;
+  uint64_t* s_full = v_empty + kMhVStages;     // [kMhSBufs]
+  uint64_t* s_empty = s_full + kMhSBufs;       // [kMhSBufs]
+  uint64_t* p_full = s_empty + kMhSBufs;       // [kMhPBufs]
+  uint64_t* p_empty = p_full + kMhPBufs;       // [kMhPBufs]
+  uint64_t* o_full = p_empty + kMhPBufs;
   uint64_t* o_empty = o_full + 1;
-  uint64_t* drain = o_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = o_empty + 1;  // [2]: one per issuing thread
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert((2 + 2 * kMhKuStages + 2 * kMhVStages + 11) * 8 + 8 <= 512, "barrier block");
+  static_assert((2 + 2 * kMhKuStages + 2 * kMhVStages + 2 * kMhSBufs + 2 * kMhPBufs + 4) * 8 + 8 <= 512,
+                "barrier block");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -145,15 +160,18 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kMhSBufs; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&s_empty[b], 2 * 4);  // one arrival per warp of a set, in both CTAs
+    }
+    for (int b = 0; b < kMhPBufs; ++b) {
       mbar_init(&p_full[b], 2 * 4);
       mbar_init(&p_empty[b], 1);
     }
     mbar_init(o_full, 1);
     mbar_init(o_empty, 2 * kMhEpiWarps);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,7 +196,6 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     if (lane == 0) {
       const uint32_t q_full_lead = map_to_rank(smem_u32(q_full), 0);
       const uint32_t ku_full_lead = map_to_rank(smem_u32(ku_full), 0);
-      const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
       const CUtensorMap* tm_b = rank == 0 ? &tmK : &tmU;  // this CTA's half of [K; U]
       uint32_t gc = 0;  // chunks loaded so far (all units)
       int lu = 0;       // units so far
@@ -198,6 +215,21 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           if (rank == 0) mbar_arrive_expect_tx(&ku_full[s], 2 * kMhKuBytes);
           tma_load_2d_pair(ku, tm_b, 0, row, ku_full_lead + s * 8);
           tma_load_2d_pair(ku + kMhBox, tm_b, 64, row, ku_full_lead + s * 8);
+        }
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V producer (both CTAs)
+    // A ring of its own: V chunks wait only for the PV products, K|U chunks only for the S
+    // products, so neither ring holds the other back.
+    if (lane == 0) {
+      const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
+      uint32_t gc = 0;
+      bool ok = true;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl) {
+        const int h = unit / args.n_pt;
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const int row = h * rows_per_head + c * kMhChunk;
           const int sv = gc % kMhVStages;
           if (!mbar_wait(&v_empty[sv], ((gc / kMhVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
           if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kMhVBytes);
@@ -207,45 +239,23 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer (even CTA)
+    // ------------------------------------------------------------ S issuer (even CTA)
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(2 * kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
-      constexpr uint32_t kIdescPV = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
       // descriptors of the first stage of each operand; every MMA moves them by a constant
       const uint64_t q_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
-      const uint64_t p_desc = smem_desc_sw128(smem_u32(smem + kMhPOff), 16, 1024);
       const uint64_t ku_desc = smem_desc_sw128(smem_u32(smem + kMhKuOff), 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kMhVOff), kMhBox, 1024);
       uint32_t gc = 0;
       int lu = 0;
       bool ok = true, issued = false;
-      // O += P_g V_g for global chunk g (first: the unit's first chunk, which starts O afresh)
-      auto pv = [&](uint32_t g, bool first, int unit_local) -> bool {
-        const uint32_t pb = g & 1u;
-        if (!mbar_wait(&p_full[pb], (g >> 1) & 1u, ctl)) return false;
-        if (first && !mbar_wait(o_empty, (unit_local & 1) ^ 1u, ctl)) return false;
-        const uint32_t sv = g % kMhVStages;
-        if (!mbar_wait(&v_full[sv], (g / kMhVStages) & 1u, ctl)) return false;
-        tc_fence_after();
-        const uint64_t pd = desc_add(p_desc, pb * kMhPBytes);
-        const uint64_t vd = desc_add(v_desc, sv * kMhVBytes);
-#pragma unroll
-        for (int k = 0; k < kMhChunk / 16; ++k)
-          umma_bf16_pair(tmem_base, desc_add(pd, k * 32), desc_add(vd, k * 2048), kIdescPV,
-                         (!first || k != 0) ? 1u : 0u);
-        umma_commit_pair(&p_empty[pb], 3);
-        umma_commit_pair(&v_empty[sv], 3);
-        return true;
-      };
       for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
         if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t gcb = gc;
         for (int c = 0; c < args.nch; ++c, ++gc) {
           const uint32_t s = gc % kMhKuStages;
           if (!mbar_wait(&ku_full[s], (gc / kMhKuStages) & 1u, ctl)) { ok = false; break; }
-          const uint32_t sb = gc & 1u;
-          if (!mbar_wait(&s_empty[sb], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          const uint32_t sb = gc % kMhSBufs;
+          if (!mbar_wait(&s_empty[sb], ((gc / kMhSBufs) & 1u) ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
           const uint64_t kd = desc_add(ku_desc, s * kMhKuBytes);
           const uint32_t d_s = tmem_base + 128 + sb * 128;
@@ -260,29 +270,51 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           umma_commit_pair(&ku_empty[s], 3);
           if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // Q no longer read in this unit
           issued = true;
-          if (c >= 2 && !pv(gc - 2, c == 2, lu)) { ok = false; break; }
         }
-        if (!ok) break;
-        for (int c = args.nch >= 2 ? args.nch - 2 : 0; c < args.nch; ++c)
-          if (!pv(gcb + c, c == 0, lu)) { ok = false; break; }
+      }
+      if (!ok && issued) drain_mma(&drain[0], abort_flag, args.status);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer (even CTA)
+    // Issues O += P_c V_c as soon as the epilogue has written P_c; its products write only O and
+    // read only P and V, so the two issuing threads share no state.
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdescPV = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
+      const uint64_t p_desc = smem_desc_sw128(smem_u32(smem + kMhPOff), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kMhVOff), kMhBox, 1024);
+      uint32_t gc = 0;
+      int lu = 0;
+      bool ok = true, issued = false;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const uint32_t pb = gc % kMhPBufs;
+          if (!mbar_wait(&p_full[pb], (gc / kMhPBufs) & 1u, ctl)) { ok = false; break; }
+          if (c == 0 && !mbar_wait(o_empty, (lu & 1) ^ 1u, ctl)) { ok = false; break; }
+          const uint32_t sv = gc % kMhVStages;
+          if (!mbar_wait(&v_full[sv], (gc / kMhVStages) & 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t pd = desc_add(p_desc, pb * kMhPBytes);
+          const uint64_t vd = desc_add(v_desc, sv * kMhVBytes);
+#pragma unroll
+          for (int k = 0; k < kMhChunk / 16; ++k)
+            umma_bf16_pair(tmem_base, desc_add(pd, k * 32), desc_add(vd, k * 2048), kIdescPV,
+                           (c != 0 || k != 0) ? 1u : 0u);
+          umma_commit_pair(&p_empty[pb], 3);
+          umma_commit_pair(&v_empty[sv], 3);
+          issued = true;
+        }
         if (!ok) break;
         umma_commit_pair(o_full, 3);
       }
-      if (!ok && issued) {
-        umma_commit_pair(drain, 1);
-        WaitCtl quick{abort_flag, args.status, 100000000ull};
-        volatile int no_abort = 0;
-        quick.abort = &no_abort;
-        mbar_wait(drain, 0, quick);
-      }
+      if (!ok && issued) drain_mma(&drain[1], abort_flag, args.status);
     }
   } else {
-    // ------------------------------------------------------------ epilogue warps 2..9
+    // ------------------------------------------------------------ epilogue warps 4..11
     const int q = warp & 3;            // TMEM lane quadrant this warp may access
-    const int set = (warp - 2) >> 2;   // chunks with (global chunk index & 1) == set; O columns
+    const int set = (warp - 4) >> 2;   // chunks with (global chunk index & 1) == set; O columns
     const int row = q * 32 + lane;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t pbuf = smem_u32(smem + kMhPOff) + set * kMhPBytes;
+    const uint32_t p_base = smem_u32(smem + kMhPOff);
     const int64_t o_ld = (int64_t)args.H * kMhDh;
     uint32_t gc = 0;
     int lu = 0;
@@ -294,38 +326,41 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       const float* rrow = args.r + ((int64_t)(tok_ok ? token : 0) * args.H + h) * args.E;
       for (int c = 0; c < args.nch; ++c, ++gc) {
         if ((int)(gc & 1u) != set) continue;
-        const uint32_t use = gc >> 1;
-        const bool ready = mbar_wait(&s_full[set], use & 1u, ctl);
+        const uint32_t pb = gc % kMhPBufs;  // the set's two buffers in turn
+        const uint32_t sb = gc % kMhSBufs;
+        const bool ready = mbar_wait(&s_full[sb], (gc / kMhSBufs) & 1u, ctl);
         __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
         if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ts = t_lane + 128 + set * 128;
+        const uint32_t ts = t_lane + 128 + sb * 128;
         const float rv = tok_ok ? rrow[c / args.ch_per_sub] : 0.f;
         uint32_t w[32];  // this row's 64 P values as bf16 pairs
-        float g[32], u[32];
+        float g0[32], u0[32], g1[32], u1[32];
+        tmem_ld32(ts, g0);
+        tmem_ld32(ts + kMhChunk, u0);
+        tmem_ld32(ts + 32, g1);
+        tmem_ld32(ts + kMhChunk + 32, u1);
+        tmem_ld_wait_regs(g0);
+        pin_regs(u0);
+        pin_regs(g1);
+        pin_regs(u1);
+        tc_fence_before();
+        warp_arrive_lead(&s_empty[sb], rank, lane);  // the S buffer is in registers
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(ts + hh * 32, g);
-          tmem_ld32(ts + kMhChunk + hh * 32, u);
-          tmem_ld_wait_regs(g);
-          pin_regs(u);
-          if (hh == 1) {
-            tc_fence_before();
-            warp_arrive_lead(&s_empty[set], rank, lane);  // the S buffer is in registers or P
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            w[hh * 16 + j] = pack_bf16x2(silu_tanh(g[2 * j]) * u[2 * j] * rv,
-                                         silu_tanh(g[2 * j + 1]) * u[2 * j + 1] * rv);
+        for (int j = 0; j < 16; ++j) {
+          w[j] = pack_bf16x2(silu_tanh(g0[2 * j]) * u0[2 * j] * rv,
+                             silu_tanh(g0[2 * j + 1]) * u0[2 * j + 1] * rv);
+          w[16 + j] = pack_bf16x2(silu_tanh(g1[2 * j]) * u1[2 * j] * rv,
+                                  silu_tanh(g1[2 * j + 1]) * u1[2 * j + 1] * rv);
         }
-        const bool p_free = mbar_wait(&p_empty[set], (use & 1u) ^ 1u, ctl);
+        const bool p_free = mbar_wait(&p_empty[pb], ((gc / kMhPBufs) & 1u) ^ 1u, ctl);
         if (!__all_sync(0xffffffffu, p_free)) { ok = false; break; }  // warp-uniform exit
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16)
-          st_shared_v4(pbuf + p_offset(row, c16), w[4 * c16], w[4 * c16 + 1], w[4 * c16 + 2],
+          st_shared_v4(p_base + pb * kMhPBytes + p_offset(row, c16), w[4 * c16], w[4 * c16 + 1], w[4 * c16 + 2],
                        w[4 * c16 + 3]);
         fence_proxy_async_smem();  // make P visible to the tensor core's reads
-        warp_arrive_lead(&p_full[set], rank, lane);
+        warp_arrive_lead(&p_full[pb], rank, lane);
       }
       if (!ok) break;
       const bool ready = mbar_wait(o_full, lu & 1, ctl);

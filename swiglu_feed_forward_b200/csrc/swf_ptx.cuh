@@ -274,6 +274,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Consumer release to the even CTA of a pair: an arrive on its mbarrier (cluster address) with
+// the default semantics (release at CTA scope).  For signals whose guarded data stays on the
+// arriving CTA's own SM (its TMEM after tcgen05.wait::ld + tcgen05.fence::before_thread_sync, or
+// its shared memory after fence.proxy.async, read back by the pair MMA on this SM), as 2-SM
+// tensor-core pipelines do; a cluster-scope release cost about a microsecond per arrive here.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // TMA tile load into this CTA's shared memory whose completion is signalled on an mbarrier of
 // either CTA of the pair (`bar_cluster` is a cluster address).  No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, int32_t c0,

@@ -30,9 +30,11 @@ def reference(inp, tokens=None):
 @pytest.mark.parametrize("T,H,E,de", [
     (200, 2, 3, 64),     # ragged token tile, 3 sub-networks of one chunk
     (1, 1, 1, 64),       # one token, one chunk
-    (128, 1, 2, 128),    # exactly one tile, two chunks per sub-network
-    (300, 3, 2, 192),    # three heads, ragged
-    (700, 2, 5, 384),    # the 1.3B sub-network width, several tiles per head
+    (260, 2, 3, 192),    # odd chunk count per sub-network
+    (128, 1, 2, 256),    # exactly one tile (and an empty partner tile), two chunks per sub-network
+    (300, 3, 2, 256),    # three heads, ragged
+    (700, 2, 5, 384),    # the 1.3B sub-network width, several tile pairs per head
+    (520, 1, 7, 384),    # the 370M configuration's E, five tile pairs
 ])
 def test_small_and_ragged(T, H, E, de):
     inp = synth.mhffn_inputs(T, H, 128, E, de, seed=T + E, with_do=False)
