@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) break;
       tc_fence_before();
-      if (PAIR && rank != 0) mbar_arrive_cluster(tempty_lead + buf * 8);
+      if (PAIR && rank != 0) mbar_arrive_remote(tempty_lead + buf * 8);  // TMEM read: own SM
       else mbar_arrive(&tempty[buf]);
     }
     if (lane == 0) {
@@ -892,7 +892,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       tc_fence_before();
-      if (PAIR && rank != 0) mbar_arrive_cluster(tempty_lead + buf * 8);
+      if (PAIR && rank != 0) mbar_arrive_remote(tempty_lead + buf * 8);  // TMEM read: own SM
       else mbar_arrive(&tempty[buf]);
       if constexpr (EPI == kEpiEnergyTopK) {
         // this thread wrote its token's whole energy row (all N-blocks of the unit): select
