@@ -359,6 +359,27 @@ def secondary_mlp2(api, steps, warmup, world, peak):
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
+def secondary_mhffn(api, steps, warmup, world, peak):
+    """FlashFFN multi-head FFN forward (one fused kernel) at the 1.3B configuration."""
+    w = synth.WORKLOADS[6]
+    T, H, dh, E, de = (w[k] for k in ("T", "H", "d_h", "E", "d_e"))
+    dev = torch.device("cuda")
+    inp = synth.mhffn_inputs(T, H, dh, E, de, w["seed"], with_do=False)
+    t = {k: v.to(dev) for k, v in inp.items()}
+    o = torch.empty_like(t["q"])
+
+    def fn():
+        api.flash_mhffn_fwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], o)
+    for _ in range(warmup):
+        fn()
+    ms = timed(fn, steps, world)
+    flops = 6.0 * T * H * dh * E * de
+    tf = flops * steps / (ms / 1e3) / 1e12
+    return {"workload": w["name"], "tflops": round(tf * world, 1), "pct_of_peak": round(100 * tf / peak, 2),
+            "ms_per_step": round(ms / steps, 3), "steps": steps, "flops_per_step": flops,
+            "intermediate_bytes_not_written": 2 * T * H * E * de}
+
+
 def run_ours(args, world, rank, local):
     from swiglu_feed_forward_b200 import api
     w = synth.WORKLOADS[WORKLOAD]
@@ -454,6 +475,12 @@ def run_ours(args, world, rank, local):
             secondary["leaky_relu_sq_mlp_step"] = secondary_mlp2(api, max(3, args.steps // 2), 3, world, peak_sus)
         except Exception as exc:
             secondary["leaky_relu_sq_mlp_step"] = {"error": str(exc)[:200]}
+        torch.cuda.empty_cache()
+        try:
+            secondary["flashffn_multihead_forward"] = secondary_mhffn(api, max(3, args.steps // 2), 3, world,
+                                                                      peak_sus)
+        except Exception as exc:
+            secondary["flashffn_multihead_forward"] = {"error": str(exc)[:200]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
