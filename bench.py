@@ -375,9 +375,24 @@ def secondary_mhffn(api, steps, warmup, world, peak):
     ms = timed(fn, steps, world)
     flops = 6.0 * T * H * dh * E * de
     tf = flops * steps / (ms / 1e3) / 1e12
+    # the whole block from x: prologue (head-normalised projection, router) + fused core
+    d_model = H * dh
+    pro = {k: v.to(dev) for k, v in synth.mhffn_prologue_inputs(T, d_model, H, dh, E, w["seed"]).items()}
+    q, r = torch.empty_like(t["q"]), torch.empty_like(t["router"])
+
+    def block():
+        api.flash_mhffn_prologue(pro["x"], pro["w_q"], pro["w_r"], H, E, q_gain=pro["q_gain"], q=q, router=r)
+        api.flash_mhffn_fwd(q, t["w_k"], t["w_u"], t["w_v"], r, o)
+    for _ in range(warmup):
+        block()
+    ms_b = timed(block, steps, world)
+    flops_b = flops + 2.0 * T * d_model * (H * dh + H * E)
     return {"workload": w["name"], "tflops": round(tf * world, 1), "pct_of_peak": round(100 * tf / peak, 2),
             "ms_per_step": round(ms / steps, 3), "steps": steps, "flops_per_step": flops,
-            "intermediate_bytes_not_written": 2 * T * H * E * de}
+            "intermediate_bytes_not_written": 2 * T * H * E * de,
+            "block_from_x": {"ms_per_step": round(ms_b / steps, 3),
+                             "tflops": round(flops_b * steps / (ms_b / 1e3) / 1e12 * world, 1),
+                             "flops_per_step": flops_b, "d_model": d_model}}
 
 
 def run_ours(args, world, rank, local):

@@ -189,6 +189,22 @@ swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void* w_u, cons
                            int32_t head_dim, int32_t num_sub, int32_t sub_dim, swf_dtype dtype,
                            void* stream);
 
+/* The multi-head block's prologue (same page, "Overview": Q is the heads' RMS-normalised
+ * projection of the input, R the sigmoid-normalised router weights):
+ *   q[t, h*head_dim + i] = z[t,h,i] / sqrt(mean_i z[t,h,i]^2 + eps) * q_gain[i],  z = x w_q^T
+ *   router[t, h, e] = sigmoid(l[t,h,e]) / sum_e' sigmoid(l[t,h,e']),         l = x w_r^T
+ *   x [T, d_model]; w_q [num_heads * head_dim, d_model]; q_gain [head_dim] fp32 or NULL (no
+ *   gain); w_r [num_heads * num_sub, d_model]; q [T, num_heads * head_dim] (the input of
+ *   flash_mhffn_fwd); router [T, num_heads, num_sub] fp32.  Outputs are overwritten.
+ * Two tcgen05 GEMMs with the normalisations fused into their epilogues.  Device pointers,
+ * caller-owned, 16-byte aligned; asynchronous on `stream`; nothing allocates.  Supported:
+ * dtype SWF_BF16, head_dim 128, d_model a multiple of 16, num_heads * num_sub <= 256; else
+ * SWF_ERR_UNSUPPORTED.  eps < 0 or NaN: SWF_ERR_INVALID_ARG. */
+swf_status flash_mhffn_prologue(const void* x, const void* w_q, const float* q_gain,
+                                const void* w_r, void* q, float* router, int64_t T,
+                                int64_t d_model, int32_t num_heads, int32_t head_dim,
+                                int32_t num_sub, float eps, swf_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------------ group-sparse variant */
 
 /* Subsample index (eugen_sparse README, make_subsample_index; drawn once per layer).  HOST
@@ -327,7 +343,8 @@ typedef enum swf_kernel_kind {
   SWF_K_MLP2_DW_UP = 24,   /* LeakyReLU^2 MLP: dpre^T x */
   SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
   SWF_K_MHFFN_FWD = 26,    /* FlashFFN multi-head FFN forward (fused, one kernel) */
-  SWF_K_NUM_KINDS = 27
+  SWF_K_MHFFN_PROLOGUE = 27, /* FlashFFN prologue: head-normalised projection, router */
+  SWF_K_NUM_KINDS = 28
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

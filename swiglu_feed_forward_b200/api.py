@@ -149,6 +149,20 @@ def flash_mhffn_fwd(q, w_k, w_u, w_v, router, o=None, stream=None):
     return o
 
 
+def flash_mhffn_prologue(x, w_q, w_r, num_heads, num_sub, q_gain=None, eps=1e-6, q=None, router=None,
+                         stream=None):
+    """x [T, d_model]; w_q [H * 128, d_model]; w_r [H * E, d_model]; q_gain [128] fp32 or None.
+    Returns (q [T, H, 128], router [T, H, E] fp32): the inputs of flash_mhffn_fwd."""
+    T, d = x.shape
+    dh = w_q.shape[0] // num_heads
+    q = _empty((T, num_heads, dh), x) if q is None else q
+    router = _empty((T, num_heads, num_sub), x, torch.float32) if router is None else router
+    _check("flash_mhffn_prologue", _lib.lib().flash_mhffn_prologue(
+        _p(x), _p(w_q), _p(q_gain), _p(w_r), _p(q), _p(router), T, d, num_heads, dh, num_sub,
+        float(eps), _dt(x), _stream(stream)))
+    return q, router
+
+
 # ------------------------------------------------------------------ group-sparse
 def make_subsample_index(d_ff, group_size, samples_per_group, seed):
     """Host call: returns (int32 CPU tensor [d_ff // group_size, spg], spg)."""

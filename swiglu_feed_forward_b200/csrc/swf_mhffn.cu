@@ -30,6 +30,7 @@
 #include <initializer_list>
 
 #include "swf_internal.h"
+#include "swf_launch.cuh"
 #include "swf_ptx.cuh"
 
 namespace swf {
@@ -461,4 +462,43 @@ extern "C" swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void
   if (cudaLaunchKernelEx(&cfg, mhffn_fwd_kernel, tq, tk, tu, tv, a) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
+// The block's prologue ("Overview": Q is the per-head RMS-normalised projection of the input, R
+// the sigmoid-normalised router weights), as two tcgen05 GEMMs with fused epilogues:
+//   q[t, h*128 + i] = z_h[i] / sqrt(mean_i z_h[i]^2 + eps) * q_gain[i],  z = x w_q^T
+//   router[t, h, e] = sigmoid(l[h*E + e]) / sum_e' sigmoid(l[h*E + e']),  l = x w_r^T
+extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const float* q_gain,
+                                           const void* w_r, void* q, float* router, int64_t T,
+                                           int64_t d_model, int32_t num_heads, int32_t head_dim,
+                                           int32_t num_sub, float eps, swf_dtype dtype,
+                                           void* stream) {
+  if (!x || !w_q || !w_r || !q || !router) return SWF_ERR_INVALID_ARG;
+  if (T <= 0 || d_model <= 0 || num_heads <= 0 || head_dim <= 0 || num_sub <= 0 || !(eps >= 0.f))
+    return SWF_ERR_INVALID_ARG;
+  if (dtype != SWF_BF16 && dtype != SWF_F32) return SWF_ERR_INVALID_ARG;
+  if (dtype != SWF_BF16 || head_dim != kMhDh || d_model % 16 != 0 || num_heads * num_sub > 256 ||
+      T > INT32_MAX / 2 || d_model > (1 << 20) || (int64_t)num_heads * kMhDh > (1 << 20))
+    return SWF_ERR_UNSUPPORTED;
+  for (const void* p : std::initializer_list<const void*>{x, w_q, w_r, q, router, q_gain})
+    if (p && !aligned16(p)) return SWF_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t nq = (int64_t)num_heads * kMhDh, nr = (int64_t)num_heads * num_sub;
+  CUtensorMap tx, tq, tr;
+  if (!encode_tmap_bf16(&tx, x, d_model, T, d_model, 64, 128) ||
+      !encode_tmap_bf16(&tq, w_q, d_model, nq, d_model, 64, 128) ||
+      !encode_tmap_bf16(&tr, w_r, d_model, nr, d_model, 64, 256))
+    return SWF_ERR_LAUNCH;
+  TcGemmArgs a = base_args(T, nq, 128, d_model);
+  a.out0 = q;
+  a.ld_out = nq;
+  a.bias = q_gain;
+  a.eps = eps;
+  swf_status s = launch_tc<128, false, false, false, kEpiHeadNorm>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st);
+  if (s != SWF_OK) return s;
+  TcGemmArgs b = base_args(T, nr, 256, d_model);
+  b.out0 = router;
+  b.ld_out = nr;
+  b.group_size = num_sub;
+  return launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, b, st);
 }

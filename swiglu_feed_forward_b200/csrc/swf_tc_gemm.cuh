@@ -34,6 +34,10 @@
 //   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
 //   kEpiPartialF32 fp32 C of K-split ks -> part[ks][m][n] (split-K weight gradients; a separate
 //                  kernel sums the splits in a fixed order)
+//   kEpiHeadNorm   BN = 128 = one head's columns: C / sqrt(mean(C^2) + eps) * gain (bias, nullable)
+//                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
+//   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
+//                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
 //   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
 //                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
 //                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
@@ -60,7 +64,9 @@ enum : int {
   kEpiLeakySq = 7,
   kEpiScale = 8,
   kEpiPartialF32 = 9,
-  kEpiEnergyTopK = 10
+  kEpiEnergyTopK = 10,
+  kEpiHeadNorm = 11,
+  kEpiRouter = 12
 };
 constexpr int kTopKMaxGroups = 64;  // kEpiEnergyTopK: groups held in registers per token
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
@@ -99,6 +105,7 @@ struct TcGemmArgs {
   int n_groups;           // kEpiEnergy: groups (columns of out0)
   int64_t ld_grp;         // kEpiEnergy*: stride of out0 between groups (0: 1); ld_out is the
                           //   stride between tokens (1 with ld_grp = M: group-major energies)
+  float eps;              // kEpiHeadNorm
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
   int sel_k;
   int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
@@ -733,6 +740,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
               }
             }
+          }
+        }
+      } else if constexpr (EPI == kEpiHeadNorm) {
+        static_assert(BN == 128, "one head per tile");
+        float v[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_acc + c * 32, v[c]);
+        tmem_ld_wait_regs(v[0]);
+        pin_regs(v[1]);
+        pin_regs(v[2]);
+        pin_regs(v[3]);
+        if (row_ok) {
+          float ss = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(v[c][j], v[c][j], ss);
+          const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
+          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + t.nb * BN;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = v[c][j] * inv * (args.bias ? args.bias[c * 32 + j] : 1.f);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
+          }
+        }
+      } else if constexpr (EPI == kEpiRouter) {
+        // pass 1: sigmoid of each logit into this token's output row; pass 2: per-head sums
+        float* rp = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float z[32];
+          tmem_ld32(t_acc + c, z);
+          tmem_ld_wait_regs(z);
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st_if(rp + c + j, sigmoidf_(z[j]), c + j < args.N);
+          }
+        }
+        if (row_ok) {
+          const int E = args.group_size;
+#pragma unroll 1
+          for (int h0 = 0; h0 < args.N; h0 += E) {
+            float sum = 0.f;
+#pragma unroll 1
+            for (int e = 0; e < E; ++e) sum += rp[h0 + e];
+            const float inv = 1.0f / sum;
+#pragma unroll 1
+            for (int e = 0; e < E; ++e) rp[h0 + e] *= inv;
           }
         }
       } else if constexpr (EPI == kEpiEnergy || EPI == kEpiEnergyTopK) {

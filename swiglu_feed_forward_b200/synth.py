@@ -38,7 +38,8 @@ WORKLOADS = {
 }
 
 _TENSOR_IDS = {"x": 1, "w_gate": 2, "w_up": 3, "w_down": 4, "dy": 5, "bias": 6,
-               "q": 7, "w_k": 8, "w_u": 9, "w_v": 10, "router": 11, "do": 12}
+               "q": 7, "w_k": 8, "w_u": 9, "w_v": 10, "router": 11, "do": 12,
+               "w_q": 13, "w_r": 14, "q_gain": 15}
 
 DY_STD = 0.1  # N(0, 1e-2) as a variance
 
@@ -97,6 +98,17 @@ def mhffn_inputs(T, H, d_h, E, d_e, seed, dtype=torch.bfloat16, with_do=True):
     if with_do:
         out["do"] = normal((T, H, d_h), DY_STD, seed, "do", dtype)
     return out
+
+
+def mhffn_prologue_inputs(T, d_model, H, d_h, E, seed, dtype=torch.bfloat16):
+    """Inputs of the multi-head block's prologue: x [T, d_model] ~ N(0, 1); w_q [H*d_h, d_model]
+    and w_r [H*E, d_model] ~ N(0, 1/d_model); q_gain [d_h] fp32 ~ U(0.5, 1.5).  CPU tensors."""
+    return {
+        "x": normal((T, d_model), 1.0, seed, "x", dtype),
+        "w_q": normal((H * d_h, d_model), d_model ** -0.5, seed, "w_q", dtype),
+        "w_r": normal((H * E, d_model), d_model ** -0.5, seed, "w_r", dtype),
+        "q_gain": torch.rand(d_h, generator=_gen(seed, "q_gain"), dtype=torch.float32) + 0.5,
+    }
 
 
 def skewed_balance_bias(num_groups, seed):

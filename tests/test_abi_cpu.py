@@ -105,6 +105,13 @@ def test_mhffn_argument_errors(lib):
     assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, F32, None) == 2     # fp32
     assert f(p, p, p, p, q, p, 256, 16, 128, 15, 384, BF, None) == 3      # unaligned router
     assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, 9, None) == 1       # bad dtype
+    g = lib.flash_mhffn_prologue
+    assert g(None, p, None, p, p, p, 256, 2048, 16, 128, 15, 1e-6, BF, None) == 1  # null x
+    assert g(p, p, None, p, p, p, 256, 2048, 16, 128, 15, -1.0, BF, None) == 1     # eps < 0
+    assert g(p, p, None, p, p, p, 256, 2048, 16, 64, 15, 1e-6, BF, None) == 2      # d_h 64
+    assert g(p, p, None, p, p, p, 256, 2040, 16, 128, 15, 1e-6, BF, None) == 2     # d_model % 16
+    assert g(p, p, None, p, p, p, 256, 2048, 16, 128, 17, 1e-6, BF, None) == 2     # 272 router columns
+    assert g(p, p, q, p, p, p, 256, 2048, 16, 128, 15, 1e-6, BF, None) == 3        # unaligned gain
 
 
 @pytest.mark.parametrize("d_ff,G,spg,seed", [(4096, 64, 8, 3), (512, 32, 8, 0), (256, 16, 16, 7),

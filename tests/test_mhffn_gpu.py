@@ -71,3 +71,46 @@ def test_full_size_sampled_tokens():
     rng = np.random.default_rng(0)
     tokens = np.sort(np.concatenate([rng.choice(w["T"] - 128, 24, replace=False), [w["T"] - 1]]))
     assert_close("o[tokens]", f64(o)[tokens], reference(inp, tokens), torch.bfloat16)
+
+
+def check_prologue(inp, H, E, use_gain, tokens=None):
+    x, wq, wr = (inp[k].cuda() for k in ("x", "w_q", "w_r"))
+    gain = inp["q_gain"].cuda() if use_gain else None
+    q, r = api.flash_mhffn_prologue(x, wq, wr, H, E, q_gain=gain, eps=1e-6)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    xs = f64(inp["x"]) if tokens is None else f64(inp["x"])[tokens]
+    q_ref = O.head_rmsnorm(xs @ f64(inp["w_q"]).T, H, eps=1e-6,
+                           weight=f64(inp["q_gain"]) if use_gain else None)
+    r_ref = O.router_weights((xs @ f64(inp["w_r"]).T).reshape(len(xs), H, E))
+    qg, rg = f64(q), f64(r)
+    if tokens is not None:
+        qg, rg = qg[tokens], rg[tokens]
+    assert_close("q", qg, q_ref, torch.bfloat16)
+    assert_close("router", rg, r_ref, torch.float32)
+    return q, r
+
+
+@pytest.mark.parametrize("T,d_model,H,E,use_gain", [
+    (300, 256, 3, 5, True),     # ragged tokens, E not a power of two
+    (1, 64, 1, 1, False),       # one token, one head, one sub-network (router weight 1)
+    (513, 768, 6, 8, True),     # the 128M configuration's heads and E
+    (256, 2048, 16, 15, False), # the 1.3B configuration: 240 router columns
+])
+def test_prologue(T, d_model, H, E, use_gain):
+    check_prologue(synth.mhffn_prologue_inputs(T, d_model, H, 128, E, seed=T + H), H, E, use_gain)
+
+
+def test_block_prologue_then_fused_forward():
+    """x -> (Q, R) -> O through both entry points against the oracle's whole block."""
+    T, d_model, H, E, de = 700, 512, 4, 3, 128
+    pro = synth.mhffn_prologue_inputs(T, d_model, H, 128, E, seed=21)
+    wts = synth.mhffn_inputs(1, H, 128, E, de, seed=21, with_do=False)
+    q, r = check_prologue(pro, H, E, True)
+    o = api.flash_mhffn_fwd(q, wts["w_k"].cuda(), wts["w_u"].cuda(), wts["w_v"].cuda(), r)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    qr = O.head_rmsnorm(f64(pro["x"]) @ f64(pro["w_q"]).T, H, eps=1e-6, weight=f64(pro["q_gain"]))
+    rr = O.router_weights((f64(pro["x"]) @ f64(pro["w_r"]).T).reshape(T, H, E))
+    ref = O.mhffn_forward(qr, f64(wts["w_k"]), f64(wts["w_u"]), f64(wts["w_v"]), rr)["o"]
+    assert_close("o", f64(o), ref, torch.bfloat16)
