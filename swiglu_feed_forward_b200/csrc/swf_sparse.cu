@@ -61,6 +61,7 @@ struct Carver {
 struct SavedView {
   int32_t *offs, *tokens, *seg_start, *seg_rows, *tile_group, *row_token, *pair_row;
   __nv_bfloat16 *h, *a, *b;
+  __nv_bfloat16* xc;  // the gathered x rows (group-major), reused by the backward
 };
 
 SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
@@ -76,33 +77,31 @@ SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
   v.h = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.a = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.b = c.take<__nv_bfloat16>(s.rmax * s.G);
+  v.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
   return v;
 }
 
 struct FwdWs {
   int32_t* counts;
-  __nv_bfloat16* xc;
   __nv_bfloat16* yc;  // per-pair contributions to y, group-major rows
 };
 FwdWs fwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   Carver c{static_cast<char*>(base)};
   FwdWs w;
   w.counts = c.take<int32_t>((size_t)s.nblk * s.ng);
-  w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.yc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
   return w;
 }
 
 struct BwdWs {
-  __nv_bfloat16 *xc, *dyc, *dgu;
+  __nv_bfloat16 *dyc, *dgu;
   __nv_bfloat16* dxc;  // per-pair contributions to dx, group-major rows
 };
 BwdWs bwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   Carver c{static_cast<char*>(base)};
   BwdWs w;
-  w.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.dyc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.dgu = c.take<__nv_bfloat16>(s.rmax * 128);
   w.dxc = c.take<__nv_bfloat16>(s.rmax * s.d);
@@ -781,11 +780,11 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
   if ((s = run_buckets(group_idx, sd, w.counts, v.offs, v.tokens, v.seg_start, v.seg_rows,
                        v.tile_group, v.row_token, v.pair_row, st)) != SWF_OK)
     return s;
-  if ((s = run_gather(x, v, sd, w.xc, st)) != SWF_OK) return s;
+  if ((s = run_gather(x, v, sd, v.xc, st)) != SWF_OK) return s;
 
   {  // gate|up per group: [h|a|b] rows = SiLU/gating of Xc [W_g[g] | W_u[g]]^T
     CUtensorMap txc, twg, twu;
-    if (!encode_tmap_bf16(&txc, w.xc, d, sd.rmax, d, 64, 128) ||
+    if (!encode_tmap_bf16(&txc, v.xc, d, sd.rmax, d, 64, 128) ||
         !encode_tmap_bf16(&twg, w_gate, d, f, d, 64, G) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, G))
       return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, G, 2 * G, d);
@@ -838,7 +837,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
   if (saved_bytes < need_saved || ws_bytes < need_ws) return SWF_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  if ((s = run_gather(x, v, sd, w.xc, st)) != SWF_OK) return s;
+  // the forward's gathered x rows are in `saved`; only dY is gathered here
   if ((s = run_gather(dy, v, sd, w.dyc, st)) != SWF_OK) return s;
   {  // dH = dYc W_d[:, g]; dG = dH * a, dU = dH * b -> dgu [R, 128] (halves padded to 64)
     CUtensorMap tdyc, twd;
@@ -878,7 +877,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
   {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ Xc_seg
     CUtensorMap tdgu, txc;
     if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64) ||
-        !encode_tmap_bf16(&txc, w.xc, d, sd.rmax, d, 64, 64))
+        !encode_tmap_bf16(&txc, v.xc, d, sd.rmax, d, 64, 64))
       return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(128, d, 256, 0);
     a.n_groups = sd.ng;
