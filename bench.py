@@ -276,6 +276,20 @@ def timed(fn, steps, world):
     return max_over_ranks(e0.elapsed_time(e1), world)
 
 
+def graph_of(fn):
+    """fn captured once into a CUDA graph (warmed on a side stream first); returns the replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def secondary_infer(api, steps, warmup, world):
     w = synth.WORKLOADS[4]
     M, d, f = w["M"], w["d_model"], w["d_ff"]
@@ -325,6 +339,11 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     for _ in range(warmup):
         fn()
     ms = timed(fn, steps, world)
+    # the same step as one CUDA graph: about 20 short launches, so launch gaps show
+    g = graph_of(fn)
+    for _ in range(warmup):
+        g.replay()
+    ms_graph = timed(g.replay, steps, world)
     useful = 2.0 * M * d * ng * spg + 18.0 * M * d * K * G
     tf = useful * steps / (ms / 1e3) / 1e12
     per_group = torch.bincount(idx.flatten().long(), minlength=ng)
@@ -332,6 +351,8 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
             "useful_tflops": round(tf * world, 3),
             "pct_of_peak": round(100 * tf / peak, 2), "ms_per_step": round(ms / steps, 3),
             "steps": steps, "useful_flops_per_step": useful,
+            "cuda_graph": {"ms_per_step": round(ms_graph / steps, 3),
+                           "useful_tflops": round(useful * steps / (ms_graph / 1e3) / 1e12 * world, 3)},
             "tokens_per_group": {"max": int(per_group.max()), "mean": round(M * K / ng, 1),
                                  "min": int(per_group.min())}}
 

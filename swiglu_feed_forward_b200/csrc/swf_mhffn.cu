@@ -486,15 +486,21 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
   const int64_t nq = (int64_t)num_heads * kMhDh, nr = (int64_t)num_heads * num_sub;
   CUtensorMap tx, tq, tr;
   if (!encode_tmap_bf16(&tx, x, d_model, T, d_model, 64, 128) ||
-      !encode_tmap_bf16(&tq, w_q, d_model, nq, d_model, 64, 128) ||
+      !encode_tmap_bf16(&tq, w_q, d_model, nq, d_model, 64, 128) ||  // 128 rows: a CTA's half
       !encode_tmap_bf16(&tr, w_r, d_model, nr, d_model, 64, 256))
     return SWF_ERR_LAUNCH;
-  TcGemmArgs a = base_args(T, nq, 128, d_model);
+  // projection: with an even head count, pair (cta_group::2) tiles of 256 tokens x 256 columns
+  // (two heads per epilogue row); otherwise one-CTA tiles of one head
+  const bool pair = nq % 256 == 0;
+  TcGemmArgs a = pair ? base_args(T, nq, 256, d_model, 2 * kTileM) : base_args(T, nq, 128, d_model);
   a.out0 = q;
   a.ld_out = nq;
   a.bias = q_gain;
   a.eps = eps;
-  swf_status s = launch_tc<128, false, false, false, kEpiHeadNorm>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st);
+  swf_status s =
+      pair ? launch_tc_pair<256, false, false, false, kEpiHeadNorm>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq,
+                                                                    EpiMaps{}, a, st)
+           : launch_tc<128, false, false, false, kEpiHeadNorm>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st);
   if (s != SWF_OK) return s;
   TcGemmArgs b = base_args(T, nr, 256, d_model);
   b.out0 = router;

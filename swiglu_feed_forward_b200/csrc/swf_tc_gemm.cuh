@@ -34,7 +34,7 @@
 //   kEpiScale      C * aux -> out0 (the stored activation gradient applied to dpost)
 //   kEpiPartialF32 fp32 C of K-split ks -> part[ks][m][n] (split-K weight gradients; a separate
 //                  kernel sums the splits in a fixed order)
-//   kEpiHeadNorm   BN = 128 = one head's columns: C / sqrt(mean(C^2) + eps) * gain (bias, nullable)
+//   kEpiHeadNorm   BN a multiple of 128, heads of 128 columns: C / sqrt(mean(C^2) + eps) * gain
 //                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
 //   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
 //                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
@@ -743,29 +743,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else if constexpr (EPI == kEpiHeadNorm) {
-        static_assert(BN == 128, "one head per tile");
-        float v[4][32];
+        static_assert(BN % 128 == 0, "whole heads per tile");
+#pragma unroll 1
+        for (int hd = 0; hd < BN / 128; ++hd) {  // each head: 128 columns of this row
+          float v[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_acc + c * 32, v[c]);
-        tmem_ld_wait_regs(v[0]);
-        pin_regs(v[1]);
-        pin_regs(v[2]);
-        pin_regs(v[3]);
-        if (row_ok) {
-          float ss = 0.f;
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_acc + hd * 128 + c * 32, v[c]);
+          tmem_ld_wait_regs(v[0]);
+          pin_regs(v[1]);
+          pin_regs(v[2]);
+          pin_regs(v[3]);
+          const int n0 = t.nb * BN + hd * 128;
+          if (row_ok && n0 < args.N) {
+            float ss = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(v[c][j], v[c][j], ss);
-          const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
-          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + t.nb * BN;
+              for (int j = 0; j < 32; ++j) ss = fmaf(v[c][j], v[c][j], ss);
+            const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
+            __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
+            for (int c = 0; c < 4; ++c) {
+              float o[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = v[c][j] * inv * (args.bias ? args.bias[c * 32 + j] : 1.f);
+              for (int j = 0; j < 32; ++j) o[j] = v[c][j] * inv * (args.bias ? args.bias[c * 32 + j] : 1.f);
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
+              for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
+            }
           }
         }
       } else if constexpr (EPI == kEpiRouter) {
