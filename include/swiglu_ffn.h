@@ -189,6 +189,26 @@ swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void* w_u, cons
                            int32_t head_dim, int32_t num_sub, int32_t sub_dim, swf_dtype dtype,
                            void* stream);
 
+/* Backward of flash_mhffn_fwd: gradients of L = sum(d_o * o) with respect to q, w_k, w_u, w_v
+ * and router (same shapes as those inputs; all overwritten, drouter fp32).  Runs per head as
+ * tcgen05 GEMMs over per-head buffers in `workspace` (flash_mhffn_bwd_workspace_bytes bytes):
+ *   dP = dO_h V_h^T;  [g | u] = Q_h [K_h ; U_h]^T with dS_g = dP r u SiLU'(g),
+ *   dS_u = dP r SiLU(g), P = SiLU(g) u r and the router partials sum dP SiLU(g) u fused into its
+ *   epilogue;  dQ_h = dS_g K_h + dS_u U_h;  [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h;  dV_h = P^T dO_h.
+ * Unlike the forward it writes the head's [T, E * sub_dim] activations (bf16) to the workspace.
+ * Device pointers, caller-owned, 16-byte aligned; asynchronous on `stream`; deterministic.
+ * Supported: dtype SWF_BF16, head_dim 128, sub_dim a multiple of 128; else SWF_ERR_UNSUPPORTED.
+ * Workspace missing or too small: SWF_ERR_WORKSPACE. */
+swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void* w_u, const void* w_v,
+                           const float* router, const void* d_o, void* dq, void* dw_k,
+                           void* dw_u, void* dw_v, float* drouter, void* workspace,
+                           size_t workspace_bytes, int64_t T, int32_t num_heads,
+                           int32_t head_dim, int32_t num_sub, int32_t sub_dim, swf_dtype dtype,
+                           void* stream);
+/* Bytes of flash_mhffn_bwd's workspace (0 for rejected arguments). */
+size_t flash_mhffn_bwd_workspace_bytes(int64_t T, int32_t num_heads, int32_t head_dim,
+                                       int32_t num_sub, int32_t sub_dim, swf_dtype dtype);
+
 /* The multi-head block's prologue (same page, "Overview": Q is the heads' RMS-normalised
  * projection of the input, R the sigmoid-normalised router weights):
  *   q[t, h*head_dim + i] = z[t,h,i] / sqrt(mean_i z[t,h,i]^2 + eps) * q_gain[i],  z = x w_q^T
@@ -345,7 +365,8 @@ typedef enum swf_kernel_kind {
   SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
   SWF_K_MHFFN_FWD = 26,    /* FlashFFN multi-head FFN forward (fused, one kernel) */
   SWF_K_MHFFN_PROLOGUE = 27, /* FlashFFN prologue: head-normalised projection, router */
-  SWF_K_NUM_KINDS = 28
+  SWF_K_MHFFN_BWD = 28,    /* FlashFFN multi-head FFN backward (per-head GEMMs) */
+  SWF_K_NUM_KINDS = 29
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

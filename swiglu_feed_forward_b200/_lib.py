@@ -39,6 +39,8 @@ SIGNATURES = {
     "leaky_relu_sq_mlp_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, SZ, I64, I64, I64, I32, P]),
     "flash_mhffn_fwd": (I32, [P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, P]),
     "flash_mhffn_prologue": (I32, [P, P, P, P, P, P, I64, I64, I32, I32, I32, C.c_float, I32, P]),
+    "flash_mhffn_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, SZ, I64, I32, I32, I32, I32, I32, P]),
+    "flash_mhffn_bwd_workspace_bytes": (SZ, [I64, I32, I32, I32, I32, I32]),
     "swf_make_subsample_index": (I32, [I64, I32, I32, U64, P]),
     "grouped_topk_select": (I32, [P, P, P, I32, P, I32, I32, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swf_group_buckets": (I32, [P, I64, I32, I32, P, P, P, SZ, P]),

@@ -149,6 +149,27 @@ def flash_mhffn_fwd(q, w_k, w_u, w_v, router, o=None, stream=None):
     return o
 
 
+def flash_mhffn_bwd(q, w_k, w_u, w_v, router, d_o, dq=None, dw_k=None, dw_u=None, dw_v=None,
+                    drouter=None, workspace=None, stream=None):
+    """Gradients of sum(d_o * flash_mhffn_fwd(q, w_k, w_u, w_v, router)).
+    Returns (dq, dw_k, dw_u, dw_v, drouter)."""
+    T, H, dh = q.shape
+    E, de = w_k.shape[1], w_k.shape[2]
+    dq = torch.empty_like(q) if dq is None else dq
+    dw_k = torch.empty_like(w_k) if dw_k is None else dw_k
+    dw_u = torch.empty_like(w_u) if dw_u is None else dw_u
+    dw_v = torch.empty_like(w_v) if dw_v is None else dw_v
+    drouter = torch.empty_like(router) if drouter is None else drouter
+    nb = _lib.lib().flash_mhffn_bwd_workspace_bytes(T, H, dh, E, de, _dt(q))
+    if workspace is None:
+        workspace = torch.empty(max(16, nb), device=q.device, dtype=torch.uint8)
+    _check("flash_mhffn_bwd", _lib.lib().flash_mhffn_bwd(
+        _p(q), _p(w_k), _p(w_u), _p(w_v), _p(router), _p(d_o), _p(dq), _p(dw_k), _p(dw_u), _p(dw_v),
+        _p(drouter), _p(workspace), workspace.numel() * workspace.element_size(), T, H, dh, E, de,
+        _dt(q), _stream(stream)))
+    return dq, dw_k, dw_u, dw_v, drouter
+
+
 def flash_mhffn_prologue(x, w_q, w_r, num_heads, num_sub, q_gain=None, eps=1e-6, q=None, router=None,
                          stream=None):
     """x [T, d_model]; w_q [H * 128, d_model]; w_r [H * E, d_model]; q_gain [128] fp32 or None.

@@ -53,6 +53,8 @@ int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
   return ks > 1 ? cdiv(kb, cdiv(kb, ks)) : 1;  // no empty trailing split
 }
 
+}  // namespace
+
 // Weight-gradient GEMM (both operands MN-major, K = tokens): split-K into fp32 partial planes
 // plus a fixed-order reduction when the planner finds too few output tiles, else direct stores.
 swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
@@ -87,7 +89,6 @@ int64_t part_elems(int64_t rows, int64_t cols, int64_t K) {
   const int ks = dw_ksplit(rows, cols, K);
   return ks > 1 ? ks * rows * cols : 0;
 }
-}  // namespace
 
 int64_t dense_bwd_part_elems(int64_t M, int64_t d, int64_t f) {
   return std::max(part_elems(2 * f, d, M), part_elems(d, f, M));

@@ -72,6 +72,14 @@ swf_status mlp2_bwd_f32(const float* dy, const float* x, const float* wu, const 
                         const float* post, const float* act_grad, float* dx, float* dwu,
                         float* dwd, float* dpre, int64_t M, int64_t d, int64_t f, cudaStream_t st);
 
+// Weight-gradient GEMM out = A^T B of rows x cols over K (tokens), both operands MN-major (maps
+// with 64 x 64 boxes), as pair tiles of 256 x 256; split-K into `part` (part_elems(...) fp32) and
+// a fixed-order reduction when the planner finds too few tiles.  Rows >= row_split go to out1.
+swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
+                     int64_t cols, int64_t K, void* out0, void* out1, int64_t row_split,
+                     float* part, cudaStream_t st);
+int64_t part_elems(int64_t rows, int64_t cols, int64_t K);
+
 // fp32 elements of the split-K partial planes the bf16 backward passes need (0: no split).
 int64_t dense_bwd_part_elems(int64_t M, int64_t d, int64_t f);
 int64_t mlp2_bwd_part_elems(int64_t M, int64_t d, int64_t f);

@@ -508,3 +508,173 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
   b.group_size = num_sub;
   return launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, b, st);
 }
+
+// ------------------------------------------------------------------ backward (per head, composed)
+// The fused forward keeps the activations on chip; a fused backward would need the dK, dU, dV
+// accumulators (384 TMEM columns for 128 sub-network rows) next to the recomputed S and dP, which
+// leaves room only for products too small to outrun the one-thread MMA issue rate.  So the
+// backward runs per head as tcgen05 GEMMs over per-head buffers:
+//   dP  = dO_h V_h^T                                   [T, F]      (F = E * d_e)
+//   S   = Q_h [K_h ; U_h]^T with the epilogue  dS_g = dP r u SiLU'(g), dS_u = dP r SiLU(g),
+//         P = SiLU(g) u r, and the router gradient's per-128-column partials sum dP SiLU(g) u
+//   dQ_h = dS_g K_h + dS_u U_h ;  [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h ;  dV_h = P^T dO_h
+// and one small kernel sums each sub-network's partials into dR.
+namespace swf {
+namespace {
+
+__global__ void mh_dr_reduce_kernel(const float* __restrict__ part, int64_t n, int per,
+                                    float* __restrict__ dr) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < per; ++k) s += part[i * per + k];  // fixed order
+    dr[i] = s;
+  }
+}
+
+struct MhBwdWs {
+  __nv_bfloat16 *dp, *dsgu, *p;
+  float *dr_part, *split;
+};
+
+MhBwdWs mh_bwd_ws(void* base, int64_t T, int64_t H, int64_t F, size_t* bytes) {
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    off = round_up(off, 256);
+    char* p = base ? static_cast<char*>(base) + off : nullptr;
+    off += n;
+    return p;
+  };
+  MhBwdWs w;
+  w.dp = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * F * 2));
+  w.dsgu = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * 2 * F * 2));
+  w.p = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * F * 2));
+  w.dr_part = reinterpret_cast<float*>(take((size_t)T * H * (F / 128) * 4));
+  const int64_t part = std::max(part_elems(2 * F, kMhDh, T), part_elems(F, kMhDh, T));
+  w.split = reinterpret_cast<float*>(take((size_t)std::max<int64_t>(part, 4) * 4));
+  if (bytes) *bytes = off;
+  return w;
+}
+
+swf_status check_mh_bwd(int64_t T, int32_t H, int32_t dh, int32_t E, int32_t de, swf_dtype dt) {
+  if (T <= 0 || H <= 0 || dh <= 0 || E <= 0 || de <= 0) return SWF_ERR_INVALID_ARG;
+  if (dt != SWF_BF16 && dt != SWF_F32) return SWF_ERR_INVALID_ARG;
+  if (dt != SWF_BF16 || dh != kMhDh || de % 128 != 0) return SWF_ERR_UNSUPPORTED;
+  if (T > INT32_MAX / 4 || (int64_t)E * de > (1 << 20) || (int64_t)H * E * de > INT32_MAX / 4 ||
+      (int64_t)H * kMhDh > (1 << 20))
+    return SWF_ERR_UNSUPPORTED;
+  return SWF_OK;
+}
+
+}  // namespace
+}  // namespace swf
+
+extern "C" size_t flash_mhffn_bwd_workspace_bytes(int64_t T, int32_t num_heads, int32_t head_dim,
+                                                  int32_t num_sub, int32_t sub_dim, swf_dtype dtype) {
+  if (check_mh_bwd(T, num_heads, head_dim, num_sub, sub_dim, dtype) != SWF_OK) return 0;
+  size_t need = 0;
+  mh_bwd_ws(nullptr, T, num_heads, (int64_t)num_sub * sub_dim, &need);
+  return need;
+}
+
+extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void* w_u,
+                                      const void* w_v, const float* router, const void* d_o,
+                                      void* dq, void* dw_k, void* dw_u, void* dw_v,
+                                      float* drouter, void* workspace, size_t workspace_bytes,
+                                      int64_t T, int32_t num_heads, int32_t head_dim,
+                                      int32_t num_sub, int32_t sub_dim, swf_dtype dtype,
+                                      void* stream) {
+  for (const void* p : std::initializer_list<const void*>{q, w_k, w_u, w_v, router, d_o, dq, dw_k,
+                                                          dw_u, dw_v, drouter})
+    if (!p) return SWF_ERR_INVALID_ARG;
+  swf_status s = check_mh_bwd(T, num_heads, head_dim, num_sub, sub_dim, dtype);
+  if (s != SWF_OK) return s;
+  for (const void* p : std::initializer_list<const void*>{q, w_k, w_u, w_v, router, d_o, dq, dw_k,
+                                                          dw_u, dw_v, drouter, workspace})
+    if (p && !aligned16(p)) return SWF_ERR_ALIGNMENT;
+  const int64_t H = num_heads, E = num_sub, de = sub_dim, F = E * de, ld = H * kMhDh;
+  size_t need = 0;
+  const MhBwdWs w = mh_bwd_ws(workspace, T, H, F, &need);
+  if (!workspace || workspace_bytes < need) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  using bf = __nv_bfloat16;
+  for (int64_t h = 0; h < H; ++h) {
+    const bf* qh = static_cast<const bf*>(q) + h * kMhDh;
+    const bf* doh = static_cast<const bf*>(d_o) + h * kMhDh;
+    const bf* kh = static_cast<const bf*>(w_k) + h * F * kMhDh;
+    const bf* uh = static_cast<const bf*>(w_u) + h * F * kMhDh;
+    const bf* vh = static_cast<const bf*>(w_v) + h * F * kMhDh;
+    {  // dP = dO_h V_h^T
+      CUtensorMap ta, tb;
+      if (!encode_tmap_bf16(&ta, doh, kMhDh, T, ld, 64, 128) ||
+          !encode_tmap_bf16(&tb, vh, kMhDh, F, kMhDh, 64, 128))
+        return SWF_ERR_LAUNCH;
+      TcGemmArgs a = base_args(T, F, 256, kMhDh, 2 * kTileM);
+      a.out0 = w.dp;
+      a.ld_out = F;
+      if ((s = launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_MHFFN_BWD, ta, tb, tb, EpiMaps{},
+                                                                 a, st)) != SWF_OK)
+        return s;
+    }
+    {  // [g | u] = Q_h [K_h ; U_h]^T -> dS_g | dS_u, P, router-gradient partials
+      CUtensorMap ta, tk, tu;
+      if (!encode_tmap_bf16(&ta, qh, kMhDh, T, ld, 64, 128) ||
+          !encode_tmap_bf16(&tk, kh, kMhDh, F, kMhDh, 64, 128) ||
+          !encode_tmap_bf16(&tu, uh, kMhDh, F, kMhDh, 64, 128))
+        return SWF_ERR_LAUNCH;
+      TcGemmArgs a = base_args(T, F, 128, kMhDh, 2 * kTileM);
+      a.aux0 = w.dp;
+      a.ld_aux = F;
+      a.out0 = w.dsgu;
+      a.ld_out = 2 * F;
+      a.d_ff = (int)F;
+      a.p_out = w.p;
+      a.ld_p = F;
+      a.rw = router + h * E;
+      a.ld_rw = H * E;
+      a.sub_dim = (int)de;
+      a.dr_part = w.dr_part + h * (F / 128);
+      a.ld_dr = H * (F / 128);
+      if ((s = launch_tc_pair<256, false, false, true, kEpiMhGrad>(SWF_K_MHFFN_BWD, ta, tk, tu, EpiMaps{},
+                                                                 a, st)) != SWF_OK)
+        return s;
+    }
+    {  // dQ_h = dS_g K_h + dS_u U_h: A = [dS_g | dS_u] (K = 2F), B segments K_h, U_h (MN-major)
+      CUtensorMap ta, tk, tu;
+      if (!encode_tmap_bf16(&ta, w.dsgu, 2 * F, T, 2 * F, 64, 128) ||
+          !encode_tmap_bf16(&tk, kh, kMhDh, F, kMhDh, 64, 64) ||
+          !encode_tmap_bf16(&tu, uh, kMhDh, F, kMhDh, 64, 64))
+        return SWF_ERR_LAUNCH;
+      TcGemmArgs a = base_args(T, kMhDh, 128, 0, 2 * kTileM);
+      a.kb_seg0 = (int)(F / kTileK);
+      a.kb_total = 2 * a.kb_seg0;
+      a.a_koff1 = (int)F;
+      a.out0 = static_cast<bf*>(dq) + h * kMhDh;
+      a.ld_out = ld;
+      if ((s = launch_tc_pair<128, false, true, false, kEpiStore>(SWF_K_MHFFN_BWD, ta, tk, tu, EpiMaps{},
+                                                                a, st)) != SWF_OK)
+        return s;
+    }
+    {  // [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h
+      CUtensorMap ta, tb;
+      if (!encode_tmap_bf16(&ta, w.dsgu, 2 * F, T, 2 * F, 64, 64) ||
+          !encode_tmap_bf16(&tb, qh, kMhDh, T, ld, 64, 64))
+        return SWF_ERR_LAUNCH;
+      if ((s = launch_dw(SWF_K_MHFFN_BWD, ta, tb, 2 * F, kMhDh, T, static_cast<bf*>(dw_k) + h * F * kMhDh,
+                         static_cast<bf*>(dw_u) + h * F * kMhDh, F, w.split, st)) != SWF_OK)
+        return s;
+    }
+    {  // dV_h = P^T dO_h
+      CUtensorMap ta, tb;
+      if (!encode_tmap_bf16(&ta, w.p, F, T, F, 64, 64) || !encode_tmap_bf16(&tb, doh, kMhDh, T, ld, 64, 64))
+        return SWF_ERR_LAUNCH;
+      bf* dv = static_cast<bf*>(dw_v) + h * F * kMhDh;
+      if ((s = launch_dw(SWF_K_MHFFN_BWD, ta, tb, F, kMhDh, T, dv, dv, F, w.split, st)) != SWF_OK) return s;
+    }
+  }
+  ProfScope prof(SWF_K_MHFFN_BWD, st);
+  const int64_t n = T * H * E;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16));
+  mh_dr_reduce_kernel<<<grid, 256, 0, st>>>(w.dr_part, n, (int)(de / 128), drouter);
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}

@@ -38,6 +38,10 @@
 //                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
 //   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
 //                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
+//   kEpiMhGrad     dual [g | u] tile of a FlashFFN head with dP (aux0) and the router weight r of
+//                  the tile's sub-network: dS_g = dP r u SiLU'(g) -> out0[n], dS_u = dP r SiLU(g)
+//                  -> out0[d_ff + n], P = SiLU(g) u r -> p_out, and per tile sum_n dP SiLU(g) u
+//                  -> dr_part[m][nb] (the router gradient's partial over the tile's columns)
 //   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
 //                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
 //                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
@@ -66,7 +70,8 @@ enum : int {
   kEpiPartialF32 = 9,
   kEpiEnergyTopK = 10,
   kEpiHeadNorm = 11,
-  kEpiRouter = 12
+  kEpiRouter = 12,
+  kEpiMhGrad = 13
 };
 constexpr int kTopKMaxGroups = 64;  // kEpiEnergyTopK: groups held in registers per token
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
@@ -106,6 +111,13 @@ struct TcGemmArgs {
   int64_t ld_grp;         // kEpiEnergy*: stride of out0 between groups (0: 1); ld_out is the
                           //   stride between tokens (1 with ld_grp = M: group-major energies)
   float eps;              // kEpiHeadNorm
+  const float* rw;        // kEpiMhGrad: router weights of the head, rw[m * ld_rw + e]
+  int64_t ld_rw;
+  int sub_dim;            //   columns per sub-network (a multiple of the tile's BN / 2)
+  __nv_bfloat16* p_out;   //   P [M][ld_p]
+  int64_t ld_p;
+  float* dr_part;         //   [M][ld_dr] partial router gradients, one per tile column block
+  int64_t ld_dr;
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
   int sel_k;
   int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
@@ -701,7 +713,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m = t.a_m + row;
       const bool row_ok = m < args.M;
 
-      if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
+      if constexpr (EPI == kEpiMhGrad) {
+        static_assert(B_DUAL && BN % 64 == 0, "dual [g | u] tile");
+        const int n_base = t.nb * (BN / 2);
+        const float rv = row_ok ? args.rw[(int64_t)m * args.ld_rw + n_base / args.sub_dim] : 0.f;
+        float dr = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          float g[32], u[32];
+          if (have_acc) {
+            tmem_ld32(t_acc + c, g);
+            tmem_ld32(t_acc + BN / 2 + c, u);
+            tmem_ld_wait_regs(g);
+            pin_regs(u);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
+          }
+          const int n0 = n_base + c;
+          if (!row_ok) continue;
+          const __nv_bfloat16* dpp = static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
+          __nv_bfloat16* gp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
+          __nv_bfloat16* pp = args.p_out + (int64_t)m * args.ld_p + n0;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            if (n0 + v * 8 + 8 <= args.N) {
+              const uint4 dq = *reinterpret_cast<const uint4*>(dpp + v * 8);
+              const uint32_t dw[4] = {dq.x, dq.y, dq.z, dq.w};
+              float sg[8], su[8], pv[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int j = v * 8 + e;
+                const float dp = (e & 1) ? bf16_hi(dw[e >> 1]) : bf16_lo(dw[e >> 1]);
+                const float sgm = sigmoidf_(g[j]);
+                const float a = g[j] * sgm;
+                dr = fmaf(dp, a * u[j], dr);
+                const float dpr = dp * rv;
+                sg[e] = dpr * u[j] * sgm * (1.f + g[j] * (1.f - sgm));
+                su[e] = dpr * a;
+                pv[e] = a * u[j] * rv;
+              }
+              store_bf16x8(gp + v * 8, sg);
+              store_bf16x8(gp + args.d_ff + v * 8, su);
+              store_bf16x8(pp + v * 8, pv);
+            }
+          }
+        }
+        if (row_ok && n_base < args.N) args.dr_part[(int64_t)m * args.ld_dr + t.nb] = dr;
+      } else if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
         constexpr int CW = BN / 2 < 32 ? BN / 2 : 32;
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += CW) {

@@ -105,6 +105,12 @@ def test_mhffn_argument_errors(lib):
     assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, F32, None) == 2     # fp32
     assert f(p, p, p, p, q, p, 256, 16, 128, 15, 384, BF, None) == 3      # unaligned router
     assert f(p, p, p, p, p, p, 256, 16, 128, 15, 384, 9, None) == 1       # bad dtype
+    b = lib.flash_mhffn_bwd
+    assert b(p, p, p, p, p, None, p, p, p, p, p, p, 1 << 30, 256, 16, 128, 15, 384, BF, None) == 1  # null d_o
+    assert b(p, p, p, p, p, p, p, p, p, p, p, p, 1 << 30, 256, 16, 128, 15, 320, BF, None) == 2     # d_e % 128
+    assert b(p, p, p, p, p, p, p, p, p, p, p, None, 0, 256, 16, 128, 15, 384, BF, None) == 4        # no workspace
+    assert lib.flash_mhffn_bwd_workspace_bytes(256, 16, 128, 15, 384, BF) > 256 * 5760 * 8
+    assert lib.flash_mhffn_bwd_workspace_bytes(256, 16, 64, 15, 384, BF) == 0
     g = lib.flash_mhffn_prologue
     assert g(None, p, None, p, p, p, 256, 2048, 16, 128, 15, 1e-6, BF, None) == 1  # null x
     assert g(p, p, None, p, p, p, 256, 2048, 16, 128, 15, -1.0, BF, None) == 1     # eps < 0

@@ -114,3 +114,29 @@ def test_block_prologue_then_fused_forward():
     rr = O.router_weights((f64(pro["x"]) @ f64(pro["w_r"]).T).reshape(T, H, E))
     ref = O.mhffn_forward(qr, f64(wts["w_k"]), f64(wts["w_u"]), f64(wts["w_v"]), rr)["o"]
     assert_close("o", f64(o), ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("T,H,E,de", [
+    (200, 2, 3, 128),    # ragged tokens, three sub-networks
+    (1, 1, 1, 128),      # one token
+    (300, 1, 2, 256),    # two 128-column blocks per sub-network
+    (700, 3, 2, 384),    # the 1.3B sub-network width, odd head count
+])
+def test_backward(T, H, E, de):
+    inp = synth.mhffn_inputs(T, H, 128, E, de, seed=T + 3 * E)
+    t = {k: v.cuda() for k, v in inp.items()}
+    grads = api.flash_mhffn_bwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], t["do"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    ref = O.mhffn_backward(*(f64(inp[k]) for k in ("q", "w_k", "w_u", "w_v", "router", "do")))
+    for name, got in zip(("dq", "dk", "du", "dv", "dr"), grads):
+        assert_close(name, f64(got), ref[name], torch.bfloat16)
+
+
+def test_backward_deterministic():
+    inp = synth.mhffn_inputs(512, 2, 128, 2, 128, seed=31)
+    t = {k: v.cuda() for k, v in inp.items()}
+    args = (t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], t["do"])
+    a, b = api.flash_mhffn_bwd(*args), api.flash_mhffn_bwd(*args)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
