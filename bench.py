@@ -408,9 +408,24 @@ def secondary_mhffn(api, steps, warmup, world, peak):
         block()
     ms_b = timed(block, steps, world)
     flops_b = flops + 2.0 * T * d_model * (H * dh + H * E)
+    # backward (per-head GEMMs; writes the head's activations to a workspace)
+    dout = synth.normal((T, H, dh), synth.DY_STD, w["seed"], "do").to(dev)
+    gq, gk, gu, gv, gr = (torch.empty_like(t[k]) for k in ("q", "w_k", "w_u", "w_v", "router"))
+    ws = torch.empty(max(16, api.flash_mhffn_bwd_workspace_bytes(T, H, dh, E, de)), device=dev,
+                     dtype=torch.uint8)
+
+    def bwd():
+        api.flash_mhffn_bwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], dout, gq, gk, gu, gv, gr, ws)
+    for _ in range(warmup):
+        bwd()
+    ms_bwd = timed(bwd, max(3, steps // 4), world)
+    flops_bwd = 16.0 * T * H * dh * E * de
+    del ws
     return {"workload": w["name"], "tflops": round(tf * world, 1), "pct_of_peak": round(100 * tf / peak, 2),
             "ms_per_step": round(ms / steps, 3), "steps": steps, "flops_per_step": flops,
             "intermediate_bytes_not_written": 2 * T * H * E * de,
+            "backward": {"ms_per_step": round(ms_bwd / max(3, steps // 4), 3), "flops_per_step": flops_bwd,
+                         "tflops": round(flops_bwd * max(3, steps // 4) / (ms_bwd / 1e3) / 1e12 * world, 1)},
             "block_from_x": {"ms_per_step": round(ms_b / steps, 3),
                              "tflops": round(flops_b * steps / (ms_b / 1e3) / 1e12 * world, 1),
                              "flops_per_step": flops_b, "d_model": d_model}}

@@ -365,8 +365,11 @@ typedef enum swf_kernel_kind {
   SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
   SWF_K_MHFFN_FWD = 26,    /* FlashFFN multi-head FFN forward (fused, one kernel) */
   SWF_K_MHFFN_PROLOGUE = 27, /* FlashFFN prologue: head-normalised projection, router */
-  SWF_K_MHFFN_BWD = 28,    /* FlashFFN multi-head FFN backward (per-head GEMMs) */
-  SWF_K_NUM_KINDS = 29
+  SWF_K_MHFFN_BWD_DP = 28, /* FlashFFN backward: dP = dO V^T */
+  SWF_K_MHFFN_BWD_DS = 29, /* FlashFFN backward: Q [K;U]^T with the gradient epilogue; dR sums */
+  SWF_K_MHFFN_BWD_DQ = 30, /* FlashFFN backward: dQ */
+  SWF_K_MHFFN_BWD_DW = 31, /* FlashFFN backward: dK, dU, dV */
+  SWF_K_NUM_KINDS = 32
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

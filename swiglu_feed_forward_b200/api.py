@@ -149,6 +149,11 @@ def flash_mhffn_fwd(q, w_k, w_u, w_v, router, o=None, stream=None):
     return o
 
 
+def flash_mhffn_bwd_workspace_bytes(T, num_heads, head_dim, num_sub, sub_dim, dtype=torch.bfloat16):
+    return _lib.lib().flash_mhffn_bwd_workspace_bytes(T, num_heads, head_dim, num_sub, sub_dim,
+                                                      SWF_BF16 if dtype == torch.bfloat16 else SWF_F32)
+
+
 def flash_mhffn_bwd(q, w_k, w_u, w_v, router, d_o, dq=None, dw_k=None, dw_u=None, dw_v=None,
                     drouter=None, workspace=None, stream=None):
     """Gradients of sum(d_o * flash_mhffn_fwd(q, w_k, w_u, w_v, router)).
@@ -160,7 +165,7 @@ def flash_mhffn_bwd(q, w_k, w_u, w_v, router, d_o, dq=None, dw_k=None, dw_u=None
     dw_u = torch.empty_like(w_u) if dw_u is None else dw_u
     dw_v = torch.empty_like(w_v) if dw_v is None else dw_v
     drouter = torch.empty_like(router) if drouter is None else drouter
-    nb = _lib.lib().flash_mhffn_bwd_workspace_bytes(T, H, dh, E, de, _dt(q))
+    nb = flash_mhffn_bwd_workspace_bytes(T, H, dh, E, de, q.dtype)
     if workspace is None:
         workspace = torch.empty(max(16, nb), device=q.device, dtype=torch.uint8)
     _check("flash_mhffn_bwd", _lib.lib().flash_mhffn_bwd(

@@ -47,7 +47,7 @@ __global__ void splitk_reduce_kernel(const float4* __restrict__ part, int64_t pl
 
 // K splits the planner gives a weight-gradient GEMM of rows x cols over K (pair tiles 256 x 256).
 int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
-  const int64_t tiles = (int64_t)cdiv(rows, 2 * kTileM) * cdiv(cols, 256);
+  const int64_t tiles = (int64_t)cdiv(rows, 2 * kTileM) * cdiv(cols, cols <= 128 ? 128 : 256);
   const int kb = cdiv(K, kTileK);
   const int ks = choose_ksplit(tiles, kb, rows * cols);
   return ks > 1 ? cdiv(kb, cdiv(kb, ks)) : 1;  // no empty trailing split
@@ -55,13 +55,33 @@ int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
 
 }  // namespace
 
+swf_status splitk_reduce(const float* part, int ks, int64_t rows, int64_t cols, int64_t row_split,
+                         void* out0, void* out1, cudaStream_t st);
+
 // Weight-gradient GEMM (both operands MN-major, K = tokens): split-K into fp32 partial planes
 // plus a fixed-order reduction when the planner finds too few output tiles, else direct stores.
 swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
                      int64_t cols, int64_t K, void* out0, void* out1, int64_t row_split,
                      float* part, cudaStream_t st) {
-  TcGemmArgs a = base_args(rows, cols, 256, K, 2 * kTileM);
   const int ks = dw_ksplit(rows, cols, K);
+  if (cols <= 128) {  // narrow outputs: pair tiles of 256 x 128
+    TcGemmArgs a = base_args(rows, cols, 128, K, 2 * kTileM);
+    if (ks <= 1) {
+      a.out0 = out0;
+      a.out1 = out1;
+      a.row_split = (int)row_split;
+      a.ld_out = cols;
+      return launch_tc_pair<128, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st);
+    }
+    a.ksplit = ks;
+    a.kb_per_split = cdiv(a.kb_total, ks);
+    a.part = part;
+    a.part_plane = rows * cols;
+    swf_status s = launch_tc_pair<128, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st);
+    if (s != SWF_OK) return s;
+    return splitk_reduce(part, ks, rows, cols, row_split, out0, out1, st);
+  }
+  TcGemmArgs a = base_args(rows, cols, 256, K, 2 * kTileM);
   if (ks <= 1) {
     a.out0 = out0;
     a.out1 = out1;
@@ -75,6 +95,11 @@ swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int
   a.part_plane = rows * cols;
   swf_status s = launch_tc_pair<256, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st);
   if (s != SWF_OK) return s;
+  return splitk_reduce(part, ks, rows, cols, row_split, out0, out1, st);
+}
+
+swf_status splitk_reduce(const float* part, int ks, int64_t rows, int64_t cols, int64_t row_split,
+                         void* out0, void* out1, cudaStream_t st) {
   ProfScope prof(SWF_K_SPLITK_REDUCE, st);
   const int64_t n8 = rows * cols / 8;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 148 * 16));

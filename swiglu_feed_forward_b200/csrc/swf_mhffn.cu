@@ -609,11 +609,12 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
       if (!encode_tmap_bf16(&ta, doh, kMhDh, T, ld, 64, 128) ||
           !encode_tmap_bf16(&tb, vh, kMhDh, F, kMhDh, 64, 128))
         return SWF_ERR_LAUNCH;
+      EpiMaps em{};  // dP leaves through the TMA epilogue's staging boxes
+      if (!encode_tmap_bf16(&em.o[0], w.dp, F, T, F, 32, 32, 64)) return SWF_ERR_LAUNCH;
+      em.o[1] = em.o[0];
       TcGemmArgs a = base_args(T, F, 256, kMhDh, 2 * kTileM);
-      a.out0 = w.dp;
-      a.ld_out = F;
-      if ((s = launch_tc_pair<256, false, false, false, kEpiStore>(SWF_K_MHFFN_BWD, ta, tb, tb, EpiMaps{},
-                                                                 a, st)) != SWF_OK)
+      if ((s = launch_tc_pair<256, false, false, false, kEpiStore, true>(SWF_K_MHFFN_BWD_DP, ta, tb, tb, em,
+                                                                       a, st)) != SWF_OK)
         return s;
     }
     {  // [g | u] = Q_h [K_h ; U_h]^T -> dS_g | dS_u, P, router-gradient partials
@@ -622,21 +623,22 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
           !encode_tmap_bf16(&tk, kh, kMhDh, F, kMhDh, 64, 128) ||
           !encode_tmap_bf16(&tu, uh, kMhDh, F, kMhDh, 64, 128))
         return SWF_ERR_LAUNCH;
+      // TMA epilogue: dS_g, dS_u (two views of dSGU) and P leave through 32 x 32 staging boxes,
+      // dP comes in the same way
+      EpiMaps em{};
+      if (!encode_tmap_bf16(&em.o[0], w.dsgu, F, T, 2 * F, 32, 32, 64) ||
+          !encode_tmap_bf16(&em.o[1], w.dsgu + F, F, T, 2 * F, 32, 32, 64) ||
+          !encode_tmap_bf16(&em.o[2], w.p, F, T, F, 32, 32, 64) ||
+          !encode_tmap_bf16(&em.o[3], w.dp, F, T, F, 32, 32, 64))
+        return SWF_ERR_LAUNCH;
       TcGemmArgs a = base_args(T, F, 128, kMhDh, 2 * kTileM);
-      a.aux0 = w.dp;
-      a.ld_aux = F;
-      a.out0 = w.dsgu;
-      a.ld_out = 2 * F;
-      a.d_ff = (int)F;
-      a.p_out = w.p;
-      a.ld_p = F;
       a.rw = router + h * E;
       a.ld_rw = H * E;
       a.sub_dim = (int)de;
       a.dr_part = w.dr_part + h * (F / 128);
       a.ld_dr = H * (F / 128);
-      if ((s = launch_tc_pair<256, false, false, true, kEpiMhGrad>(SWF_K_MHFFN_BWD, ta, tk, tu, EpiMaps{},
-                                                                 a, st)) != SWF_OK)
+      if ((s = launch_tc_pair<256, false, false, true, kEpiMhGrad, true>(SWF_K_MHFFN_BWD_DS, ta, tk, tu,
+                                                                       em, a, st)) != SWF_OK)
         return s;
     }
     {  // dQ_h = dS_g K_h + dS_u U_h: A = [dS_g | dS_u] (K = 2F), B segments K_h, U_h (MN-major)
@@ -651,7 +653,7 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
       a.a_koff1 = (int)F;
       a.out0 = static_cast<bf*>(dq) + h * kMhDh;
       a.ld_out = ld;
-      if ((s = launch_tc_pair<128, false, true, false, kEpiStore>(SWF_K_MHFFN_BWD, ta, tk, tu, EpiMaps{},
+      if ((s = launch_tc_pair<128, false, true, false, kEpiStore>(SWF_K_MHFFN_BWD_DQ, ta, tk, tu, EpiMaps{},
                                                                 a, st)) != SWF_OK)
         return s;
     }
@@ -660,7 +662,7 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
       if (!encode_tmap_bf16(&ta, w.dsgu, 2 * F, T, 2 * F, 64, 64) ||
           !encode_tmap_bf16(&tb, qh, kMhDh, T, ld, 64, 64))
         return SWF_ERR_LAUNCH;
-      if ((s = launch_dw(SWF_K_MHFFN_BWD, ta, tb, 2 * F, kMhDh, T, static_cast<bf*>(dw_k) + h * F * kMhDh,
+      if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, 2 * F, kMhDh, T, static_cast<bf*>(dw_k) + h * F * kMhDh,
                          static_cast<bf*>(dw_u) + h * F * kMhDh, F, w.split, st)) != SWF_OK)
         return s;
     }
@@ -669,10 +671,10 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
       if (!encode_tmap_bf16(&ta, w.p, F, T, F, 64, 64) || !encode_tmap_bf16(&tb, doh, kMhDh, T, ld, 64, 64))
         return SWF_ERR_LAUNCH;
       bf* dv = static_cast<bf*>(dw_v) + h * F * kMhDh;
-      if ((s = launch_dw(SWF_K_MHFFN_BWD, ta, tb, F, kMhDh, T, dv, dv, F, w.split, st)) != SWF_OK) return s;
+      if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, F, kMhDh, T, dv, dv, F, w.split, st)) != SWF_OK) return s;
     }
   }
-  ProfScope prof(SWF_K_MHFFN_BWD, st);
+  ProfScope prof(SWF_K_MHFFN_BWD_DS, st);
   const int64_t n = T * H * E;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16));
   mh_dr_reduce_kernel<<<grid, 256, 0, st>>>(w.dr_part, n, (int)(de / 128), drouter);

@@ -38,10 +38,10 @@
 //                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
 //   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
 //                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
-//   kEpiMhGrad     dual [g | u] tile of a FlashFFN head with dP (aux0) and the router weight r of
-//                  the tile's sub-network: dS_g = dP r u SiLU'(g) -> out0[n], dS_u = dP r SiLU(g)
-//                  -> out0[d_ff + n], P = SiLU(g) u r -> p_out, and per tile sum_n dP SiLU(g) u
-//                  -> dr_part[m][nb] (the router gradient's partial over the tile's columns)
+//   kEpiMhGrad     (TMA epilogue only) dual [g | u] tile of a FlashFFN head with dP (TMA-loaded)
+//                  and the router weight r of the tile's sub-network: outputs dS_g = dP r u
+//                  SiLU'(g), dS_u = dP r SiLU(g), P = SiLU(g) u r, and per tile the router
+//                  gradient's partial sum_n dP SiLU(g) u -> dr_part[m][nb]
 //   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
 //                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
 //                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
@@ -114,8 +114,6 @@ struct TcGemmArgs {
   const float* rw;        // kEpiMhGrad: router weights of the head, rw[m * ld_rw + e]
   int64_t ld_rw;
   int sub_dim;            //   columns per sub-network (a multiple of the tile's BN / 2)
-  __nv_bfloat16* p_out;   //   P [M][ld_p]
-  int64_t ld_p;
   float* dr_part;         //   [M][ld_dr] partial router gradients, one per tile column block
   int64_t ld_dr;
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
@@ -134,11 +132,15 @@ struct TcGemmArgs {
 // loaded by TMA into the same kind of buffers.
 template <int EPI>
 constexpr int tma_epi_outputs() {
-  return EPI == kEpiSwiGLU ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
+  return (EPI == kEpiSwiGLU || EPI == kEpiMhGrad) ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
 }
 template <int EPI>
 constexpr int tma_epi_aux() {
-  return EPI == kEpiDGate ? 2 : (EPI == kEpiScale ? 1 : 0);
+  return EPI == kEpiDGate ? 2 : ((EPI == kEpiScale || EPI == kEpiMhGrad) ? 1 : 0);
+}
+template <int EPI>
+constexpr int aux_map0() {
+  return EPI == kEpiMhGrad ? 3 : 2;
 }
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <int EPI, bool TMA_EPI>
@@ -147,7 +149,8 @@ constexpr int epi_smem_bytes() {
                                : (TMA_EPI ? 4 * (tma_epi_outputs<EPI>() + tma_epi_aux<EPI>()) * 2 * kEpiBox : 0);
 }
 
-// Tensor maps of a TMA epilogue: outputs in o[0..], kEpiDGate's a/b factors in o[2], o[3].
+// Tensor maps of a TMA epilogue: outputs in o[0..], then the factors it loads by TMA from
+// o[aux_map0<EPI>()] on (kEpiDGate's a/b in o[2], o[3]; kEpiScale's in o[2]; kEpiMhGrad's dP in o[3]).
 struct EpiMaps {
   CUtensorMap o[4];
 };
@@ -343,7 +346,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
                                                     EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
-                                                    EPI == kEpiScale || EPI == kEpiLeakySq)) ||
+                                                    EPI == kEpiScale || EPI == kEpiLeakySq ||
+                                                    EPI == kEpiMhGrad)) ||
                     (MODE == kModeRowGrouped && EPI == kEpiStore),
                 "TMA epilogue: dense bf16 outputs, or row-grouped plain stores");
 
@@ -520,7 +524,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int NOUT = tma_epi_outputs<EPI>();
     constexpr int NAUX = tma_epi_aux<EPI>();
     constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
-    constexpr int NCH = (kGLU ? BN / 2 : BN) / 32;
+    constexpr bool kDual = kGLU || EPI == kEpiMhGrad;  // [g | u] accumulator halves
+    constexpr int NCH = (kDual ? BN / 2 : BN) / 32;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
     uint8_t* ebase = smem + L::kEpiOffset + ew * (NOUT + NAUX) * 2 * kEpiBox;
@@ -539,13 +544,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       ++local;
       const int m_slab = t.a_m + q * 32;
-      const int n_base = t.nb * (kGLU ? BN / 2 : BN);
+      const int n_base = t.nb * (kDual ? BN / 2 : BN);
       auto issue_aux = [&](int c) {
         if constexpr (NAUX > 0) {
           if (lane == 0) {
             const int db = aux_issued & 1;
             mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
-            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[2], n_base + c * 32, m_slab, &abar[db]);
+            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[aux_map0<EPI>()], n_base + c * 32, m_slab,
+                        &abar[db]);
             if constexpr (NAUX > 1)
               tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
           }
@@ -562,6 +568,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
       const bool have_acc = t.kb > 0;
+      float mh_r = 0.f, mh_dr = 0.f;  // kEpiMhGrad: the row's router weight, gradient partial
+      if constexpr (EPI == kEpiMhGrad) {
+        if (m_slab + lane < args.M) mh_r = args.rw[(int64_t)(m_slab + lane) * args.ld_rw + n_base / args.sub_dim];
+      }
 #pragma unroll 1
       for (int c = 0; c < NCH; ++c) {
         const uint8_t* aux = nullptr;
@@ -580,8 +590,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float v0[32], v1[32];
         if (have_acc) {
           tmem_ld32(t_acc + c * 32, v0);
-          if constexpr (kGLU) tmem_ld32(t_acc + BN / 2 + c * 32, v1);
-          tmem_ld_wait();
+          if constexpr (kDual) tmem_ld32(t_acc + BN / 2 + c * 32, v1);
+          tmem_ld_wait_regs(v0);
+          if constexpr (kDual) pin_regs(v1);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0.f;
@@ -632,6 +643,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               w[0][c4 * 4 + p] = pack_bf16x2(v0[c4 * 8 + p * 2] * bf16_lo(aw[p]),
                                              v0[c4 * 8 + p * 2 + 1] * bf16_hi(aw[p]));
           }
+        } else if constexpr (EPI == kEpiMhGrad) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 dv = *reinterpret_cast<const uint4*>(aux + lane * 64 + ((c4 ^ swz) * 16));
+            const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              float sg[2], su[2], pv[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = c4 * 8 + p * 2 + e;
+                const float g = v0[j], u = v1[j];
+                const float dp = e ? bf16_hi(dw[p]) : bf16_lo(dw[p]);
+                const float sgm = sigmoidf_(g);
+                const float a = g * sgm;
+                mh_dr = fmaf(dp, a * u, mh_dr);
+                const float dpr = dp * mh_r;
+                sg[e] = dpr * u * sgm * (1.f + g * (1.f - sgm));
+                su[e] = dpr * a;
+                pv[e] = a * u * mh_r;
+              }
+              w[0][c4 * 4 + p] = pack_bf16x2(sg[0], sg[1]);
+              w[1][c4 * 4 + p] = pack_bf16x2(su[0], su[1]);
+              w[2][c4 * 4 + p] = pack_bf16x2(pv[0], pv[1]);
+            }
+          }
         } else if constexpr (EPI == kEpiDGate) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
@@ -679,6 +716,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ++chunks;
       }
       if (!ok) break;
+      if constexpr (EPI == kEpiMhGrad) {
+        if (m_slab + lane < args.M && n_base < args.N)
+          args.dr_part[(int64_t)(m_slab + lane) * args.ld_dr + t.nb] = mh_dr;
+      }
       tc_fence_before();
       if (PAIR && rank != 0) mbar_arrive_remote(tempty_lead + buf * 8);  // TMEM read: own SM
       else mbar_arrive(&tempty[buf]);
@@ -713,54 +754,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m = t.a_m + row;
       const bool row_ok = m < args.M;
 
-      if constexpr (EPI == kEpiMhGrad) {
-        static_assert(B_DUAL && BN % 64 == 0, "dual [g | u] tile");
-        const int n_base = t.nb * (BN / 2);
-        const float rv = row_ok ? args.rw[(int64_t)m * args.ld_rw + n_base / args.sub_dim] : 0.f;
-        float dr = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          float g[32], u[32];
-          if (have_acc) {
-            tmem_ld32(t_acc + c, g);
-            tmem_ld32(t_acc + BN / 2 + c, u);
-            tmem_ld_wait_regs(g);
-            pin_regs(u);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
-          }
-          const int n0 = n_base + c;
-          if (!row_ok) continue;
-          const __nv_bfloat16* dpp = static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
-          __nv_bfloat16* gp = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
-          __nv_bfloat16* pp = args.p_out + (int64_t)m * args.ld_p + n0;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (n0 + v * 8 + 8 <= args.N) {
-              const uint4 dq = *reinterpret_cast<const uint4*>(dpp + v * 8);
-              const uint32_t dw[4] = {dq.x, dq.y, dq.z, dq.w};
-              float sg[8], su[8], pv[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int j = v * 8 + e;
-                const float dp = (e & 1) ? bf16_hi(dw[e >> 1]) : bf16_lo(dw[e >> 1]);
-                const float sgm = sigmoidf_(g[j]);
-                const float a = g[j] * sgm;
-                dr = fmaf(dp, a * u[j], dr);
-                const float dpr = dp * rv;
-                sg[e] = dpr * u[j] * sgm * (1.f + g[j] * (1.f - sgm));
-                su[e] = dpr * a;
-                pv[e] = a * u[j] * rv;
-              }
-              store_bf16x8(gp + v * 8, sg);
-              store_bf16x8(gp + args.d_ff + v * 8, su);
-              store_bf16x8(pp + v * 8, pv);
-            }
-          }
-        }
-        if (row_ok && n_base < args.N) args.dr_part[(int64_t)m * args.ld_dr + t.nb] = dr;
-      } else if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
+      if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf) {
         constexpr int CW = BN / 2 < 32 ? BN / 2 : 32;
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += CW) {
