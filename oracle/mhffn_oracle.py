@@ -39,7 +39,8 @@ import numpy as np
 
 from .swiglu_oracle import silu, silu_prime
 
-__all__ = ["mhffn_forward", "mhffn_backward", "head_rmsnorm", "router_weights"]
+__all__ = ["mhffn_forward", "mhffn_backward", "head_rmsnorm", "router_weights",
+           "mhffn_prologue_forward", "mhffn_prologue_backward"]
 
 
 def _f64(a):
@@ -97,3 +98,39 @@ def router_weights(logits):
     sub-networks of each head.  logits [T, H, E]."""
     s = 1.0 / (1.0 + np.exp(-_f64(logits)))
     return s / np.sum(s, axis=-1, keepdims=True)
+
+
+def mhffn_prologue_forward(x, w_q, w_r, num_heads, num_sub, gain=None, eps=1e-6):
+    """The block's prologue: q = head_rmsnorm(x w_q^T) [T, H, dh] and router weights
+    r = router_weights((x w_r^T) as [T, H, E])."""
+    x, w_q, w_r = _f64(x), _f64(w_q), _f64(w_r)
+    T = x.shape[0]
+    q = head_rmsnorm(x @ w_q.T, num_heads, eps, gain)
+    r = router_weights((x @ w_r.T).reshape(T, num_heads, num_sub))
+    return {"q": q, "r": r}
+
+
+def mhffn_prologue_backward(x, w_q, w_r, num_heads, num_sub, dq, dr, gain=None, eps=1e-6):
+    """Gradients of L = sum(dq * q) + sum(dr * r) for the prologue above with respect to x,
+    w_q, w_r and the gain (chain rule through the RMS normalisation and the normalised
+    sigmoid)."""
+    x, w_q, w_r, dq, dr = (_f64(a) for a in (x, w_q, w_r, dq, dr))
+    T = x.shape[0]
+    H, E = num_heads, num_sub
+    z = (x @ w_q.T).reshape(T, H, -1)
+    dh = z.shape[-1]
+    inv = 1.0 / np.sqrt(np.mean(z * z, axis=-1, keepdims=True) + eps)
+    n = z * inv
+    g = np.ones(dh) if gain is None else _f64(gain)
+    dgain = np.einsum("thd,thd->d", dq, n)
+    dn = dq * g
+    dz = inv * (dn - n * np.mean(dn * n, axis=-1, keepdims=True))
+    l = (x @ w_r.T).reshape(T, H, E)
+    sg = 1.0 / (1.0 + np.exp(-l))
+    S = np.sum(sg, axis=-1, keepdims=True)
+    r = sg / S
+    ds = (dr - np.sum(dr * r, axis=-1, keepdims=True)) / S
+    dl = ds * sg * (1.0 - sg)
+    dz2, dl2 = dz.reshape(T, H * dh), dl.reshape(T, H * E)
+    dx = dz2 @ w_q + dl2 @ w_r
+    return {"dx": dx, "dw_q": dz2.T @ x, "dw_r": dl2.T @ x, "dgain": dgain}

@@ -426,3 +426,34 @@ def test_head_rmsnorm_and_router_weights():
     # order follows the logits; sigmoid(0) = 1/2 against sigmoid(large) ~ 1
     w2 = O.router_weights(np.array([[[0.0, 50.0]]]))
     np.testing.assert_allclose(w2[0, 0], [1 / 3, 2 / 3], rtol=1e-12)
+
+
+@pytest.mark.parametrize("use_gain", [True, False])
+def test_mhffn_prologue_backward_matches_autograd_and_fd(use_gain):
+    T, d, H, dh, E = 5, 12, 3, 4, 3
+    x, wq, wr = rnd((T, d), 90), rnd((H * dh, d), 91, d ** -0.5), rnd((H * E, d), 92, d ** -0.5)
+    gain = np.random.default_rng(93).uniform(0.5, 1.5, dh) if use_gain else None
+    dq, dr = rnd((T, H, dh), 94, 0.1), rnd((T, H, E), 95, 0.1)
+    ts = [torch.from_numpy(a.copy()).requires_grad_(True) for a in (x, wq, wr)]
+    tg = torch.from_numpy(gain.copy()).requires_grad_(True) if use_gain else None
+    z = (ts[0] @ ts[1].T).reshape(T, H, dh)
+    qn = z / torch.sqrt((z * z).mean(-1, keepdim=True) + 1e-6)
+    if use_gain:
+        qn = qn * tg
+    sg = torch.sigmoid((ts[0] @ ts[2].T).reshape(T, H, E))
+    rr = sg / sg.sum(-1, keepdim=True)
+    fw = O.mhffn_prologue_forward(x, wq, wr, H, E, gain, 1e-6)
+    np.testing.assert_allclose(fw["q"], qn.detach().numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(fw["r"], rr.detach().numpy(), rtol=1e-12, atol=1e-14)
+    ((qn * torch.from_numpy(dq)).sum() + (rr * torch.from_numpy(dr)).sum()).backward()
+    bw = O.mhffn_prologue_backward(x, wq, wr, H, E, dq, dr, gain, 1e-6)
+    for name, t in zip(("dx", "dw_q", "dw_r"), ts):
+        np.testing.assert_allclose(bw[name], t.grad.numpy(), rtol=1e-10, atol=1e-12)
+    if use_gain:
+        np.testing.assert_allclose(bw["dgain"], tg.grad.numpy(), rtol=1e-10, atol=1e-12)
+    xs, wqs, wrs = x[:2].copy(), wq.copy(), wr.copy()
+    dqs, drs = dq[:2].copy(), dr[:2].copy()
+    loss = lambda: float(np.sum(dqs * O.mhffn_prologue_forward(xs, wqs, wrs, H, E, gain, 1e-6)["q"])
+                         + np.sum(drs * O.mhffn_prologue_forward(xs, wqs, wrs, H, E, gain, 1e-6)["r"]))
+    b2 = O.mhffn_prologue_backward(xs, wqs, wrs, H, E, dqs, drs, gain, 1e-6)
+    _fd_check(loss, [xs, wqs, wrs], [b2["dx"], b2["dw_q"], b2["dw_r"]], tol=1e-5)
