@@ -225,6 +225,22 @@ swf_status flash_mhffn_prologue(const void* x, const void* w_q, const float* q_g
                                 int64_t d_model, int32_t num_heads, int32_t head_dim,
                                 int32_t num_sub, float eps, swf_dtype dtype, void* stream);
 
+/* Backward of flash_mhffn_prologue given dq [T, num_heads * head_dim] (bf16) and drouter
+ * [T, num_heads, num_sub] (fp32): dx [T, d_model], dw_q, dw_r (shapes of w_q, w_r) and, when
+ * both q_gain and dq_gain are given, dq_gain [head_dim] fp32 (dq_gain alone: written as zeros).
+ * The projection and router GEMMs are recomputed with the normalisations' backward in their
+ * epilogues; then dx = [dz | dl] [w_q ; w_r] and [dw_q ; dw_r] = [dz | dl]^T x.  Workspace:
+ * flash_mhffn_prologue_bwd_workspace_bytes bytes.  Same support rules and error codes as the
+ * forward; outputs overwritten; deterministic. */
+swf_status flash_mhffn_prologue_bwd(const void* x, const void* w_q, const float* q_gain,
+                                    const void* w_r, const void* dq, const float* drouter,
+                                    void* dx, void* dw_q, float* dq_gain, void* dw_r,
+                                    void* workspace, size_t workspace_bytes, int64_t T,
+                                    int64_t d_model, int32_t num_heads, int32_t head_dim,
+                                    int32_t num_sub, float eps, swf_dtype dtype, void* stream);
+size_t flash_mhffn_prologue_bwd_workspace_bytes(int64_t T, int64_t d_model, int32_t num_heads,
+                                                int32_t head_dim, int32_t num_sub, swf_dtype dtype);
+
 /* ------------------------------------------------------------------ group-sparse variant */
 
 /* Subsample index (eugen_sparse README, make_subsample_index; drawn once per layer).  HOST

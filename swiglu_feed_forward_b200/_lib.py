@@ -41,6 +41,9 @@ SIGNATURES = {
     "flash_mhffn_prologue": (I32, [P, P, P, P, P, P, I64, I64, I32, I32, I32, C.c_float, I32, P]),
     "flash_mhffn_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, SZ, I64, I32, I32, I32, I32, I32, P]),
     "flash_mhffn_bwd_workspace_bytes": (SZ, [I64, I32, I32, I32, I32, I32]),
+    "flash_mhffn_prologue_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, SZ, I64, I64, I32, I32, I32,
+                                       C.c_float, I32, P]),
+    "flash_mhffn_prologue_bwd_workspace_bytes": (SZ, [I64, I64, I32, I32, I32, I32]),
     "swf_make_subsample_index": (I32, [I64, I32, I32, U64, P]),
     "grouped_topk_select": (I32, [P, P, P, I32, P, I32, I32, P, P, P, SZ, I64, I64, I64, I32, P]),
     "swf_group_buckets": (I32, [P, I64, I32, I32, P, P, P, SZ, P]),

@@ -189,6 +189,26 @@ def flash_mhffn_prologue(x, w_q, w_r, num_heads, num_sub, q_gain=None, eps=1e-6,
     return q, router
 
 
+def flash_mhffn_prologue_bwd(x, w_q, w_r, num_heads, num_sub, dq, drouter, q_gain=None, eps=1e-6,
+                             dx=None, dw_q=None, dw_r=None, dq_gain=None, workspace=None, stream=None):
+    """Backward of flash_mhffn_prologue: returns (dx, dw_q, dw_r, dq_gain or None)."""
+    T, d = x.shape
+    dh = w_q.shape[0] // num_heads
+    dx = torch.empty_like(x) if dx is None else dx
+    dw_q = torch.empty_like(w_q) if dw_q is None else dw_q
+    dw_r = torch.empty_like(w_r) if dw_r is None else dw_r
+    if q_gain is not None and dq_gain is None:
+        dq_gain = torch.empty_like(q_gain)
+    nb = _lib.lib().flash_mhffn_prologue_bwd_workspace_bytes(T, d, num_heads, dh, num_sub, _dt(x))
+    if workspace is None:
+        workspace = torch.empty(max(16, nb), device=x.device, dtype=torch.uint8)
+    _check("flash_mhffn_prologue_bwd", _lib.lib().flash_mhffn_prologue_bwd(
+        _p(x), _p(w_q), _p(q_gain), _p(w_r), _p(dq), _p(drouter), _p(dx), _p(dw_q), _p(dq_gain), _p(dw_r),
+        _p(workspace), workspace.numel() * workspace.element_size(), T, d, num_heads, dh, num_sub,
+        float(eps), _dt(x), _stream(stream)))
+    return dx, dw_q, dw_r, dq_gain
+
+
 # ------------------------------------------------------------------ group-sparse
 def make_subsample_index(d_ff, group_size, samples_per_group, seed):
     """Host call: returns (int32 CPU tensor [d_ff // group_size, spg], spg)."""

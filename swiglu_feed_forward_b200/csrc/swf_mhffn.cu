@@ -680,3 +680,145 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
   mh_dr_reduce_kernel<<<grid, 256, 0, st>>>(w.dr_part, n, (int)(de / 128), drouter);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
+
+// ------------------------------------------------------------------ prologue backward
+// Gradients of the prologue given dq and drouter: the projection and router GEMMs are recomputed
+// with epilogues that apply the normalisations' backward (kEpiHeadNormBwd: dz and the gain's
+// partial sums; kEpiRouterBwd: dl), writing dz | dl side by side; then dx = [dz | dl] [W_q ; W_r]
+// (two K segments) and [dW_q ; dW_r] = [dz | dl]^T x (split-K weight-gradient GEMM); one kernel
+// sums the gain partials in a fixed order.
+namespace swf {
+namespace {
+
+__global__ void dgain_reduce_kernel(const float* __restrict__ part, int64_t rows, float* __restrict__ dgain) {
+  const int i = threadIdx.x;  // 128 columns
+  float s = 0.f;
+  for (int64_t r = 0; r < rows; ++r) s += part[r * 128 + i];
+  dgain[i] = s;
+}
+
+struct ProBwdWs {
+  __nv_bfloat16* dzl;
+  float *sig, *gain_part, *split;
+  int64_t ld;
+};
+
+ProBwdWs pro_bwd_ws(void* base, int64_t T, int64_t d_model, int64_t H, int64_t E, size_t* bytes) {
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    off = round_up(off, 256);
+    char* p = base ? static_cast<char*>(base) + off : nullptr;
+    off += n;
+    return p;
+  };
+  const int64_t nq = H * kMhDh, nr = H * E;
+  ProBwdWs w;
+  w.ld = (int64_t)round_up(nq + nr, 8);
+  w.dzl = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * w.ld * 2));
+  w.sig = reinterpret_cast<float*>(take((size_t)T * nr * 4));
+  w.gain_part = reinterpret_cast<float*>(take((size_t)round_up(T, 256) / 32 * H * 128 * 4));
+  w.split = reinterpret_cast<float*>(take((size_t)std::max<int64_t>(part_elems(nq + nr, d_model, T), 4) * 4));
+  if (bytes) *bytes = off;
+  return w;
+}
+
+swf_status check_pro(int64_t T, int64_t d_model, int32_t H, int32_t dh, int32_t E, float eps, swf_dtype dt) {
+  if (T <= 0 || d_model <= 0 || H <= 0 || dh <= 0 || E <= 0 || !(eps >= 0.f)) return SWF_ERR_INVALID_ARG;
+  if (dt != SWF_BF16 && dt != SWF_F32) return SWF_ERR_INVALID_ARG;
+  if (dt != SWF_BF16 || dh != kMhDh || d_model % 16 != 0 || (int64_t)H * E > 256 || T > INT32_MAX / 2 ||
+      d_model > (1 << 20) || (int64_t)H * kMhDh > (1 << 20))
+    return SWF_ERR_UNSUPPORTED;
+  return SWF_OK;
+}
+
+}  // namespace
+}  // namespace swf
+
+extern "C" size_t flash_mhffn_prologue_bwd_workspace_bytes(int64_t T, int64_t d_model,
+                                                           int32_t num_heads, int32_t head_dim,
+                                                           int32_t num_sub, swf_dtype dtype) {
+  if (check_pro(T, d_model, num_heads, head_dim, num_sub, 0.f, dtype) != SWF_OK) return 0;
+  size_t need = 0;
+  pro_bwd_ws(nullptr, T, d_model, num_heads, num_sub, &need);
+  return need;
+}
+
+extern "C" swf_status flash_mhffn_prologue_bwd(
+    const void* x, const void* w_q, const float* q_gain, const void* w_r, const void* dq,
+    const float* drouter, void* dx, void* dw_q, float* dq_gain, void* dw_r, void* workspace,
+    size_t workspace_bytes, int64_t T, int64_t d_model, int32_t num_heads, int32_t head_dim,
+    int32_t num_sub, float eps, swf_dtype dtype, void* stream) {
+  for (const void* p : std::initializer_list<const void*>{x, w_q, w_r, dq, drouter, dx, dw_q, dw_r})
+    if (!p) return SWF_ERR_INVALID_ARG;
+  swf_status s = check_pro(T, d_model, num_heads, head_dim, num_sub, eps, dtype);
+  if (s != SWF_OK) return s;
+  for (const void* p : std::initializer_list<const void*>{x, w_q, q_gain, w_r, dq, drouter, dx, dw_q,
+                                                          dq_gain, dw_r, workspace})
+    if (p && !aligned16(p)) return SWF_ERR_ALIGNMENT;
+  const int64_t H = num_heads, E = num_sub, nq = H * kMhDh, nr = H * E;
+  size_t need = 0;
+  const ProBwdWs w = pro_bwd_ws(workspace, T, d_model, H, E, &need);
+  if (!workspace || workspace_bytes < need) return SWF_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap tx, tq, tr;
+  if (!encode_tmap_bf16(&tx, x, d_model, T, d_model, 64, 128) ||
+      !encode_tmap_bf16(&tq, w_q, d_model, nq, d_model, 64, 128) ||
+      !encode_tmap_bf16(&tr, w_r, d_model, nr, d_model, 64, 256))
+    return SWF_ERR_LAUNCH;
+  {  // dz from the recomputed projection (one-CTA tiles of one head; the gain partials are per
+     // 32-row slab and head)
+    TcGemmArgs a = base_args(T, nq, 128, d_model);
+    a.aux0 = dq;
+    a.ld_aux = nq;
+    a.bias = q_gain;
+    a.eps = eps;
+    a.out0 = w.dzl;
+    a.ld_out = w.ld;
+    a.dgain_part = (q_gain && dq_gain) ? w.gain_part : nullptr;
+    a.heads = num_heads;
+    if ((s = launch_tc<128, false, false, false, kEpiHeadNormBwd>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st)) != SWF_OK)
+      return s;
+  }
+  {  // dl from the recomputed router logits, into the columns after dz
+    TcGemmArgs a = base_args(T, nr, 256, d_model);
+    a.rw = drouter;
+    a.ld_rw = nr;
+    a.part = w.sig;
+    a.group_size = num_sub;
+    a.out0 = w.dzl + nq;
+    a.ld_out = w.ld;
+    if ((s = launch_tc<256, false, false, false, kEpiRouterBwd>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, a, st)) != SWF_OK)
+      return s;
+  }
+  {  // dx = dz W_q + dl W_r: A = [dz | dl] (K = nq + nr), B segments W_q, W_r (MN-major)
+    CUtensorMap ta, tbq, tbr;
+    if (!encode_tmap_bf16(&ta, w.dzl, nq + nr, T, w.ld, 64, 128) ||
+        !encode_tmap_bf16(&tbq, w_q, d_model, nq, d_model, 64, 64) ||
+        !encode_tmap_bf16(&tbr, w_r, d_model, nr, d_model, 64, 64))
+      return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(T, d_model, 256, 0, 2 * kTileM);
+    a.kb_seg0 = (int)(nq / kTileK);
+    a.kb_total = a.kb_seg0 + cdiv(nr, kTileK);
+    a.a_koff1 = (int)nq;
+    a.out0 = dx;
+    a.ld_out = d_model;
+    if ((s = launch_tc_pair<256, false, true, false, kEpiStore>(SWF_K_MHFFN_PROLOGUE, ta, tbq, tbr, EpiMaps{},
+                                                              a, st)) != SWF_OK)
+      return s;
+  }
+  {  // [dW_q ; dW_r] = [dz | dl]^T x
+    CUtensorMap ta, tb;
+    if (!encode_tmap_bf16(&ta, w.dzl, nq + nr, T, w.ld, 64, 64) || !encode_tmap_bf16(&tb, x, d_model, T, d_model, 64, 64))
+      return SWF_ERR_LAUNCH;
+    if ((s = launch_dw(SWF_K_MHFFN_PROLOGUE, ta, tb, nq + nr, d_model, T, dw_q, dw_r, nq, w.split, st)) != SWF_OK)
+      return s;
+  }
+  if (q_gain && dq_gain) {
+    ProfScope prof(SWF_K_MHFFN_PROLOGUE, st);
+    dgain_reduce_kernel<<<1, 128, 0, st>>>(w.gain_part, (int64_t)cdiv(T, 128) * 4 * H, dq_gain);
+    if (cudaGetLastError() != cudaSuccess) return SWF_ERR_LAUNCH;
+  } else if (dq_gain) {
+    if (cudaMemsetAsync(dq_gain, 0, 128 * sizeof(float), st) != cudaSuccess) return SWF_ERR_LAUNCH;
+  }
+  return SWF_OK;
+}

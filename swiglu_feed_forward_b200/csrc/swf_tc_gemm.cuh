@@ -42,6 +42,13 @@
 //                  and the router weight r of the tile's sub-network: outputs dS_g = dP r u
 //                  SiLU'(g), dS_u = dP r SiLU(g), P = SiLU(g) u r, and per tile the router
 //                  gradient's partial sum_n dP SiLU(g) u -> dr_part[m][nb]
+//   kEpiHeadNormBwd C = z (the projection), heads of 128 columns, with dq (aux0, ld_aux) and the
+//                  gain (bias, nullable): dz = inv (dn - n mean(dn n)), n = z inv, dn = dq gain,
+//                  inv = 1 / sqrt(mean(z^2) + eps) -> bf16 out0; if dgain_part, per 32-row slab
+//                  and head the column sums of dq n -> dgain_part[(m / 32) * heads + h][i]
+//   kEpiRouterBwd  C = router logits l (N <= BN = 256, heads of group_size columns) with dR
+//                  (rw, ld_rw): s = sigmoid(l) -> fp32 scratch (part, ld N) in a first pass, then
+//                  dl = s (1 - s) (dR - sum_e dR R) / sum_e s with R = s / sum_e s -> bf16 out0
 //   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
 //                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
 //                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
@@ -71,7 +78,9 @@ enum : int {
   kEpiEnergyTopK = 10,
   kEpiHeadNorm = 11,
   kEpiRouter = 12,
-  kEpiMhGrad = 13
+  kEpiMhGrad = 13,
+  kEpiHeadNormBwd = 14,
+  kEpiRouterBwd = 15
 };
 constexpr int kTopKMaxGroups = 64;  // kEpiEnergyTopK: groups held in registers per token
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
@@ -116,6 +125,8 @@ struct TcGemmArgs {
   int sub_dim;            //   columns per sub-network (a multiple of the tile's BN / 2)
   float* dr_part;         //   [M][ld_dr] partial router gradients, one per tile column block
   int64_t ld_dr;
+  float* dgain_part;      // kEpiHeadNormBwd (nullable): [M / 32 * heads][128] gain-gradient partials
+  int heads;
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
   int sel_k;
   int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
@@ -822,6 +833,107 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int j = 0; j < 32; ++j) o[j] = v[c][j] * inv * (args.bias ? args.bias[c * 32 + j] : 1.f);
 #pragma unroll
               for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
+            }
+          }
+        }
+      } else if constexpr (EPI == kEpiHeadNormBwd) {
+        static_assert(BN % 128 == 0, "whole heads per tile");
+#pragma unroll 1
+        for (int hd = 0; hd < BN / 128; ++hd) {
+          float z[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(t_acc + hd * 128 + c * 32, z[c]);
+          tmem_ld_wait_regs(z[0]);
+          pin_regs(z[1]);
+          pin_regs(z[2]);
+          pin_regs(z[3]);
+          const int n0 = t.nb * BN + hd * 128;
+          if (n0 >= args.N) continue;  // warp-uniform
+          const __nv_bfloat16* dqp = static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
+          float ss = 0.f, dot = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(z[c][j], z[c][j], ss);
+          const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
+          // dq of this row (zero for rows past M), kept packed
+          uint32_t dqw[4][16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 d4 = row_ok ? *reinterpret_cast<const uint4*>(dqp + c * 32 + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+              dqw[c][v * 4] = d4.x, dqw[c][v * 4 + 1] = d4.y, dqw[c][v * 4 + 2] = d4.z, dqw[c][v * 4 + 3] = d4.w;
+            }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
+              const float nv = z[c][j] * inv;
+              const float dn = dq * (args.bias ? args.bias[c * 32 + j] : 1.f);
+              dot = fmaf(dn, nv, dot);
+            }
+          const float mdot = dot * (1.0f / 128.0f);
+          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
+              const float nv = z[c][j] * inv;
+              const float dn = dq * (args.bias ? args.bias[c * 32 + j] : 1.f);
+              o[j] = inv * (dn - nv * mdot);
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
+            }
+          }
+          if (args.dgain_part) {  // column sums of dq * n over the warp's 32 rows (fixed order)
+            float* gp = args.dgain_part + ((int64_t)((t.a_m + (warp & 3) * 32) / 32) * args.heads + n0 / 128) * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
+                float v = dq * z[c][j] * inv;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == j) gp[c * 32 + j] = v;
+              }
+          }
+        }
+      } else if constexpr (EPI == kEpiRouterBwd) {
+        float* sp = args.part + (int64_t)m * args.N;  // sigmoid scratch row
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float zl[32];
+          tmem_ld32(t_acc + c, zl);
+          tmem_ld_wait_regs(zl);
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st_if(sp + c + j, sigmoidf_(zl[j]), c + j < args.N);
+          }
+        }
+        if (row_ok) {
+          const int E = args.group_size;
+          const float* drp = args.rw + (int64_t)m * args.ld_rw;
+          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out;
+#pragma unroll 1
+          for (int h0 = 0; h0 < args.N; h0 += E) {
+            float S = 0.f;
+#pragma unroll 1
+            for (int e = 0; e < E; ++e) S += sp[h0 + e];
+            const float invS = 1.0f / S;
+            float cdot = 0.f;
+#pragma unroll 1
+            for (int e = 0; e < E; ++e) cdot = fmaf(drp[h0 + e], sp[h0 + e] * invS, cdot);
+#pragma unroll 1
+            for (int e = 0; e < E; ++e) {
+              const float sv = sp[h0 + e];
+              op[h0 + e] = __float2bfloat16_rn(sv * (1.f - sv) * (drp[h0 + e] - cdot) * invS);
             }
           }
         }

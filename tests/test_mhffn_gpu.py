@@ -140,3 +140,30 @@ def test_backward_deterministic():
     a, b = api.flash_mhffn_bwd(*args), api.flash_mhffn_bwd(*args)
     for x, y in zip(a, b):
         assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+@pytest.mark.parametrize("T,d_model,H,E,use_gain", [
+    (300, 256, 3, 5, True),     # odd head count, ragged tokens
+    (1, 64, 1, 1, False),       # one token, one sub-network (router gradient 0)
+    (513, 512, 4, 15, True),    # the 1.3B E
+])
+def test_prologue_backward(T, d_model, H, E, use_gain):
+    pro = synth.mhffn_prologue_inputs(T, d_model, H, 128, E, seed=T + 7)
+    dq = synth.normal((T, H, 128), 0.1, T, "do")
+    dr = synth.normal((T, H, E), 0.1, T, "dy", torch.float32)
+    gain = pro["q_gain"] if use_gain else None
+    dx, dwq, dwr, dg = api.flash_mhffn_prologue_bwd(
+        pro["x"].cuda(), pro["w_q"].cuda(), pro["w_r"].cuda(), H, E, dq.cuda(), dr.cuda(),
+        q_gain=None if gain is None else gain.cuda())
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    ref = O.mhffn_prologue_backward(f64(pro["x"]), f64(pro["w_q"]), f64(pro["w_r"]), H, E, f64(dq), f64(dr),
+                                    None if gain is None else f64(gain), 1e-6)
+    assert_close("dx", f64(dx), ref["dx"], torch.bfloat16)
+    assert_close("dw_q", f64(dwq), ref["dw_q"], torch.bfloat16)
+    if E > 1:
+        assert_close("dw_r", f64(dwr), ref["dw_r"], torch.bfloat16)
+    else:
+        assert float(dwr.float().abs().max()) < 1e-5  # one sub-network: its weight is always 1
+    if use_gain:
+        assert_close("dq_gain", f64(dg), ref["dgain"], torch.float32)
