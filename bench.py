@@ -420,12 +420,31 @@ def secondary_mhffn(api, steps, warmup, world, peak):
         bwd()
     ms_bwd = timed(bwd, max(3, steps // 4), world)
     flops_bwd = 16.0 * T * H * dh * E * de
-    del ws
+    # the whole block's training step from x: prologue, fused core, core backward, prologue backward
+    ws_p = torch.empty(max(16, api.flash_mhffn_prologue_bwd_workspace_bytes(T, d_model, H, dh, E)),
+                       device=dev, dtype=torch.uint8)
+    q2, r2 = torch.empty_like(t["q"]), torch.empty_like(t["router"])
+    gx, gwq, gwr, ggain = (torch.empty_like(pro[k]) for k in ("x", "w_q", "w_r", "q_gain"))
+
+    def step():
+        api.flash_mhffn_prologue(pro["x"], pro["w_q"], pro["w_r"], H, E, q_gain=pro["q_gain"], q=q2, router=r2)
+        api.flash_mhffn_fwd(q2, t["w_k"], t["w_u"], t["w_v"], r2, o)
+        api.flash_mhffn_bwd(q2, t["w_k"], t["w_u"], t["w_v"], r2, dout, gq, gk, gu, gv, gr, ws)
+        api.flash_mhffn_prologue_bwd(pro["x"], pro["w_q"], pro["w_r"], H, E, gq, gr, q_gain=pro["q_gain"],
+                                     dx=gx, dw_q=gwq, dw_r=gwr, dq_gain=ggain, workspace=ws_p)
+    for _ in range(2):
+        step()
+    n_step = max(3, steps // 4)
+    ms_step = timed(step, n_step, world)
+    flops_step = flops_b + flops_bwd + 2 * 2.0 * T * d_model * (H * dh + H * E)
+    del ws, ws_p
     return {"workload": w["name"], "tflops": round(tf * world, 1), "pct_of_peak": round(100 * tf / peak, 2),
             "ms_per_step": round(ms / steps, 3), "steps": steps, "flops_per_step": flops,
             "intermediate_bytes_not_written": 2 * T * H * E * de,
             "backward": {"ms_per_step": round(ms_bwd / max(3, steps // 4), 3), "flops_per_step": flops_bwd,
                          "tflops": round(flops_bwd * max(3, steps // 4) / (ms_bwd / 1e3) / 1e12 * world, 1)},
+            "block_training_step_from_x": {"ms_per_step": round(ms_step / n_step, 3), "flops_per_step": flops_step,
+                                           "tflops": round(flops_step * n_step / (ms_step / 1e3) / 1e12 * world, 1)},
             "block_from_x": {"ms_per_step": round(ms_b / steps, 3),
                              "tflops": round(flops_b * steps / (ms_b / 1e3) / 1e12 * world, 1),
                              "flops_per_step": flops_b, "d_model": d_model}}

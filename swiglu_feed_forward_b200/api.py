@@ -189,6 +189,11 @@ def flash_mhffn_prologue(x, w_q, w_r, num_heads, num_sub, q_gain=None, eps=1e-6,
     return q, router
 
 
+def flash_mhffn_prologue_bwd_workspace_bytes(T, d_model, num_heads, head_dim, num_sub, dtype=torch.bfloat16):
+    return _lib.lib().flash_mhffn_prologue_bwd_workspace_bytes(T, d_model, num_heads, head_dim, num_sub,
+                                                               SWF_BF16 if dtype == torch.bfloat16 else SWF_F32)
+
+
 def flash_mhffn_prologue_bwd(x, w_q, w_r, num_heads, num_sub, dq, drouter, q_gain=None, eps=1e-6,
                              dx=None, dw_q=None, dw_r=None, dq_gain=None, workspace=None, stream=None):
     """Backward of flash_mhffn_prologue: returns (dx, dw_q, dw_r, dq_gain or None)."""
@@ -199,7 +204,7 @@ def flash_mhffn_prologue_bwd(x, w_q, w_r, num_heads, num_sub, dq, drouter, q_gai
     dw_r = torch.empty_like(w_r) if dw_r is None else dw_r
     if q_gain is not None and dq_gain is None:
         dq_gain = torch.empty_like(q_gain)
-    nb = _lib.lib().flash_mhffn_prologue_bwd_workspace_bytes(T, d, num_heads, dh, num_sub, _dt(x))
+    nb = flash_mhffn_prologue_bwd_workspace_bytes(T, d, num_heads, dh, num_sub, x.dtype)
     if workspace is None:
         workspace = torch.empty(max(16, nb), device=x.device, dtype=torch.uint8)
     _check("flash_mhffn_prologue_bwd", _lib.lib().flash_mhffn_prologue_bwd(

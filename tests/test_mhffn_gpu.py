@@ -167,3 +167,31 @@ def test_prologue_backward(T, d_model, H, E, use_gain):
         assert float(dwr.float().abs().max()) < 1e-5  # one sub-network: its weight is always 1
     if use_gain:
         assert_close("dq_gain", f64(dg), ref["dgain"], torch.float32)
+
+
+def test_block_training_step_end_to_end():
+    """x -> prologue -> fused core -> O, then dO back to dx and every weight gradient, against
+    the oracle's block (prologue and core chained)."""
+    T, d_model, H, E, de = 260, 256, 2, 3, 128
+    pro = synth.mhffn_prologue_inputs(T, d_model, H, 128, E, seed=41)
+    core = synth.mhffn_inputs(T, H, 128, E, de, seed=41)
+    g = {k: v.cuda() for k, v in pro.items()}
+    c = {k: v.cuda() for k, v in core.items()}
+    q, r = api.flash_mhffn_prologue(g["x"], g["w_q"], g["w_r"], H, E, q_gain=g["q_gain"])
+    o = api.flash_mhffn_fwd(q, c["w_k"], c["w_u"], c["w_v"], r)
+    dq, dk, du, dv, dr = api.flash_mhffn_bwd(q, c["w_k"], c["w_u"], c["w_v"], r, c["do"])
+    dx, dwq, dwr, dg = api.flash_mhffn_prologue_bwd(g["x"], g["w_q"], g["w_r"], H, E, dq, dr,
+                                                    q_gain=g["q_gain"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    x, wq, wr, gain = (f64(pro[k]) for k in ("x", "w_q", "w_r", "q_gain"))
+    wk, wu, wv, do = (f64(core[k]) for k in ("w_k", "w_u", "w_v", "do"))
+    pf = O.mhffn_prologue_forward(x, wq, wr, H, E, gain, 1e-6)
+    ref_o = O.mhffn_forward(pf["q"], wk, wu, wv, pf["r"])["o"]
+    cb = O.mhffn_backward(pf["q"], wk, wu, wv, pf["r"], do)
+    pb = O.mhffn_prologue_backward(x, wq, wr, H, E, cb["dq"], cb["dr"], gain, 1e-6)
+    assert_close("o", f64(o), ref_o, torch.bfloat16)
+    for name, got, ref in (("dk", dk, cb["dk"]), ("du", du, cb["du"]), ("dv", dv, cb["dv"]),
+                           ("dx", dx, pb["dx"]), ("dw_q", dwq, pb["dw_q"]), ("dw_r", dwr, pb["dw_r"]),
+                           ("dq_gain", dg, pb["dgain"])):
+        assert_close(name, f64(got), ref, torch.bfloat16)
