@@ -190,12 +190,15 @@ swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void* w_u, cons
                            void* stream);
 
 /* Backward of flash_mhffn_fwd: gradients of L = sum(d_o * o) with respect to q, w_k, w_u, w_v
- * and router (same shapes as those inputs; all overwritten, drouter fp32).  Runs per head as
- * tcgen05 GEMMs over per-head buffers in `workspace` (flash_mhffn_bwd_workspace_bytes bytes):
- *   dP = dO_h V_h^T;  [g | u] = Q_h [K_h ; U_h]^T with dS_g = dP r u SiLU'(g),
- *   dS_u = dP r SiLU(g), P = SiLU(g) u r and the router partials sum dP SiLU(g) u fused into its
- *   epilogue;  dQ_h = dS_g K_h + dS_u U_h;  [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h;  dV_h = P^T dO_h.
- * Unlike the forward it writes the head's [T, E * sub_dim] activations (bf16) to the workspace.
+ * and router (same shapes as those inputs; all overwritten, drouter fp32).  With dA = d_o_h V_e^T,
+ * act = SiLU(g) u (g = q_h K_e^T, u = q_h U_e^T) and r the sub-network's router weight:
+ *   drouter = sum over the sub-network's columns of dA act;  dS_g = dA r u SiLU'(g);
+ *   dS_u = dA r SiLU(g);  P = r act;  dq_h = sum_e dS_g K_e + dS_u U_e;
+ *   [dw_k ; dw_u]_e = [dS_g | dS_u]^T q_h;  dw_v_e = P^T d_o_h.
+ * One fused tcgen05 kernel per group of up to four heads recomputes g and u, forms dA on chip
+ * (never stored), accumulates dq and writes dS_g | dS_u and P (bf16) to `workspace`; split-K
+ * tcgen05 GEMMs then reduce them over the tokens into the weight gradients.  Workspace:
+ * flash_mhffn_bwd_workspace_bytes bytes (about 6 * min(num_heads, 4) * T * num_sub * sub_dim).
  * Device pointers, caller-owned, 16-byte aligned; asynchronous on `stream`; deterministic.
  * Supported: dtype SWF_BF16, head_dim 128, sub_dim a multiple of 128; else SWF_ERR_UNSUPPORTED.
  * Workspace missing or too small: SWF_ERR_WORKSPACE. */
@@ -381,11 +384,10 @@ typedef enum swf_kernel_kind {
   SWF_K_SPLITK_REDUCE = 25,/* fixed-order sum of split-K weight-gradient partials */
   SWF_K_MHFFN_FWD = 26,    /* FlashFFN multi-head FFN forward (fused, one kernel) */
   SWF_K_MHFFN_PROLOGUE = 27, /* FlashFFN prologue: head-normalised projection, router */
-  SWF_K_MHFFN_BWD_DP = 28, /* FlashFFN backward: dP = dO V^T */
-  SWF_K_MHFFN_BWD_DS = 29, /* FlashFFN backward: Q [K;U]^T with the gradient epilogue; dR sums */
-  SWF_K_MHFFN_BWD_DQ = 30, /* FlashFFN backward: dQ */
-  SWF_K_MHFFN_BWD_DW = 31, /* FlashFFN backward: dK, dU, dV */
-  SWF_K_NUM_KINDS = 32
+  SWF_K_MHFFN_BWD = 28,    /* FlashFFN backward, fused per token tile: dA, dS_g | dS_u, P, dQ */
+  SWF_K_MHFFN_BWD_DW = 29, /* FlashFFN backward: dK, dU, dV */
+  SWF_K_MHFFN_BWD_DR = 30, /* FlashFFN backward: router-gradient sums */
+  SWF_K_NUM_KINDS = 31
 } swf_kernel_kind;
 
 /* While enabled, every kernel the library launches is bracketed by a pair of CUDA events on

@@ -509,35 +509,452 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
   return launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, b, st);
 }
 
-// ------------------------------------------------------------------ backward (per head, composed)
-// The fused forward keeps the activations on chip; a fused backward would need the dK, dU, dV
-// accumulators (384 TMEM columns for 128 sub-network rows) next to the recomputed S and dP, which
-// leaves room only for products too small to outrun the one-thread MMA issue rate.  So the
-// backward runs per head as tcgen05 GEMMs over per-head buffers:
-//   dP  = dO_h V_h^T                                   [T, F]      (F = E * d_e)
-//   S   = Q_h [K_h ; U_h]^T with the epilogue  dS_g = dP r u SiLU'(g), dS_u = dP r SiLU(g),
-//         P = SiLU(g) u r, and the router gradient's per-128-column partials sum dP SiLU(g) u
-//   dQ_h = dS_g K_h + dS_u U_h ;  [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h ;  dV_h = P^T dO_h
-// and one small kernel sums each sub-network's partials into dR.
+// ------------------------------------------------------------------ backward (fused per token tile)
+// Gradients of L = sum(dO * O) for the block above ("Overview" formula, chain rule), per head:
+//   dA  = dO V_e^T                      (the gradient reaching R_e * act)
+//   dR_e = sum over the sub-network's d_e columns of dA * act,   act = SiLU(S_g) * S_u
+//   dS_g = R_e dA S_u SiLU'(S_g),  dS_u = R_e dA SiLU(S_g),  P = R_e act
+//   dQ  = sum_e dS_g K_e + dS_u U_e,  dK_e = dS_g^T Q,  dU_e = dS_u^T Q,  dV_e = P^T dO.
+// One kernel does everything that is local to a token tile: per work unit (head, 256 tokens on a
+// pair of CTAs) and per 64-column chunk c of the head's E*d_e columns it
+//   recomputes [S_g | S_u] = Q [K_c ; U_c]^T and dA = dO V_c^T   (tcgen05 pair, into one of two
+//     192-column TMEM buffers: S_g 64 | S_u 64 | dA 64),
+//   forms dS_g, dS_u, P and the router-gradient sums in the epilogue warps (dS_g, dS_u into
+//     shared memory in the operand layout; P straight to HBM),
+//   accumulates dQ += dS_g K_c + dS_u U_c in TMEM (128 columns) with dS from shared memory,
+//   and sends dS_g, dS_u to HBM by TMA stores from the same shared-memory tiles.
+// dA never leaves the chip; the [T, E*d_e] planes that reach HBM are dS_g | dS_u and P, the A
+// operands of the weight gradients (a reduction over all tokens, run after it as split-K GEMMs).
+//
+// Operand placement.  The S products split each weight chunk across the pair by rows (even CTA
+// K_c, odd CTA U_c, as in the forward); the dQ products split it by d_h columns (even CTA
+// K_c[:, :64] and U_c[:, :64], odd CTA the other halves), so the chunk is staged twice: a ring for
+// the S products and a ring for the dQ products, each 16 KB per CTA and stage.  V_c is split by
+// rows (32 per CTA) for dA.  Shared memory: Q and dO 64 KB, S ring 2 x 16, V ring 2 x 8, dQ ring
+// 3 x 16, two dS buffers of 32 KB = 224 KB.
+//
+// Threads (384 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 3 lane 0
+// the V ring; warp 2 lane 0 the dQ ring and, in the even CTA, issues the dQ products; warp 1 owns
+// TMEM and, in the even CTA, issues the S and dA products; warps 4..11 are two sets of four
+// epilogue warps taking alternate chunks (set s uses TMEM buffer s and dS buffer s), each thread
+// one token row, and at the end of a unit they drain dQ.  Every wait is bounded.
 namespace swf {
 namespace {
 
-__global__ void mh_dr_reduce_kernel(const float* __restrict__ part, int64_t n, int per,
-                                    float* __restrict__ dr) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    float s = 0.f;
-    for (int k = 0; k < per; ++k) s += part[i * per + k];  // fixed order
-    dr[i] = s;
+constexpr int kBwSuStages = 2;
+constexpr int kBwVStages = 2;
+constexpr int kBwDqStages = 3;
+constexpr int kBwVBox = 32 * 64 * 2;          // 32 V rows x 64 d_h (4 KB)
+constexpr int kBwVBytes = 2 * kBwVBox;        // this CTA's 32 rows of V_c
+constexpr int kBwDsBytes = 2 * kMhPBytes;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
+constexpr int kBwDoOff = kMhQBytes;
+constexpr int kBwSuOff = 2 * kMhQBytes;
+constexpr int kBwVOff = kBwSuOff + kBwSuStages * kMhKuBytes;
+constexpr int kBwDqOff = kBwVOff + kBwVStages * kBwVBytes;
+constexpr int kBwDsOff = kBwDqOff + kBwDqStages * kMhKuBytes;
+constexpr int kBwBarOff = kBwDsOff + 2 * kBwDsBytes;
+constexpr int kBwSmemBytes = kBwBarOff + 512 + 1024;
+static_assert(kBwSmemBytes <= 232448, "shared memory per CTA");
+constexpr int kBwBufCols = 192;               // S_g 64 | S_u 64 | dA 64 per TMEM buffer
+static_assert(kMhDh + 2 * kBwBufCols == kMhTmemCols, "TMEM: dQ + two buffers");
+
+struct MhBwArgs {
+  int T, H, E, de;
+  int h0;            // first head of this launch
+  int n_pt;          // pairs of 128-token tiles
+  int n_units;       // n_pt * heads of this launch, head-major
+  int nch;           // 64-column chunks per head (even: d_e is a multiple of 128)
+  int ch_per_sub;    // chunks per sub-network
+  int F;             // E * d_e
+  int tp;            // rows per head in the dS / P planes (n_pt * 256)
+  const float* r;    // [T][H][E]
+  __nv_bfloat16* p;  // [heads of this launch][tp][F]
+  __nv_bfloat16* dq; // [T][H * 128]
+  float* dr_part;    // [T][H][E][2]: the two epilogue sets' partial sums
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+__global__ void __launch_bounds__(kMhThreads, 1)
+    mhffn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmU,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDS,
+                     const MhBwArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBwBarOff);
+  uint64_t* q_full = bars + 0;                 // Q and dO of a unit
+  uint64_t* q_empty = bars + 1;
+  uint64_t* su_full = bars + 2;                // [kBwSuStages]
+  uint64_t* su_empty = su_full + kBwSuStages;  // [kBwSuStages]
+  uint64_t* v_full = su_empty + kBwSuStages;   // [kBwVStages]
+  uint64_t* v_empty = v_full + kBwVStages;     // [kBwVStages]
+  uint64_t* w_full = v_empty + kBwVStages;     // [kBwDqStages] dQ operand stages
+  uint64_t* w_empty = w_full + kBwDqStages;    // [kBwDqStages]
+  uint64_t* s_full = w_empty + kBwDqStages;    // [2] TMEM buffers
+  uint64_t* s_empty = s_full + 2;              // [2]
+  uint64_t* ds_full = s_empty + 2;             // [2] dS shared-memory buffers
+  uint64_t* ds_empty = ds_full + 2;            // [2]
+  uint64_t* dq_full = ds_empty + 2;
+  uint64_t* dq_empty = dq_full + 1;
+  uint64_t* drain = dq_empty + 1;              // [2]: one per issuing thread
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert((2 + 2 * kBwSuStages + 2 * kBwVStages + 2 * kBwDqStages + 8 + 4) * 8 + 8 <= 512,
+                "barrier block");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cl = static_cast<int>(blockIdx.x >> 1), n_cl = static_cast<int>(gridDim.x >> 1);
+  if (threadIdx.x == 0) {
+    // arrival counts are those of the even CTA's barriers, the only ones waited on with them
+    // (the dQ-ring and dS barriers are also waited on in the odd CTA: commit arrivals only)
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kBwSuStages; ++s) {
+      mbar_init(&su_full[s], 1);
+      mbar_init(&su_empty[s], 1);
+    }
+    for (int s = 0; s < kBwVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int s = 0; s < kBwDqStages; ++s) {
+      mbar_init(&w_full[s], 1);
+      mbar_init(&w_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 2 * 4);  // one arrival per warp of a set, in both CTAs
+      mbar_init(&ds_full[b], 2 * 4);
+      mbar_init(&ds_empty[b], 1);
+    }
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 2 * kMhEpiWarps);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(rank == 0 ? &tmK : &tmU);
+  }
+  if (warp == 3 && lane == 0) tma_prefetch_desc(&tmV);
+  if (warp == 4 && lane == 0) tma_prefetch_desc(&tmDS);
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kMhTmemCols);
+    tmem_relinquish_pair();
+  }
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, args.status, args.wait_limit_ns};
+  const int rows_per_head = args.F;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q, dO and S-ring producer
+    if (lane == 0) {
+      const uint32_t q_full_lead = map_to_rank(smem_u32(q_full), 0);
+      const uint32_t su_full_lead = map_to_rank(smem_u32(su_full), 0);
+      const CUtensorMap* tm_b = rank == 0 ? &tmK : &tmU;  // this CTA's half of [K_c; U_c]
+      uint32_t gc = 0;
+      int lu = 0;
+      bool ok = true;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+        const int hl = unit / args.n_pt, pt = unit - hl * args.n_pt;
+        const int h = args.h0 + hl;
+        const int tt = 2 * pt + static_cast<int>(rank);  // may lie past the last tile: zero rows
+        if (!mbar_wait(q_empty, (lu & 1) ^ 1u, ctl)) { ok = false; break; }
+        if (rank == 0) mbar_arrive_expect_tx(q_full, 4 * kMhQBytes);  // Q and dO of both CTAs
+        tma_load_2d_pair(smem, &tmQ, h * kMhDh, tt * kMhTile, q_full_lead);
+        tma_load_2d_pair(smem + kMhQBytes / 2, &tmQ, h * kMhDh + 64, tt * kMhTile, q_full_lead);
+        tma_load_2d_pair(smem + kBwDoOff, &tmDO, h * kMhDh, tt * kMhTile, q_full_lead);
+        tma_load_2d_pair(smem + kBwDoOff + kMhQBytes / 2, &tmDO, h * kMhDh + 64, tt * kMhTile,
+                         q_full_lead);
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const int row = h * rows_per_head + c * kMhChunk;
+          const int s = gc % kBwSuStages;
+          if (!mbar_wait(&su_empty[s], ((gc / kBwSuStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* su = smem + kBwSuOff + s * kMhKuBytes;
+          if (rank == 0) mbar_arrive_expect_tx(&su_full[s], 2 * kMhKuBytes);
+          tma_load_2d_pair(su, tm_b, 0, row, su_full_lead + s * 8);
+          tma_load_2d_pair(su + kMhBox, tm_b, 64, row, su_full_lead + s * 8);
+        }
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ V-ring producer
+    if (lane == 0) {
+      const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
+      uint32_t gc = 0;
+      bool ok = true;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl) {
+        const int h = args.h0 + unit / args.n_pt;
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const int row = h * rows_per_head + c * kMhChunk + static_cast<int>(rank) * 32;
+          const int sv = gc % kBwVStages;
+          if (!mbar_wait(&v_empty[sv], ((gc / kBwVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* vb = smem + kBwVOff + sv * kBwVBytes;
+          if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kBwVBytes);
+          tma_load_2d_pair(vb, &tmV, 0, row, v_full_lead + sv * 8);
+          tma_load_2d_pair(vb + kBwVBox, &tmV, 64, row, v_full_lead + sv * 8);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ S and dA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(2 * kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
+      constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);      // dA
+      const uint64_t q_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
+      const uint64_t su_desc = smem_desc_sw128(smem_u32(smem + kBwSuOff), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
+      uint32_t gc = 0;
+      int lu = 0;
+      bool ok = true, issued = false;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+        if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const uint32_t s = gc % kBwSuStages, sv = gc % kBwVStages, b = gc & 1u;
+          if (!mbar_wait(&su_full[s], (gc / kBwSuStages) & 1u, ctl)) { ok = false; break; }
+          if (!mbar_wait(&v_full[sv], (gc / kBwVStages) & 1u, ctl)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + kMhDh + b * kBwBufCols;
+          const uint64_t sd = desc_add(su_desc, s * kMhKuBytes);
+          const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_pair(d, desc_add(q_desc, kb * (kMhQBytes / 2) + k * 32),
+                             desc_add(sd, kb * kMhBox + k * 32), kIdescS, (kb | k) != 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_pair(d + 2 * kMhChunk, desc_add(do_desc, kb * (kMhQBytes / 2) + k * 32),
+                             desc_add(vd, kb * kBwVBox + k * 32), kIdescA, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&s_full[b], 3);
+          umma_commit_pair(&su_empty[s], 3);
+          umma_commit_pair(&v_empty[sv], 3);
+          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // Q, dO no longer read in this unit
+          issued = true;
+        }
+      }
+      if (!ok && issued) drain_mma(&drain[0], abort_flag, args.status);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ dQ ring and dQ issuer
+    // The loads run at most kBwDqStages - 1 chunks ahead of the products: a stage is free once
+    // the dQ products of the chunk that used it are done, and in the even CTA this same thread
+    // issued those products.
+    if (lane == 0) {
+      const uint32_t w_full_lead = map_to_rank(smem_u32(w_full), 0);
+      const int my_units = cl < args.n_units ? (args.n_units - cl + n_cl - 1) / n_cl : 0;
+      const uint32_t total = static_cast<uint32_t>(my_units) * static_cast<uint32_t>(args.nch);
+      uint32_t nl = 0;  // chunks whose dQ operands were requested
+      bool ok = true, issued = false;
+      auto load_next = [&]() -> bool {
+        const int unit = cl + static_cast<int>(nl / args.nch) * n_cl;
+        const int c = static_cast<int>(nl % args.nch);
+        const int row = (args.h0 + unit / args.n_pt) * rows_per_head + c * kMhChunk;
+        const uint32_t st = nl % kBwDqStages;
+        if (!mbar_wait(&w_empty[st], ((nl / kBwDqStages) & 1u) ^ 1u, ctl)) return false;
+        uint8_t* wb = smem + kBwDqOff + st * kMhKuBytes;
+        if (rank == 0) mbar_arrive_expect_tx(&w_full[st], 2 * kMhKuBytes);
+        tma_load_2d_pair(wb, &tmK, static_cast<int>(rank) * 64, row, w_full_lead + st * 8);
+        tma_load_2d_pair(wb + kMhBox, &tmU, static_cast<int>(rank) * 64, row, w_full_lead + st * 8);
+        ++nl;
+        return true;
+      };
+      if (rank != 0) {
+        while (ok && nl < total) ok = load_next();
+      } else {
+        constexpr uint32_t kIdescDQ = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
+        const uint64_t ds_desc = smem_desc_sw128(smem_u32(smem + kBwDsOff), 16, 1024);
+        const uint64_t w_desc = smem_desc_sw128(smem_u32(smem + kBwDqOff), kMhBox, 1024);
+        int lu = -1;
+        for (uint32_t i = 0; ok && i < total; ++i) {
+          while (ok && nl < total && nl < i + kBwDqStages) ok = load_next();
+          if (!ok) break;
+          const int c = static_cast<int>(i % args.nch);
+          if (c == 0) {
+            ++lu;
+            if (!mbar_wait(dq_empty, (lu & 1) ^ 1u, ctl)) { ok = false; break; }
+          }
+          const uint32_t b = i & 1u, st = i % kBwDqStages;
+          if (!mbar_wait(&ds_full[b], (i >> 1) & 1u, ctl)) { ok = false; break; }
+          if (!mbar_wait(&w_full[st], (i / kBwDqStages) & 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = desc_add(ds_desc, b * kBwDsBytes);
+          const uint64_t bd = desc_add(w_desc, st * kMhKuBytes);
+#pragma unroll
+          for (int seg = 0; seg < 2; ++seg) {  // dS_g with K_c, then dS_u with U_c
+#pragma unroll
+            for (int k = 0; k < kMhChunk / 16; ++k)
+              umma_bf16_pair(tmem_base, desc_add(ad, seg * kMhPBytes + k * 32),
+                             desc_add(bd, seg * kMhBox + k * 2048), kIdescDQ,
+                             (c | seg | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&ds_empty[b], 3);
+          umma_commit_pair(&w_empty[st], 3);
+          if (c == args.nch - 1) umma_commit_pair(dq_full, 3);
+          issued = true;
+        }
+        if (!ok && issued) drain_mma(&drain[1], abort_flag, args.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 4..11
+    const int q = warp & 3;           // TMEM lane quadrant this warp may access
+    const int set = (warp - 4) >> 2;  // chunks with (index & 1) == set; TMEM and dS buffer `set`
+    const int row = q * 32 + lane;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t tb = t_lane + kMhDh + set * kBwBufCols;
+    const uint32_t dsg = smem_u32(smem + kBwDsOff + set * kBwDsBytes);
+    const uint32_t dsu = dsg + kMhPBytes;
+    const int64_t q_ld = (int64_t)args.H * kMhDh;
+    uint32_t gc = 0;
+    int lu = 0;
+    bool ok = true;
+    for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+      const int hl = unit / args.n_pt, pt = unit - hl * args.n_pt;
+      const int h = args.h0 + hl;
+      const int tile_row0 = (2 * pt + static_cast<int>(rank)) * kMhTile;
+      const int token = tile_row0 + row;
+      const bool tok_ok = token < args.T;
+      const float* rrow = args.r + ((int64_t)(tok_ok ? token : 0) * args.H + h) * args.E;
+      __nv_bfloat16* prow = args.p + ((int64_t)hl * args.tp + token) * args.F;
+      float dr_acc = 0.f;
+      for (int c = 0; c < args.nch; ++c, ++gc) {
+        if ((int)(gc & 1u) != set) continue;
+        const int e = c / args.ch_per_sub;
+        const float rv = tok_ok ? rrow[e] : 0.f;
+        // dS buffer `set` is free once this warp's TMA stores have read it and the dQ products
+        // of the set's previous chunk are done
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        bool ready = mbar_wait(&ds_empty[set], ((gc >> 1) & 1u) ^ 1u, ctl);
+        ready = ready && mbar_wait(&s_full[set], (gc >> 1) & 1u, ctl);
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread waits
+        if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float g[32], u[32], a[32];
+          tmem_ld32(tb + half * 32, g);
+          tmem_ld32(tb + kMhChunk + half * 32, u);
+          tmem_ld32(tb + 2 * kMhChunk + half * 32, a);
+          tmem_ld_wait_regs(g);
+          pin_regs(u);
+          pin_regs(a);
+          if (half == 1) {
+            tc_fence_before();
+            warp_arrive_lead(&s_empty[set], rank, lane);  // the TMEM buffer is in registers
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t wg[4], wu[4], wp[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float vg[2], vu[2], vp[2];
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                const int k = c8 * 8 + 2 * j + t;
+                const float sg = sigmoidf_(g[k]);
+                const float silu = g[k] * sg;
+                const float act = silu * u[k];
+                const float dact = rv * a[k];
+                dr_acc = fmaf(a[k], act, dr_acc);
+                vp[t] = rv * act;
+                vu[t] = dact * silu;
+                vg[t] = dact * u[k] * fmaf(silu, 1.f - sg, sg);  // SiLU' = s + SiLU (1 - s)
+              }
+              wg[j] = pack_bf16x2(vg[0], vg[1]);
+              wu[j] = pack_bf16x2(vu[0], vu[1]);
+              wp[j] = pack_bf16x2(vp[0], vp[1]);
+            }
+            const int c16 = half * 4 + c8;
+            st_shared_v4(dsg + p_offset(row, c16), wg[0], wg[1], wg[2], wg[3]);
+            st_shared_v4(dsu + p_offset(row, c16), wu[0], wu[1], wu[2], wu[3]);
+            *reinterpret_cast<uint4*>(prow + c * kMhChunk + c16 * 8) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+          }
+        }
+        fence_proxy_async_smem();  // dS visible to the tensor core and to the TMA stores
+        __syncwarp();
+        if (lane == 0) {
+          const int prow0 = hl * args.tp + tile_row0 + q * 32;
+          tma_store_2d(&tmDS, c * kMhChunk, prow0, smem + kBwDsOff + set * kBwDsBytes + q * 4096);
+          tma_store_2d(&tmDS, args.F + c * kMhChunk, prow0,
+                       smem + kBwDsOff + set * kBwDsBytes + kMhPBytes + q * 4096);
+          bulk_commit();
+        }
+        warp_arrive_lead(&ds_full[set], rank, lane);
+        if (c + 2 >= (e + 1) * args.ch_per_sub) {  // the set's last chunk of sub-network e
+          if (tok_ok) args.dr_part[(((int64_t)token * args.H + h) * args.E + e) * 2 + set] = dr_acc;
+          dr_acc = 0.f;
+        }
+      }
+      if (!ok) break;
+      const bool ready = mbar_wait(dq_full, lu & 1, ctl);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
+      tc_fence_after();
+      __nv_bfloat16* dqrow = args.dq + (int64_t)(tok_ok ? token : 0) * q_ld + h * kMhDh;
+#pragma unroll 1
+      for (int cc = set * 64; cc < set * 64 + 64; cc += 32) {
+        float ov[32];
+        tmem_ld32(t_lane + cc, ov);
+        tmem_ld_wait_regs(ov);
+        if (tok_ok) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(dqrow + cc + 8 * v) =
+                make_uint4(pack_bf16x2(ov[8 * v], ov[8 * v + 1]), pack_bf16x2(ov[8 * v + 2], ov[8 * v + 3]),
+                           pack_bf16x2(ov[8 * v + 4], ov[8 * v + 5]), pack_bf16x2(ov[8 * v + 6], ov[8 * v + 7]));
+        }
+      }
+      tc_fence_before();
+      warp_arrive_lead(dq_empty, rank, lane);
+    }
+    if (lane == 0) bulk_wait_all();  // the TMA stores are done before the CTA leaves
+  }
+
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs and TMEM reads are all done
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kMhTmemCols);
   }
 }
 
+__global__ void mh_dr_reduce_kernel(const float* __restrict__ part, int64_t n, float* __restrict__ dr) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dr[i] = part[2 * i] + part[2 * i + 1];
+}
+
+constexpr int kMhBwdHeads = 4;  // heads per fused launch: sizes the dS / P planes of the workspace
+
 struct MhBwdWs {
-  __nv_bfloat16 *dp, *dsgu, *p;
+  __nv_bfloat16 *dsgu, *p;  // [hg][tp][2F], [hg][tp][F]
   float *dr_part, *split;
+  int64_t tp;
+  int hg;
 };
 
-MhBwdWs mh_bwd_ws(void* base, int64_t T, int64_t H, int64_t F, size_t* bytes) {
+MhBwdWs mh_bwd_ws(void* base, int64_t T, int64_t H, int64_t E, int64_t F, size_t* bytes) {
   size_t off = 0;
   auto take = [&](size_t n) {
     off = round_up(off, 256);
@@ -546,10 +963,12 @@ MhBwdWs mh_bwd_ws(void* base, int64_t T, int64_t H, int64_t F, size_t* bytes) {
     return p;
   };
   MhBwdWs w;
-  w.dp = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * F * 2));
-  w.dsgu = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * 2 * F * 2));
-  w.p = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * F * 2));
-  w.dr_part = reinterpret_cast<float*>(take((size_t)T * H * (F / 128) * 4));
+  const int64_t n_pt = ((T + kMhTile - 1) / kMhTile + 1) / 2;
+  w.tp = n_pt * 2 * kMhTile;
+  w.hg = static_cast<int>(std::min<int64_t>(H, kMhBwdHeads));
+  w.dsgu = reinterpret_cast<__nv_bfloat16*>(take((size_t)w.hg * w.tp * 2 * F * 2));
+  w.p = reinterpret_cast<__nv_bfloat16*>(take((size_t)w.hg * w.tp * F * 2));
+  w.dr_part = reinterpret_cast<float*>(take((size_t)T * H * E * 2 * 4));
   const int64_t part = std::max(part_elems(2 * F, kMhDh, T), part_elems(F, kMhDh, T));
   w.split = reinterpret_cast<float*>(take((size_t)std::max<int64_t>(part, 4) * 4));
   if (bytes) *bytes = off;
@@ -561,7 +980,7 @@ swf_status check_mh_bwd(int64_t T, int32_t H, int32_t dh, int32_t E, int32_t de,
   if (dt != SWF_BF16 && dt != SWF_F32) return SWF_ERR_INVALID_ARG;
   if (dt != SWF_BF16 || dh != kMhDh || de % 128 != 0) return SWF_ERR_UNSUPPORTED;
   if (T > INT32_MAX / 4 || (int64_t)E * de > (1 << 20) || (int64_t)H * E * de > INT32_MAX / 4 ||
-      (int64_t)H * kMhDh > (1 << 20))
+      (int64_t)H * kMhDh > (1 << 20) || (int64_t)kMhBwdHeads * (T + 2 * kMhTile) > INT32_MAX / 2)
     return SWF_ERR_UNSUPPORTED;
   return SWF_OK;
 }
@@ -573,7 +992,7 @@ extern "C" size_t flash_mhffn_bwd_workspace_bytes(int64_t T, int32_t num_heads, 
                                                   int32_t num_sub, int32_t sub_dim, swf_dtype dtype) {
   if (check_mh_bwd(T, num_heads, head_dim, num_sub, sub_dim, dtype) != SWF_OK) return 0;
   size_t need = 0;
-  mh_bwd_ws(nullptr, T, num_heads, (int64_t)num_sub * sub_dim, &need);
+  mh_bwd_ws(nullptr, T, num_heads, num_sub, (int64_t)num_sub * sub_dim, &need);
   return need;
 }
 
@@ -594,90 +1013,92 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
     if (p && !aligned16(p)) return SWF_ERR_ALIGNMENT;
   const int64_t H = num_heads, E = num_sub, de = sub_dim, F = E * de, ld = H * kMhDh;
   size_t need = 0;
-  const MhBwdWs w = mh_bwd_ws(workspace, T, H, F, &need);
+  const MhBwdWs w = mh_bwd_ws(workspace, T, H, E, F, &need);
   if (!workspace || workspace_bytes < need) return SWF_ERR_WORKSPACE;
+  DevCtx ctx;
+  if ((s = get_ctx(&ctx)) != SWF_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   using bf = __nv_bfloat16;
-  for (int64_t h = 0; h < H; ++h) {
-    const bf* qh = static_cast<const bf*>(q) + h * kMhDh;
-    const bf* doh = static_cast<const bf*>(d_o) + h * kMhDh;
-    const bf* kh = static_cast<const bf*>(w_k) + h * F * kMhDh;
-    const bf* uh = static_cast<const bf*>(w_u) + h * F * kMhDh;
-    const bf* vh = static_cast<const bf*>(w_v) + h * F * kMhDh;
-    {  // dP = dO_h V_h^T
-      CUtensorMap ta, tb;
-      if (!encode_tmap_bf16(&ta, doh, kMhDh, T, ld, 64, 128) ||
-          !encode_tmap_bf16(&tb, vh, kMhDh, F, kMhDh, 64, 128))
+  const int64_t rows = H * F;
+  CUtensorMap tq, tdo, tk, tu, tv;
+  if (!encode_tmap_bf16(&tq, q, ld, T, ld, 64, kMhTile) ||
+      !encode_tmap_bf16(&tdo, d_o, ld, T, ld, 64, kMhTile) ||
+      !encode_tmap_bf16(&tk, w_k, kMhDh, rows, kMhDh, 64, 64) ||
+      !encode_tmap_bf16(&tu, w_u, kMhDh, rows, kMhDh, 64, 64) ||
+      !encode_tmap_bf16(&tv, w_v, kMhDh, rows, kMhDh, 64, 32))
+    return SWF_ERR_LAUNCH;
+  if (cudaFuncSetAttribute(mhffn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kBwSmemBytes) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  MhBwArgs a{};
+  a.T = (int)T;
+  a.H = num_heads;
+  a.E = num_sub;
+  a.de = sub_dim;
+  a.n_pt = (int)(w.tp / (2 * kMhTile));
+  a.nch = (int)(F / kMhChunk);
+  a.ch_per_sub = (int)(de / kMhChunk);
+  a.F = (int)F;
+  a.tp = (int)w.tp;
+  a.r = router;
+  a.p = w.p;
+  a.dq = static_cast<bf*>(dq);
+  a.dr_part = w.dr_part;
+  a.status = ctx.status;
+  a.wait_limit_ns = kDefaultWaitNs;
+  for (int64_t h0 = 0; h0 < H; h0 += w.hg) {
+    const int g = (int)std::min<int64_t>(w.hg, H - h0);
+    {  // fused: dA, [S_g | S_u], dS_g | dS_u and P planes, router-gradient partials, dQ
+      CUtensorMap tds;  // dS_g | dS_u planes of this launch's heads, 32-row boxes of 64 columns
+      if (!encode_tmap_bf16(&tds, w.dsgu, 2 * F, (uint64_t)g * w.tp, 2 * F, 64, 32))
         return SWF_ERR_LAUNCH;
-      EpiMaps em{};  // dP leaves through the TMA epilogue's staging boxes
-      if (!encode_tmap_bf16(&em.o[0], w.dp, F, T, F, 32, 32, 64)) return SWF_ERR_LAUNCH;
-      em.o[1] = em.o[0];
-      TcGemmArgs a = base_args(T, F, 256, kMhDh, 2 * kTileM);
-      if ((s = launch_tc_pair<256, false, false, false, kEpiStore, true>(SWF_K_MHFFN_BWD_DP, ta, tb, tb, em,
-                                                                       a, st)) != SWF_OK)
-        return s;
+      a.h0 = (int)h0;
+      a.n_units = a.n_pt * g;
+      const int clusters = std::min(a.n_units, ctx.num_sms / 2);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * clusters, 1, 1);
+      cfg.blockDim = dim3(kMhThreads, 1, 1);
+      cfg.dynamicSmemBytes = kBwSmemBytes;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      ProfScope prof(SWF_K_MHFFN_BWD, st);
+      if (cudaLaunchKernelEx(&cfg, mhffn_bwd_kernel, tq, tdo, tk, tu, tv, tds, a) != cudaSuccess)
+        return SWF_ERR_LAUNCH;
     }
-    {  // [g | u] = Q_h [K_h ; U_h]^T -> dS_g | dS_u, P, router-gradient partials
-      CUtensorMap ta, tk, tu;
-      if (!encode_tmap_bf16(&ta, qh, kMhDh, T, ld, 64, 128) ||
-          !encode_tmap_bf16(&tk, kh, kMhDh, F, kMhDh, 64, 128) ||
-          !encode_tmap_bf16(&tu, uh, kMhDh, F, kMhDh, 64, 128))
-        return SWF_ERR_LAUNCH;
-      // TMA epilogue: dS_g, dS_u (two views of dSGU) and P leave through 32 x 32 staging boxes,
-      // dP comes in the same way
-      EpiMaps em{};
-      if (!encode_tmap_bf16(&em.o[0], w.dsgu, F, T, 2 * F, 32, 32, 64) ||
-          !encode_tmap_bf16(&em.o[1], w.dsgu + F, F, T, 2 * F, 32, 32, 64) ||
-          !encode_tmap_bf16(&em.o[2], w.p, F, T, F, 32, 32, 64) ||
-          !encode_tmap_bf16(&em.o[3], w.dp, F, T, F, 32, 32, 64))
-        return SWF_ERR_LAUNCH;
-      TcGemmArgs a = base_args(T, F, 128, kMhDh, 2 * kTileM);
-      a.rw = router + h * E;
-      a.ld_rw = H * E;
-      a.sub_dim = (int)de;
-      a.dr_part = w.dr_part + h * (F / 128);
-      a.ld_dr = H * (F / 128);
-      if ((s = launch_tc_pair<256, false, false, true, kEpiMhGrad, true>(SWF_K_MHFFN_BWD_DS, ta, tk, tu,
-                                                                       em, a, st)) != SWF_OK)
-        return s;
-    }
-    {  // dQ_h = dS_g K_h + dS_u U_h: A = [dS_g | dS_u] (K = 2F), B segments K_h, U_h (MN-major)
-      CUtensorMap ta, tk, tu;
-      if (!encode_tmap_bf16(&ta, w.dsgu, 2 * F, T, 2 * F, 64, 128) ||
-          !encode_tmap_bf16(&tk, kh, kMhDh, F, kMhDh, 64, 64) ||
-          !encode_tmap_bf16(&tu, uh, kMhDh, F, kMhDh, 64, 64))
-        return SWF_ERR_LAUNCH;
-      TcGemmArgs a = base_args(T, kMhDh, 128, 0, 2 * kTileM);
-      a.kb_seg0 = (int)(F / kTileK);
-      a.kb_total = 2 * a.kb_seg0;
-      a.a_koff1 = (int)F;
-      a.out0 = static_cast<bf*>(dq) + h * kMhDh;
-      a.ld_out = ld;
-      if ((s = launch_tc_pair<128, false, true, false, kEpiStore>(SWF_K_MHFFN_BWD_DQ, ta, tk, tu, EpiMaps{},
-                                                                a, st)) != SWF_OK)
-        return s;
-    }
-    {  // [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h
-      CUtensorMap ta, tb;
-      if (!encode_tmap_bf16(&ta, w.dsgu, 2 * F, T, 2 * F, 64, 64) ||
-          !encode_tmap_bf16(&tb, qh, kMhDh, T, ld, 64, 64))
-        return SWF_ERR_LAUNCH;
-      if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, 2 * F, kMhDh, T, static_cast<bf*>(dw_k) + h * F * kMhDh,
-                         static_cast<bf*>(dw_u) + h * F * kMhDh, F, w.split, st)) != SWF_OK)
-        return s;
-    }
-    {  // dV_h = P^T dO_h
-      CUtensorMap ta, tb;
-      if (!encode_tmap_bf16(&ta, w.p, F, T, F, 64, 64) || !encode_tmap_bf16(&tb, doh, kMhDh, T, ld, 64, 64))
-        return SWF_ERR_LAUNCH;
-      bf* dv = static_cast<bf*>(dw_v) + h * F * kMhDh;
-      if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, F, kMhDh, T, dv, dv, F, w.split, st)) != SWF_OK) return s;
+    for (int hl = 0; hl < g; ++hl) {
+      const int64_t h = h0 + hl;
+      const bf* qh = static_cast<const bf*>(q) + h * kMhDh;
+      const bf* doh = static_cast<const bf*>(d_o) + h * kMhDh;
+      const bf* dsgu_h = w.dsgu + (int64_t)hl * w.tp * 2 * F;
+      const bf* p_h = w.p + (int64_t)hl * w.tp * F;
+      {  // [dK_h ; dU_h] = [dS_g | dS_u]^T Q_h
+        CUtensorMap ta, tb;
+        if (!encode_tmap_bf16(&ta, dsgu_h, 2 * F, T, 2 * F, 64, 64) ||
+            !encode_tmap_bf16(&tb, qh, kMhDh, T, ld, 64, 64))
+          return SWF_ERR_LAUNCH;
+        if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, 2 * F, kMhDh, T, static_cast<bf*>(dw_k) + h * F * kMhDh,
+                           static_cast<bf*>(dw_u) + h * F * kMhDh, F, w.split, st)) != SWF_OK)
+          return s;
+      }
+      {  // dV_h = P^T dO_h
+        CUtensorMap ta, tb;
+        if (!encode_tmap_bf16(&ta, p_h, F, T, F, 64, 64) || !encode_tmap_bf16(&tb, doh, kMhDh, T, ld, 64, 64))
+          return SWF_ERR_LAUNCH;
+        bf* dv = static_cast<bf*>(dw_v) + h * F * kMhDh;
+        if ((s = launch_dw(SWF_K_MHFFN_BWD_DW, ta, tb, F, kMhDh, T, dv, dv, F, w.split, st)) != SWF_OK) return s;
+      }
     }
   }
-  ProfScope prof(SWF_K_MHFFN_BWD_DS, st);
+  ProfScope prof(SWF_K_MHFFN_BWD_DR, st);
   const int64_t n = T * H * E;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16));
-  mh_dr_reduce_kernel<<<grid, 256, 0, st>>>(w.dr_part, n, (int)(de / 128), drouter);
+  mh_dr_reduce_kernel<<<grid, 256, 0, st>>>(w.dr_part, n, drouter);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 

@@ -42,8 +42,8 @@ const char* const kNames[SWF_K_NUM_KINDS] = {
     "select_topk",     "buckets",              "sparse_gather", "sparse_up",     "sparse_down",
     "sparse_dgate",    "sparse_dx",            "sparse_dw",     "elementwise",   "pair_sum",
     "balance",         "mlp2_up",              "mlp2_dpre",     "mlp2_dx",       "mlp2_dw_up",
-    "splitk_reduce", "mhffn_fwd", "mhffn_prologue", "mhffn_bwd_dp", "mhffn_bwd_ds",
-    "mhffn_bwd_dq", "mhffn_bwd_dw"};
+    "splitk_reduce", "mhffn_fwd", "mhffn_prologue", "mhffn_bwd", "mhffn_bwd_dw",
+    "mhffn_bwd_dr"};
 
 }  // namespace
 

@@ -1,4 +1,4 @@
-"""GPU parity of the FlashFFN multi-head FFN forward (one fused kernel) against the fp64
+"""GPU parity of the FlashFFN multi-head FFN (fused forward, prologue, fused backward) against the fp64
 oracle, through the C ABI: small and ragged token counts, several heads and sub-network widths,
 and sampled token rows of the full 1.3B-configuration workload."""
 import numpy as np
@@ -121,6 +121,7 @@ def test_block_prologue_then_fused_forward():
     (1, 1, 1, 128),      # one token
     (300, 1, 2, 256),    # two 128-column blocks per sub-network
     (700, 3, 2, 384),    # the 1.3B sub-network width, odd head count
+    (4000, 5, 1, 128),   # two launches (four heads, then one), more units than clusters
 ])
 def test_backward(T, H, E, de):
     inp = synth.mhffn_inputs(T, H, 128, E, de, seed=T + 3 * E)
@@ -140,6 +141,30 @@ def test_backward_deterministic():
     a, b = api.flash_mhffn_bwd(*args), api.flash_mhffn_bwd(*args)
     for x, y in zip(a, b):
         assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+
+
+def test_backward_full_size_sampled():
+    """32768 tokens x 16 heads x 15 sub-networks of 384 (the bench's launch configuration):
+    dq and the router gradient on sampled tokens; dK, dU, dV on sampled rows of every kind of
+    sub-network (each such row sums over all 32768 tokens but needs only its own weight rows)."""
+    w = synth.WORKLOADS[6]
+    inp = synth.mhffn_inputs(w["T"], w["H"], w["d_h"], w["E"], w["d_e"], w["seed"])
+    t = {k: v.cuda() for k, v in inp.items()}
+    dq, dk, du, dv, dr = api.flash_mhffn_bwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], t["do"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    q, k, u, v, r, do = (f64(inp[n]) for n in ("q", "w_k", "w_u", "w_v", "router", "do"))
+    rng = np.random.default_rng(1)
+    tokens = np.sort(np.concatenate([rng.choice(w["T"] - 128, 16, replace=False), [w["T"] - 1]]))
+    ref = O.mhffn_backward(q[tokens], k, u, v, r[tokens], do[tokens])
+    assert_close("dq[tokens]", f64(dq)[tokens], ref["dq"], torch.bfloat16)
+    assert_close("dr[tokens]", f64(dr)[tokens], ref["dr"], torch.bfloat16)
+    for h, e in ((0, 0), (7, 14), (15, 6)):
+        rows = np.sort(rng.choice(w["d_e"], 6, replace=False))
+        sub = O.mhffn_backward(q[:, [h]], k[[h]][:, [e]][:, :, rows], u[[h]][:, [e]][:, :, rows],
+                               v[[h]][:, [e]][:, :, rows], r[:, [h]][:, :, [e]], do[:, [h]])
+        for name, got in (("dk", dk), ("du", du), ("dv", dv)):
+            assert_close(f"{name}[{h},{e},rows]", f64(got)[h, e][rows], sub[name][0, 0], torch.bfloat16)
 
 
 @pytest.mark.parametrize("T,d_model,H,E,use_gain", [
