@@ -520,9 +520,10 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
 //   recomputes [S_g | S_u] = Q [K_c ; U_c]^T and dA = dO V_c^T   (tcgen05 pair, into one of two
 //     192-column TMEM buffers: S_g 64 | S_u 64 | dA 64),
 //   forms dS_g, dS_u, P and the router-gradient sums in the epilogue warps (dS_g, dS_u into
-//     shared memory in the operand layout; P straight to HBM),
+//     shared memory in the operand layout, 64-byte swizzled K-major atoms; P into a staging tile),
 //   accumulates dQ += dS_g K_c + dS_u U_c in TMEM (128 columns) with dS from shared memory,
-//   and sends dS_g, dS_u to HBM by TMA stores from the same shared-memory tiles.
+//   and sends dS_g, dS_u and P to HBM by TMA stores from those shared-memory tiles (each warp its
+//     own 32 x 32 boxes; per-thread global stores of rows 11 KB apart were the bottleneck).
 // dA never leaves the chip; the [T, E*d_e] planes that reach HBM are dS_g | dS_u and P, the A
 // operands of the weight gradients (a reduction over all tokens, run after it as split-K GEMMs).
 //
@@ -531,31 +532,37 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
 // K_c[:, :64] and U_c[:, :64], odd CTA the other halves), so the chunk is staged twice: a ring for
 // the S products and a ring for the dQ products, each 16 KB per CTA and stage.  V_c is split by
 // rows (32 per CTA) for dA.  Shared memory: Q and dO 64 KB, S ring 2 x 16, V ring 2 x 8, dQ ring
-// 3 x 16, two dS buffers of 32 KB = 224 KB.
+// 2 x 16, two dS buffers of 32 KB, P staging 16 KB = 224 KB.
 //
 // Threads (384 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 3 lane 0
-// the V ring; warp 2 lane 0 the dQ ring and, in the even CTA, issues the dQ products; warp 1 owns
-// TMEM and, in the even CTA, issues the S and dA products; warps 4..11 are two sets of four
-// epilogue warps taking alternate chunks (set s uses TMEM buffer s and dS buffer s), each thread
-// one token row, and at the end of a unit they drain dQ.  Every wait is bounded.
+// the V ring and, in the even CTA, issues the dA products; warp 2 lane 0 the dQ ring and, in the
+// even CTA, issues the dQ products; warp 1 owns TMEM and, in the even CTA, issues the S products
+// (one issuing thread per product stream: a thread issues about one tcgen05.mma per 60-90
+// cycles); warps 4..11 form dS_g, dS_u, P for every chunk (warp (q, hc): token rows 32q..32q+31,
+// the chunk's columns 32hc..32hc+31; chunk c uses TMEM buffer c & 1 and dS buffer c & 1), and at
+// the end of a unit they drain dQ.  Every wait is bounded.
 namespace swf {
 namespace {
 
 constexpr int kBwSuStages = 2;
 constexpr int kBwVStages = 2;
-constexpr int kBwDqStages = 3;
+constexpr int kBwDqStages = 2;
 constexpr int kBwVBox = 32 * 64 * 2;          // 32 V rows x 64 d_h (4 KB)
 constexpr int kBwVBytes = 2 * kBwVBox;        // this CTA's 32 rows of V_c
-constexpr int kBwDsBytes = 2 * kMhPBytes;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
+constexpr int kBwDsAtom = 128 * 64;           // 128 rows x 32 bf16 (64-byte rows): one K atom
+constexpr int kBwDsBytes = 4 * kBwDsAtom;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
 constexpr int kBwDoOff = kMhQBytes;
 constexpr int kBwSuOff = 2 * kMhQBytes;
 constexpr int kBwVOff = kBwSuOff + kBwSuStages * kMhKuBytes;
 constexpr int kBwDqOff = kBwVOff + kBwVStages * kBwVBytes;
 constexpr int kBwDsOff = kBwDqOff + kBwDqStages * kMhKuBytes;
-constexpr int kBwBarOff = kBwDsOff + 2 * kBwDsBytes;
+constexpr int kBwPOff = kBwDsOff + 2 * kBwDsBytes;  // P staging: 2 atoms of 128 x 32 bf16
+constexpr int kBwBarOff = kBwPOff + 2 * kBwDsAtom;
 constexpr int kBwSmemBytes = kBwBarOff + 512 + 1024;
 static_assert(kBwSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kBwBufCols = 192;               // S_g 64 | S_u 64 | dA 64 per TMEM buffer
+__device__ constexpr float2 kHalf2 = {0.5f, 0.5f};
+__device__ constexpr float2 kMinusHalf2 = {-0.5f, -0.5f};
 static_assert(kMhDh + 2 * kBwBufCols == kMhTmemCols, "TMEM: dQ + two buffers");
 
 struct MhBwArgs {
@@ -568,9 +575,8 @@ struct MhBwArgs {
   int F;             // E * d_e
   int tp;            // rows per head in the dS / P planes (n_pt * 256)
   const float* r;    // [T][H][E]
-  __nv_bfloat16* p;  // [heads of this launch][tp][F]
   __nv_bfloat16* dq; // [T][H * 128]
-  float* dr_part;    // [T][H][E][2]: the two epilogue sets' partial sums
+  float* dr_part;    // [T][H][E][2]: partial sums of the two column halves
   int* status;
   uint64_t wait_limit_ns;
 };
@@ -579,7 +585,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     mhffn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDS,
-                     const MhBwArgs args) {
+                     const __grid_constant__ CUtensorMap tmP, const MhBwArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -598,10 +604,10 @@ __global__ void __launch_bounds__(kMhThreads, 1)
   uint64_t* ds_empty = ds_full + 2;            // [2]
   uint64_t* dq_full = ds_empty + 2;
   uint64_t* dq_empty = dq_full + 1;
-  uint64_t* drain = dq_empty + 1;              // [2]: one per issuing thread
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* drain = dq_empty + 1;              // [3]: one per issuing thread
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert((2 + 2 * kBwSuStages + 2 * kBwVStages + 2 * kBwDqStages + 8 + 4) * 8 + 8 <= 512,
+  static_assert((2 + 2 * kBwSuStages + 2 * kBwVStages + 2 * kBwDqStages + 8 + 5) * 8 + 8 <= 512,
                 "barrier block");
 
   const int warp = threadIdx.x >> 5;
@@ -612,7 +618,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     // arrival counts are those of the even CTA's barriers, the only ones waited on with them
     // (the dQ-ring and dS barriers are also waited on in the odd CTA: commit arrivals only)
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, 2);  // the S and the dA issuer each release Q / dO
     for (int s = 0; s < kBwSuStages; ++s) {
       mbar_init(&su_full[s], 1);
       mbar_init(&su_empty[s], 1);
@@ -626,15 +632,14 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       mbar_init(&w_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 2 * 4);  // one arrival per warp of a set, in both CTAs
-      mbar_init(&ds_full[b], 2 * 4);
+      mbar_init(&s_full[b], 2);                   // S products and dA products
+      mbar_init(&s_empty[b], 2 * kMhEpiWarps);    // one arrival per epilogue warp, both CTAs
+      mbar_init(&ds_full[b], 2 * kMhEpiWarps);
       mbar_init(&ds_empty[b], 1);
     }
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 2 * kMhEpiWarps);
-    mbar_init(&drain[0], 1);
-    mbar_init(&drain[1], 1);
+    for (int d = 0; d < 3; ++d) mbar_init(&drain[d], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -644,7 +649,10 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     tma_prefetch_desc(rank == 0 ? &tmK : &tmU);
   }
   if (warp == 3 && lane == 0) tma_prefetch_desc(&tmV);
-  if (warp == 4 && lane == 0) tma_prefetch_desc(&tmDS);
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmDS);
+    tma_prefetch_desc(&tmP);
+  }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kMhTmemCols);
     tmem_relinquish_pair();
@@ -688,33 +696,71 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       }
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------ V-ring producer
+    // ------------------------------------------------------------ V ring and dA issuer
+    // The loads run at most kBwVStages - 1 chunks ahead of the dA products (in the even CTA this
+    // thread issues the products that free the stages).
     if (lane == 0) {
       const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
-      uint32_t gc = 0;
-      bool ok = true;
-      for (int unit = cl; ok && unit < args.n_units; unit += n_cl) {
-        const int h = args.h0 + unit / args.n_pt;
-        for (int c = 0; c < args.nch; ++c, ++gc) {
-          const int row = h * rows_per_head + c * kMhChunk + static_cast<int>(rank) * 32;
-          const int sv = gc % kBwVStages;
-          if (!mbar_wait(&v_empty[sv], ((gc / kBwVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
-          uint8_t* vb = smem + kBwVOff + sv * kBwVBytes;
-          if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kBwVBytes);
-          tma_load_2d_pair(vb, &tmV, 0, row, v_full_lead + sv * 8);
-          tma_load_2d_pair(vb + kBwVBox, &tmV, 64, row, v_full_lead + sv * 8);
+      const int my_units = cl < args.n_units ? (args.n_units - cl + n_cl - 1) / n_cl : 0;
+      const uint32_t total = static_cast<uint32_t>(my_units) * static_cast<uint32_t>(args.nch);
+      uint32_t nl = 0;  // chunks whose V rows were requested
+      bool ok = true, issued = false;
+      auto load_next = [&]() -> bool {
+        const int unit = cl + static_cast<int>(nl / args.nch) * n_cl;
+        const int c = static_cast<int>(nl % args.nch);
+        const int row = (args.h0 + unit / args.n_pt) * rows_per_head + c * kMhChunk +
+                        static_cast<int>(rank) * 32;
+        const uint32_t sv = nl % kBwVStages;
+        if (!mbar_wait(&v_empty[sv], ((nl / kBwVStages) & 1u) ^ 1u, ctl)) return false;
+        uint8_t* vb = smem + kBwVOff + sv * kBwVBytes;
+        if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kBwVBytes);
+        tma_load_2d_pair(vb, &tmV, 0, row, v_full_lead + sv * 8);
+        tma_load_2d_pair(vb + kBwVBox, &tmV, 64, row, v_full_lead + sv * 8);
+        ++nl;
+        return true;
+      };
+      if (rank != 0) {
+        while (ok && nl < total) ok = load_next();
+      } else {
+        constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);
+        const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
+        const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
+        while (ok && nl < total && nl < static_cast<uint32_t>(kBwVStages)) ok = load_next();
+        int lu = -1;
+        for (uint32_t i = 0; ok && i < total; ++i) {
+          const int c = static_cast<int>(i % args.nch);
+          if (c == 0) {
+            ++lu;
+            if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
+          }
+          const uint32_t sv = i % kBwVStages, b = i & 1u;
+          if (!mbar_wait(&v_full[sv], (i / kBwVStages) & 1u, ctl)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[b], ((i >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + kMhDh + b * kBwBufCols + 2 * kMhChunk;
+          const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_pair(d, desc_add(do_desc, kb * (kMhQBytes / 2) + k * 32),
+                             desc_add(vd, kb * kBwVBox + k * 32), kIdescA, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&s_full[b], 3);
+          umma_commit_pair(&v_empty[sv], 3);
+          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // dO no longer read in this unit
+          issued = true;
+          while (ok && nl < total && nl < i + kBwVStages) ok = load_next();
         }
+        if (!ok && issued) drain_mma(&drain[2], abort_flag, args.status);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ S and dA issuer (even CTA)
+    // ------------------------------------------------------------ S issuer (even CTA)
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(2 * kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
-      constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);      // dA
       const uint64_t q_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
-      const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
       const uint64_t su_desc = smem_desc_sw128(smem_u32(smem + kBwSuOff), 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
       uint32_t gc = 0;
       int lu = 0;
       bool ok = true, issued = false;
@@ -722,14 +768,12 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         for (int c = 0; c < args.nch; ++c, ++gc) {
-          const uint32_t s = gc % kBwSuStages, sv = gc % kBwVStages, b = gc & 1u;
+          const uint32_t s = gc % kBwSuStages, b = gc & 1u;
           if (!mbar_wait(&su_full[s], (gc / kBwSuStages) & 1u, ctl)) { ok = false; break; }
-          if (!mbar_wait(&v_full[sv], (gc / kBwVStages) & 1u, ctl)) { ok = false; break; }
           if (!mbar_wait(&s_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem_base + kMhDh + b * kBwBufCols;
           const uint64_t sd = desc_add(su_desc, s * kMhKuBytes);
-          const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
@@ -737,17 +781,9 @@ __global__ void __launch_bounds__(kMhThreads, 1)
               umma_bf16_pair(d, desc_add(q_desc, kb * (kMhQBytes / 2) + k * 32),
                              desc_add(sd, kb * kMhBox + k * 32), kIdescS, (kb | k) != 0 ? 1u : 0u);
           }
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16_pair(d + 2 * kMhChunk, desc_add(do_desc, kb * (kMhQBytes / 2) + k * 32),
-                             desc_add(vd, kb * kBwVBox + k * 32), kIdescA, (kb | k) != 0 ? 1u : 0u);
-          }
           umma_commit_pair(&s_full[b], 3);
           umma_commit_pair(&su_empty[s], 3);
-          umma_commit_pair(&v_empty[sv], 3);
-          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // Q, dO no longer read in this unit
+          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // Q no longer read in this unit
           issued = true;
         }
       }
@@ -757,7 +793,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     // ------------------------------------------------------------ dQ ring and dQ issuer
     // The loads run at most kBwDqStages - 1 chunks ahead of the products: a stage is free once
     // the dQ products of the chunk that used it are done, and in the even CTA this same thread
-    // issued those products.
+    // issues those products (it refills a stage after issuing the next chunk's products).
     if (lane == 0) {
       const uint32_t w_full_lead = map_to_rank(smem_u32(w_full), 0);
       const int my_units = cl < args.n_units ? (args.n_units - cl + n_cl - 1) / n_cl : 0;
@@ -781,12 +817,11 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         while (ok && nl < total) ok = load_next();
       } else {
         constexpr uint32_t kIdescDQ = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
-        const uint64_t ds_desc = smem_desc_sw128(smem_u32(smem + kBwDsOff), 16, 1024);
+        const uint64_t ds_desc = smem_desc_sw64(smem_u32(smem + kBwDsOff), 512);
         const uint64_t w_desc = smem_desc_sw128(smem_u32(smem + kBwDqOff), kMhBox, 1024);
+        while (ok && nl < total && nl < static_cast<uint32_t>(kBwDqStages)) ok = load_next();
         int lu = -1;
         for (uint32_t i = 0; ok && i < total; ++i) {
-          while (ok && nl < total && nl < i + kBwDqStages) ok = load_next();
-          if (!ok) break;
           const int c = static_cast<int>(i % args.nch);
           if (c == 0) {
             ++lu;
@@ -801,8 +836,9 @@ __global__ void __launch_bounds__(kMhThreads, 1)
 #pragma unroll
           for (int seg = 0; seg < 2; ++seg) {  // dS_g with K_c, then dS_u with U_c
 #pragma unroll
-            for (int k = 0; k < kMhChunk / 16; ++k)
-              umma_bf16_pair(tmem_base, desc_add(ad, seg * kMhPBytes + k * 32),
+            for (int k = 0; k < kMhChunk / 16; ++k)  // two K16 steps per 64-byte atom
+              umma_bf16_pair(tmem_base,
+                             desc_add(ad, seg * 2 * kBwDsAtom + (k >> 1) * kBwDsAtom + (k & 1) * 32),
                              desc_add(bd, seg * kMhBox + k * 2048), kIdescDQ,
                              (c | seg | k) != 0 ? 1u : 0u);
           }
@@ -810,19 +846,26 @@ __global__ void __launch_bounds__(kMhThreads, 1)
           umma_commit_pair(&w_empty[st], 3);
           if (c == args.nch - 1) umma_commit_pair(dq_full, 3);
           issued = true;
+          // refill after issuing: the stage of chunk i + kBwDqStages - 1 waits only for the
+          // products of chunk i - 1, issued a chunk ago
+          while (ok && nl < total && nl < i + kBwDqStages) ok = load_next();
         }
         if (!ok && issued) drain_mma(&drain[1], abort_flag, args.status);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue warps 4..11
+    // Every chunk goes through all eight warps: warp (q, hc) takes TMEM lane quadrant q and the
+    // chunk's columns [32 hc, 32 hc + 32), so each thread loads its 96 values (g, u, dA) with one
+    // round of tcgen05 loads and frees the TMEM buffer at once.  dS tiles are stored K-major in
+    // 64-byte swizzled atoms of 32 columns (atom hc belongs to the warps of column half hc), so each
+    // warp sends its own 32 x 32 boxes to HBM.
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
-    const int set = (warp - 4) >> 2;  // chunks with (index & 1) == set; TMEM and dS buffer `set`
+    const int hc = (warp - 4) >> 2;   // column half of every chunk
     const int row = q * 32 + lane;
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this thread's row
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t tb = t_lane + kMhDh + set * kBwBufCols;
-    const uint32_t dsg = smem_u32(smem + kBwDsOff + set * kBwDsBytes);
-    const uint32_t dsu = dsg + kMhPBytes;
+    const uint32_t ds_row = smem_u32(smem + kBwDsOff) + hc * kBwDsAtom + row * 64;
     const int64_t q_ld = (int64_t)args.H * kMhDh;
     uint32_t gc = 0;
     int lu = 0;
@@ -834,75 +877,87 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       const int token = tile_row0 + row;
       const bool tok_ok = token < args.T;
       const float* rrow = args.r + ((int64_t)(tok_ok ? token : 0) * args.H + h) * args.E;
-      __nv_bfloat16* prow = args.p + ((int64_t)hl * args.tp + token) * args.F;
-      float dr_acc = 0.f;
+      float2 dr2 = make_float2(0.f, 0.f);     // router-gradient sum (even | odd columns)
+      float rv_next = tok_ok ? rrow[0] : 0.f;  // router weight of the next chunk (loaded ahead)
       for (int c = 0; c < args.nch; ++c, ++gc) {
-        if ((int)(gc & 1u) != set) continue;
+        const uint32_t b = gc & 1u;
         const int e = c / args.ch_per_sub;
-        const float rv = tok_ok ? rrow[e] : 0.f;
-        // dS buffer `set` is free once this warp's TMA stores have read it and the dQ products
-        // of the set's previous chunk are done
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-        bool ready = mbar_wait(&ds_empty[set], ((gc >> 1) & 1u) ^ 1u, ctl);
-        ready = ready && mbar_wait(&s_full[set], (gc >> 1) & 1u, ctl);
-        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread waits
+        const float2 rv2 = make_float2(rv_next, rv_next);
+        if (c + 1 < args.nch) rv_next = tok_ok ? rrow[(c + 1) / args.ch_per_sub] : 0.f;
+        const bool ready = mbar_wait(&s_full[b], (gc >> 1) & 1u, ctl);
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
         if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float g[32], u[32], a[32];
-          tmem_ld32(tb + half * 32, g);
-          tmem_ld32(tb + kMhChunk + half * 32, u);
-          tmem_ld32(tb + 2 * kMhChunk + half * 32, a);
-          tmem_ld_wait_regs(g);
-          pin_regs(u);
-          pin_regs(a);
-          if (half == 1) {
-            tc_fence_before();
-            warp_arrive_lead(&s_empty[set], rank, lane);  // the TMEM buffer is in registers
+        const uint32_t tb = t_lane + kMhDh + b * kBwBufCols + hc * 32;
+        float g[32], u[32], a[32];
+        tmem_ld32(tb, g);
+        tmem_ld32(tb + kMhChunk, u);
+        tmem_ld32(tb + 2 * kMhChunk, a);
+        tmem_ld_wait_regs(g);
+        pin_regs(u);
+        pin_regs(a);
+        tc_fence_before();
+        warp_arrive_lead(&s_empty[b], rank, lane);  // the TMEM buffer is in registers
+        // dS buffer b is free once this warp's TMA stores from it (two chunks ago) have read it
+        // and the dQ products of that chunk are done; the P staging once the previous chunk's
+        // stores have read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        const bool free_ds = mbar_wait(&ds_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl);
+        if (!__all_sync(0xffffffffu, free_ds)) { ok = false; break; }
+        const uint32_t dsg = ds_row + b * kBwDsBytes;
+        const uint32_t dsu = dsg + 2 * kBwDsAtom;
+        const uint32_t pst = ds_row + (kBwPOff - kBwDsOff);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t wg[4], wu[4], wp[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // two columns at a time with Blackwell's paired fp32 operations (fma/mul .f32x2,
+            // IEEE round-to-nearest like the scalar forms); sigmoid(g) = (1 + tanh(g / 2)) / 2 is
+            // one MUFU operation (tanh.approx.f32, relative error about 2^-11), and every result
+            // is rounded to bf16 (2^-9) after
+            const int k = c4 * 8 + 2 * j;
+            const float2 g2 = make_float2(g[k], g[k + 1]);
+            const float2 u2 = make_float2(u[k], u[k + 1]);
+            const float2 a2 = make_float2(a[k], a[k + 1]);
+            const float2 h2 = __fmul2_rn(g2, kHalf2);
+            float2 th;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(h2.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(h2.y));
+            const float2 sg = __ffma2_rn(th, kHalf2, kHalf2);           // sigmoid
+            const float2 silu = __ffma2_rn(h2, th, h2);                  // g sigmoid(g)
+            const float2 dsilu = __ffma2_rn(silu, __ffma2_rn(th, kMinusHalf2, kHalf2), sg);  // s + SiLU (1 - s)
+            const float2 act = __fmul2_rn(silu, u2);
+            const float2 dact = __fmul2_rn(rv2, a2);
+            dr2 = __ffma2_rn(a2, act, dr2);
+            const float2 vp = __fmul2_rn(rv2, act);
+            const float2 vu = __fmul2_rn(dact, silu);
+            const float2 vg = __fmul2_rn(__fmul2_rn(dact, u2), dsilu);
+            wg[j] = pack_bf16x2(vg.x, vg.y);
+            wu[j] = pack_bf16x2(vu.x, vu.y);
+            wp[j] = pack_bf16x2(vp.x, vp.y);
           }
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t wg[4], wu[4], wp[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float vg[2], vu[2], vp[2];
-#pragma unroll
-              for (int t = 0; t < 2; ++t) {
-                const int k = c8 * 8 + 2 * j + t;
-                const float sg = sigmoidf_(g[k]);
-                const float silu = g[k] * sg;
-                const float act = silu * u[k];
-                const float dact = rv * a[k];
-                dr_acc = fmaf(a[k], act, dr_acc);
-                vp[t] = rv * act;
-                vu[t] = dact * silu;
-                vg[t] = dact * u[k] * fmaf(silu, 1.f - sg, sg);  // SiLU' = s + SiLU (1 - s)
-              }
-              wg[j] = pack_bf16x2(vg[0], vg[1]);
-              wu[j] = pack_bf16x2(vu[0], vu[1]);
-              wp[j] = pack_bf16x2(vp[0], vp[1]);
-            }
-            const int c16 = half * 4 + c8;
-            st_shared_v4(dsg + p_offset(row, c16), wg[0], wg[1], wg[2], wg[3]);
-            st_shared_v4(dsu + p_offset(row, c16), wu[0], wu[1], wu[2], wu[3]);
-            *reinterpret_cast<uint4*>(prow + c * kMhChunk + c16 * 8) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
-          }
+          const uint32_t off = static_cast<uint32_t>((c4 ^ swz) << 4);
+          st_shared_v4(dsg + off, wg[0], wg[1], wg[2], wg[3]);
+          st_shared_v4(dsu + off, wu[0], wu[1], wu[2], wu[3]);
+          st_shared_v4(pst + off, wp[0], wp[1], wp[2], wp[3]);
         }
-        fence_proxy_async_smem();  // dS visible to the tensor core and to the TMA stores
+        fence_proxy_async_smem();  // dS and P visible to the tensor core and to the TMA stores
         __syncwarp();
         if (lane == 0) {
           const int prow0 = hl * args.tp + tile_row0 + q * 32;
-          tma_store_2d(&tmDS, c * kMhChunk, prow0, smem + kBwDsOff + set * kBwDsBytes + q * 4096);
-          tma_store_2d(&tmDS, args.F + c * kMhChunk, prow0,
-                       smem + kBwDsOff + set * kBwDsBytes + kMhPBytes + q * 4096);
+          uint8_t* box = smem + kBwDsOff + b * kBwDsBytes + hc * kBwDsAtom + q * 32 * 64;
+          tma_store_2d(&tmDS, c * kMhChunk + hc * 32, prow0, box);
+          tma_store_2d(&tmDS, args.F + c * kMhChunk + hc * 32, prow0, box + 2 * kBwDsAtom);
+          tma_store_2d(&tmP, c * kMhChunk + hc * 32, prow0,
+                       smem + kBwPOff + hc * kBwDsAtom + q * 32 * 64);
           bulk_commit();
         }
-        warp_arrive_lead(&ds_full[set], rank, lane);
-        if (c + 2 >= (e + 1) * args.ch_per_sub) {  // the set's last chunk of sub-network e
-          if (tok_ok) args.dr_part[(((int64_t)token * args.H + h) * args.E + e) * 2 + set] = dr_acc;
-          dr_acc = 0.f;
+        warp_arrive_lead(&ds_full[b], rank, lane);
+        if (c == (e + 1) * args.ch_per_sub - 1) {  // last chunk of sub-network e
+          if (tok_ok) args.dr_part[(((int64_t)token * args.H + h) * args.E + e) * 2 + hc] = dr2.x + dr2.y;
+          dr2 = make_float2(0.f, 0.f);
         }
       }
       if (!ok) break;
@@ -912,7 +967,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       tc_fence_after();
       __nv_bfloat16* dqrow = args.dq + (int64_t)(tok_ok ? token : 0) * q_ld + h * kMhDh;
 #pragma unroll 1
-      for (int cc = set * 64; cc < set * 64 + 64; cc += 32) {
+      for (int cc = hc * 64; cc < hc * 64 + 64; cc += 32) {
         float ov[32];
         tmem_ld32(t_lane + cc, ov);
         tmem_ld_wait_regs(ov);
@@ -1041,7 +1096,6 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
   a.F = (int)F;
   a.tp = (int)w.tp;
   a.r = router;
-  a.p = w.p;
   a.dq = static_cast<bf*>(dq);
   a.dr_part = w.dr_part;
   a.status = ctx.status;
@@ -1049,8 +1103,9 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
   for (int64_t h0 = 0; h0 < H; h0 += w.hg) {
     const int g = (int)std::min<int64_t>(w.hg, H - h0);
     {  // fused: dA, [S_g | S_u], dS_g | dS_u and P planes, router-gradient partials, dQ
-      CUtensorMap tds;  // dS_g | dS_u planes of this launch's heads, 32-row boxes of 64 columns
-      if (!encode_tmap_bf16(&tds, w.dsgu, 2 * F, (uint64_t)g * w.tp, 2 * F, 64, 32))
+      CUtensorMap tds, tp;  // dS_g | dS_u and P planes of this launch's heads, 32 x 32 boxes
+      if (!encode_tmap_bf16(&tds, w.dsgu, 2 * F, (uint64_t)g * w.tp, 2 * F, 32, 32, 64) ||
+          !encode_tmap_bf16(&tp, w.p, F, (uint64_t)g * w.tp, F, 32, 32, 64))
         return SWF_ERR_LAUNCH;
       a.h0 = (int)h0;
       a.n_units = a.n_pt * g;
@@ -1068,7 +1123,7 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       ProfScope prof(SWF_K_MHFFN_BWD, st);
-      if (cudaLaunchKernelEx(&cfg, mhffn_bwd_kernel, tq, tdo, tk, tu, tv, tds, a) != cudaSuccess)
+      if (cudaLaunchKernelEx(&cfg, mhffn_bwd_kernel, tq, tdo, tk, tu, tv, tds, tp, a) != cudaSuccess)
         return SWF_ERR_LAUNCH;
     }
     for (int hl = 0; hl < g; ++hl) {

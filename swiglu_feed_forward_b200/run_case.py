@@ -5,7 +5,7 @@ python -m swiglu_feed_forward_b200.run_case --op sparse_step --M 16384 --d 1024 
     --G 64 --K 8 --spg 8
 
 Ops: fwd, fwd_infer, bwd (fwd once, then timed bwd), step (fwd + bwd), select, sparse_step
-(select + sparse fwd + sparse bwd).  Each rep is timed with CUDA events; the per-kernel split
+(select + sparse fwd + sparse bwd), mhffn_fwd, mhffn_bwd (FlashFFN block core, --T --H --E --de).  Each rep is timed with CUDA events; the per-kernel split
 comes from the library's profiling hooks.  Also a convenient target for ncu (-k regex:...)."""
 from __future__ import annotations
 
@@ -21,7 +21,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", default="step",
                     choices=["fwd", "fwd_infer", "bwd", "step", "select", "sparse_step", "mlp2_step",
-                             "mhffn_fwd"])
+                             "mhffn_fwd", "mhffn_bwd"])
     ap.add_argument("--M", type=int, default=32768)
     ap.add_argument("--d", type=int, default=2048)
     ap.add_argument("--f", type=int, default=5504)
@@ -37,7 +37,7 @@ def main():
     ap.add_argument("--reps", type=int, default=5)
     a = ap.parse_args()
     dev = torch.device("cuda")
-    if a.op == "mhffn_fwd":
+    if a.op in ("mhffn_fwd", "mhffn_bwd"):
         return run_mhffn(a, dev)
     M, d, f, G, K = a.M, a.d, a.f, a.G, a.K
     inp = synth.dense_inputs(M, d, f, a.seed, torch.bfloat16)
@@ -118,14 +118,23 @@ def timed_reps(fn, a):
 
 
 def run_mhffn(a, dev):
-    inp = synth.mhffn_inputs(a.T, a.H, 128, a.E, a.de, a.seed, with_do=False)
+    bwd = a.op == "mhffn_bwd"
+    inp = synth.mhffn_inputs(a.T, a.H, 128, a.E, a.de, a.seed, with_do=bwd)
     t = {k: v.to(dev) for k, v in inp.items()}
-    o = torch.empty_like(t["q"])
-    ms, kern = timed_reps(lambda: api.flash_mhffn_fwd(t["q"], t["w_k"], t["w_u"], t["w_v"],
-                                                      t["router"], o), a)
-    flops = 6.0 * a.T * a.H * 128 * a.E * a.de
+    if bwd:
+        ws = torch.empty(max(16, api.flash_mhffn_bwd_workspace_bytes(a.T, a.H, 128, a.E, a.de)),
+                         device=dev, dtype=torch.uint8)
+        outs = [torch.empty_like(t[k]) for k in ("q", "w_k", "w_u", "w_v", "router")]
+        fn = lambda: api.flash_mhffn_bwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], t["do"],
+                                         *outs, workspace=ws)
+        flops = 16.0 * a.T * a.H * 128 * a.E * a.de
+    else:
+        o = torch.empty_like(t["q"])
+        fn = lambda: api.flash_mhffn_fwd(t["q"], t["w_k"], t["w_u"], t["w_v"], t["router"], o)
+        flops = 6.0 * a.T * a.H * 128 * a.E * a.de
+    ms, kern = timed_reps(fn, a)
     status = api.device_status()
-    print(json.dumps({"op": "mhffn_fwd", "T": a.T, "H": a.H, "E": a.E, "de": a.de,
+    print(json.dumps({"op": a.op, "T": a.T, "H": a.H, "E": a.E, "de": a.de,
                       "ms_per_rep": round(ms, 4), "tflops": round(flops / (ms / 1e3) / 1e12, 1),
                       "status": status,
                       "kernels": {k: {"launches": n, "avg_ms": round(v / n, 4)} for k, (n, v) in kern.items()}}))
