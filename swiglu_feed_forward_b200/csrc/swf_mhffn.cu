@@ -88,6 +88,20 @@ __device__ __forceinline__ float silu_tanh(float z) {
   return fmaf(hz, t, hz);
 }
 
+__device__ constexpr float2 kHalf2 = {0.5f, 0.5f};
+__device__ constexpr float2 kMinusHalf2 = {-0.5f, -0.5f};
+
+// SiLU(g) * u * r for two columns with Blackwell's paired fp32 operations (mul/fma .f32x2, IEEE
+// round-to-nearest like the scalar forms, so the result equals silu_tanh(g) * u * r), as bf16x2.
+__device__ __forceinline__ uint32_t silu_mul_pair(float ga, float gb, float ua, float ub, float2 r2) {
+  const float2 h2 = __fmul2_rn(make_float2(ga, gb), kHalf2);
+  float2 th;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(h2.x));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(h2.y));
+  const float2 v = __fmul2_rn(__fmul2_rn(__ffma2_rn(h2, th, h2), make_float2(ua, ub)), r2);
+  return pack_bf16x2(v.x, v.y);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -104,6 +118,21 @@ __device__ __forceinline__ void warp_arrive_lead(uint64_t* bar, uint32_t rank, i
     if (rank == 0) mbar_arrive(bar);
     else mbar_arrive_remote(map_to_rank(smem_u32(bar), 0));
   }
+}
+
+// UMMA shared-memory descriptor (sm_100 format) of a K-major operand in the 64-byte-swizzle
+// layout: rows of 64 bytes (32 bf16 of K), 16-byte chunk c of row r at chunk position
+// c ^ ((r >> 1) & 3), 8-row groups `sbo_bytes` apart (layout type 4 at bits 61..63; the leading
+// byte offset is not used by swizzled K-major layouts).  Tiles are 512-byte aligned so the
+// swizzle phase is that of the address.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
 }
 
 // UMMA shared-memory descriptor moved by `bytes` (a multiple of 16): the start address is the
@@ -347,12 +376,11 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         pin_regs(u1);
         tc_fence_before();
         warp_arrive_lead(&s_empty[sb], rank, lane);  // the S buffer is in registers
+        const float2 rv2 = make_float2(rv, rv);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          w[j] = pack_bf16x2(silu_tanh(g0[2 * j]) * u0[2 * j] * rv,
-                             silu_tanh(g0[2 * j + 1]) * u0[2 * j + 1] * rv);
-          w[16 + j] = pack_bf16x2(silu_tanh(g1[2 * j]) * u1[2 * j] * rv,
-                                  silu_tanh(g1[2 * j + 1]) * u1[2 * j + 1] * rv);
+          w[j] = silu_mul_pair(g0[2 * j], g0[2 * j + 1], u0[2 * j], u0[2 * j + 1], rv2);
+          w[16 + j] = silu_mul_pair(g1[2 * j], g1[2 * j + 1], u1[2 * j], u1[2 * j + 1], rv2);
         }
         const bool p_free = mbar_wait(&p_empty[pb], ((gc / kMhPBufs) & 1u) ^ 1u, ctl);
         if (!__all_sync(0xffffffffu, p_free)) { ok = false; break; }  // warp-uniform exit
@@ -561,8 +589,6 @@ constexpr int kBwBarOff = kBwPOff + 2 * kBwDsAtom;
 constexpr int kBwSmemBytes = kBwBarOff + 512 + 1024;
 static_assert(kBwSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kBwBufCols = 192;               // S_g 64 | S_u 64 | dA 64 per TMEM buffer
-__device__ constexpr float2 kHalf2 = {0.5f, 0.5f};
-__device__ constexpr float2 kMinusHalf2 = {-0.5f, -0.5f};
 static_assert(kMhDh + 2 * kBwBufCols == kMhTmemCols, "TMEM: dQ + two buffers");
 
 struct MhBwArgs {

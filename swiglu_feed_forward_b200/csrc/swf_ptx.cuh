@@ -345,20 +345,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// The same for a K-major operand in the 64-byte-swizzle layout: rows of 64 bytes (32 bf16 of K),
-// 16-byte chunk c of row r at chunk position c ^ ((r >> 1) & 3), 8-row groups `sbo_bytes` apart
-// (layout type 4 at bits 61..63; the leading byte offset is not used by swizzled K-major layouts).
-// Tiles are 512-byte aligned so the swizzle phase is that of the address.
-__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;
-  d |= 4ull << 61;
-  return d;
-}
-
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
