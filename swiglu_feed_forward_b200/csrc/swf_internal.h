@@ -19,9 +19,9 @@ struct DevCtx {
 // Current device's context (SM count, status word address); cached per device.
 swf_status get_ctx(DevCtx* out);
 
-// 2-D bf16 tensor map with 128-byte (or 64-byte) swizzle over a row-major matrix of `rows` x `cols`
-// elements whose rows are `row_elems` apart; box of box_cols x box_rows.  Out-of-range
-// elements of a box read as zero.
+// 2-D bf16 tensor map with 128-byte (or 64- or 32-byte) swizzle over a row-major matrix of
+// `rows` x `cols` elements whose rows are `row_elems` apart; box of box_cols x box_rows.
+// Out-of-range elements of a box read as zero.
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                       uint64_t row_elems, uint32_t box_cols, uint32_t box_rows,
                       int swizzle_bytes = 128);

@@ -135,6 +135,39 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_
   return d;
 }
 
+// The same for the 32-byte-swizzle layout: rows of 32 bytes (16 bf16 of K, one K16 step), 16-byte
+// chunk c of row r at chunk position c ^ ((r >> 2) & 1), 8-row groups `sbo_bytes` apart (layout
+// type 6).  Tiles are 256-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 6ull << 61;
+  return d;
+}
+
+// 32 lanes x 16 consecutive fp32 columns (thread i gets lane taddr.lane + i), and the wait that
+// ties three such loads' registers to it.
+__device__ __forceinline__ void tmem_ld16x(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait16x3(float (&x)[16], float (&y)[16], float (&z)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) asm volatile("" : "+f"(x[j]), "+f"(y[j]), "+f"(z[j])::"memory");
+}
+
 // UMMA shared-memory descriptor moved by `bytes` (a multiple of 16): the start address is the
 // low 14-bit field in 16-byte units, which stays below 2^14 for any address in the 227 KB.
 __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
@@ -577,15 +610,18 @@ constexpr int kBwVStages = 2;
 constexpr int kBwDqStages = 2;
 constexpr int kBwVBox = 32 * 64 * 2;          // 32 V rows x 64 d_h (4 KB)
 constexpr int kBwVBytes = 2 * kBwVBox;        // this CTA's 32 rows of V_c
-constexpr int kBwDsAtom = 128 * 64;           // 128 rows x 32 bf16 (64-byte rows): one K atom
-constexpr int kBwDsBytes = 4 * kBwDsAtom;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
+constexpr int kBwEpiWarps = 16;              // four per TMEM lane quadrant, 16 columns each
+constexpr int kBwThreads = 128 + 32 * kBwEpiWarps;
+constexpr int kBwCols = kMhChunk / 4;         // columns of a chunk per epilogue warp
+constexpr int kBwDsAtom = 128 * kBwCols * 2;  // 128 rows x 16 bf16 (32-byte rows): one K16 atom
+constexpr int kBwDsBytes = 8 * kBwDsAtom;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
 constexpr int kBwDoOff = kMhQBytes;
 constexpr int kBwSuOff = 2 * kMhQBytes;
 constexpr int kBwVOff = kBwSuOff + kBwSuStages * kMhKuBytes;
 constexpr int kBwDqOff = kBwVOff + kBwVStages * kBwVBytes;
 constexpr int kBwDsOff = kBwDqOff + kBwDqStages * kMhKuBytes;
-constexpr int kBwPOff = kBwDsOff + 2 * kBwDsBytes;  // P staging: 2 atoms of 128 x 32 bf16
-constexpr int kBwBarOff = kBwPOff + 2 * kBwDsAtom;
+constexpr int kBwPOff = kBwDsOff + 2 * kBwDsBytes;  // P staging: 4 atoms of 128 x 16 bf16
+constexpr int kBwBarOff = kBwPOff + 4 * kBwDsAtom;
 constexpr int kBwSmemBytes = kBwBarOff + 512 + 1024;
 static_assert(kBwSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kBwBufCols = 192;               // S_g 64 | S_u 64 | dA 64 per TMEM buffer
@@ -602,12 +638,12 @@ struct MhBwArgs {
   int tp;            // rows per head in the dS / P planes (n_pt * 256)
   const float* r;    // [T][H][E]
   __nv_bfloat16* dq; // [T][H * 128]
-  float* dr_part;    // [T][H][E][2]: partial sums of the two column halves
+  float* dr_part;    // [T][H][E][4]: partial sums of the four column quarters
   int* status;
   uint64_t wait_limit_ns;
 };
 
-__global__ void __launch_bounds__(kMhThreads, 1)
+__global__ void __launch_bounds__(kBwThreads, 1)
     mhffn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDS,
@@ -659,12 +695,12 @@ __global__ void __launch_bounds__(kMhThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 2);                   // S products and dA products
-      mbar_init(&s_empty[b], 2 * kMhEpiWarps);    // one arrival per epilogue warp, both CTAs
-      mbar_init(&ds_full[b], 2 * kMhEpiWarps);
+      mbar_init(&s_empty[b], 2 * kBwEpiWarps);    // one arrival per epilogue warp, both CTAs
+      mbar_init(&ds_full[b], 2 * kBwEpiWarps);
       mbar_init(&ds_empty[b], 1);
     }
     mbar_init(dq_full, 1);
-    mbar_init(dq_empty, 2 * kMhEpiWarps);
+    mbar_init(dq_empty, 2 * kBwEpiWarps);
     for (int d = 0; d < 3; ++d) mbar_init(&drain[d], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -843,7 +879,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         while (ok && nl < total) ok = load_next();
       } else {
         constexpr uint32_t kIdescDQ = idesc_bf16(2 * kMhTile, kMhDh, 0, 1);
-        const uint64_t ds_desc = smem_desc_sw64(smem_u32(smem + kBwDsOff), 512);
+        const uint64_t ds_desc = smem_desc_sw32(smem_u32(smem + kBwDsOff), 256);
         const uint64_t w_desc = smem_desc_sw128(smem_u32(smem + kBwDqOff), kMhBox, 1024);
         while (ok && nl < total && nl < static_cast<uint32_t>(kBwDqStages)) ok = load_next();
         int lu = -1;
@@ -862,9 +898,8 @@ __global__ void __launch_bounds__(kMhThreads, 1)
 #pragma unroll
           for (int seg = 0; seg < 2; ++seg) {  // dS_g with K_c, then dS_u with U_c
 #pragma unroll
-            for (int k = 0; k < kMhChunk / 16; ++k)  // two K16 steps per 64-byte atom
-              umma_bf16_pair(tmem_base,
-                             desc_add(ad, seg * 2 * kBwDsAtom + (k >> 1) * kBwDsAtom + (k & 1) * 32),
+            for (int k = 0; k < kMhChunk / 16; ++k)  // one K16 step per 32-byte atom
+              umma_bf16_pair(tmem_base, desc_add(ad, seg * 4 * kBwDsAtom + k * kBwDsAtom),
                              desc_add(bd, seg * kMhBox + k * 2048), kIdescDQ,
                              (c | seg | k) != 0 ? 1u : 0u);
           }
@@ -880,18 +915,19 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue warps 4..11
-    // Every chunk goes through all eight warps: warp (q, hc) takes TMEM lane quadrant q and the
-    // chunk's columns [32 hc, 32 hc + 32), so each thread loads its 96 values (g, u, dA) with one
-    // round of tcgen05 loads and frees the TMEM buffer at once.  dS tiles are stored K-major in
-    // 64-byte swizzled atoms of 32 columns (atom hc belongs to the warps of column half hc), so each
-    // warp sends its own 32 x 32 boxes to HBM.
+    // ------------------------------------------------------------ epilogue warps 4..19
+    // Every chunk goes through all sixteen warps: warp (q, qc) takes TMEM lane quadrant q and the
+    // chunk's columns [16 qc, 16 qc + 16), so each thread loads its 48 values (g, u, dA) with one
+    // round of tcgen05 loads and frees the TMEM buffer at once, and four warps per SM sub-partition
+    // hide each other's latencies.  dS and P tiles are stored K-major in 32-byte swizzled atoms of
+    // 16 columns (atom qc belongs to the warps of column quarter qc), so each warp sends its own
+    // 32-row boxes to HBM.
     const int q = warp & 3;           // TMEM lane quadrant this warp may access
-    const int hc = (warp - 4) >> 2;   // column half of every chunk
+    const int qc = (warp - 4) >> 2;   // column quarter of every chunk
     const int row = q * 32 + lane;
-    const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this thread's row
+    const int swz = (lane >> 2) & 1;  // 32-byte swizzle phase of this thread's row
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t ds_row = smem_u32(smem + kBwDsOff) + hc * kBwDsAtom + row * 64;
+    const uint32_t ds_row = smem_u32(smem + kBwDsOff) + qc * kBwDsAtom + row * (2 * kBwCols);
     const int64_t q_ld = (int64_t)args.H * kMhDh;
     uint32_t gc = 0;
     int lu = 0;
@@ -914,14 +950,12 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the per-thread wait
         if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tb = t_lane + kMhDh + b * kBwBufCols + hc * 32;
-        float g[32], u[32], a[32];
-        tmem_ld32(tb, g);
-        tmem_ld32(tb + kMhChunk, u);
-        tmem_ld32(tb + 2 * kMhChunk, a);
-        tmem_ld_wait_regs(g);
-        pin_regs(u);
-        pin_regs(a);
+        const uint32_t tb = t_lane + kMhDh + b * kBwBufCols + qc * kBwCols;
+        float g[16], u[16], a[16];
+        tmem_ld16x(tb, g);
+        tmem_ld16x(tb + kMhChunk, u);
+        tmem_ld16x(tb + 2 * kMhChunk, a);
+        tmem_wait16x3(g, u, a);
         tc_fence_before();
         warp_arrive_lead(&s_empty[b], rank, lane);  // the TMEM buffer is in registers
         // dS buffer b is free once this warp's TMA stores from it (two chunks ago) have read it
@@ -932,10 +966,10 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         const bool free_ds = mbar_wait(&ds_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl);
         if (!__all_sync(0xffffffffu, free_ds)) { ok = false; break; }
         const uint32_t dsg = ds_row + b * kBwDsBytes;
-        const uint32_t dsu = dsg + 2 * kBwDsAtom;
+        const uint32_t dsu = dsg + 4 * kBwDsAtom;
         const uint32_t pst = ds_row + (kBwPOff - kBwDsOff);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c8 = 0; c8 < 2; ++c8) {
           uint32_t wg[4], wu[4], wp[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -943,7 +977,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
             // IEEE round-to-nearest like the scalar forms); sigmoid(g) = (1 + tanh(g / 2)) / 2 is
             // one MUFU operation (tanh.approx.f32, relative error about 2^-11), and every result
             // is rounded to bf16 (2^-9) after
-            const int k = c4 * 8 + 2 * j;
+            const int k = c8 * 8 + 2 * j;
             const float2 g2 = make_float2(g[k], g[k + 1]);
             const float2 u2 = make_float2(u[k], u[k + 1]);
             const float2 a2 = make_float2(a[k], a[k + 1]);
@@ -964,7 +998,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
             wu[j] = pack_bf16x2(vu.x, vu.y);
             wp[j] = pack_bf16x2(vp.x, vp.y);
           }
-          const uint32_t off = static_cast<uint32_t>((c4 ^ swz) << 4);
+          const uint32_t off = static_cast<uint32_t>((c8 ^ swz) << 4);
           st_shared_v4(dsg + off, wg[0], wg[1], wg[2], wg[3]);
           st_shared_v4(dsu + off, wu[0], wu[1], wu[2], wu[3]);
           st_shared_v4(pst + off, wp[0], wp[1], wp[2], wp[3]);
@@ -973,16 +1007,16 @@ __global__ void __launch_bounds__(kMhThreads, 1)
         __syncwarp();
         if (lane == 0) {
           const int prow0 = hl * args.tp + tile_row0 + q * 32;
-          uint8_t* box = smem + kBwDsOff + b * kBwDsBytes + hc * kBwDsAtom + q * 32 * 64;
-          tma_store_2d(&tmDS, c * kMhChunk + hc * 32, prow0, box);
-          tma_store_2d(&tmDS, args.F + c * kMhChunk + hc * 32, prow0, box + 2 * kBwDsAtom);
-          tma_store_2d(&tmP, c * kMhChunk + hc * 32, prow0,
-                       smem + kBwPOff + hc * kBwDsAtom + q * 32 * 64);
+          const int col = c * kMhChunk + qc * kBwCols;
+          uint8_t* box = smem + kBwDsOff + b * kBwDsBytes + qc * kBwDsAtom + q * 32 * (2 * kBwCols);
+          tma_store_2d(&tmDS, col, prow0, box);
+          tma_store_2d(&tmDS, args.F + col, prow0, box + 4 * kBwDsAtom);
+          tma_store_2d(&tmP, col, prow0, smem + kBwPOff + qc * kBwDsAtom + q * 32 * (2 * kBwCols));
           bulk_commit();
         }
         warp_arrive_lead(&ds_full[b], rank, lane);
         if (c == (e + 1) * args.ch_per_sub - 1) {  // last chunk of sub-network e
-          if (tok_ok) args.dr_part[(((int64_t)token * args.H + h) * args.E + e) * 2 + hc] = dr2.x + dr2.y;
+          if (tok_ok) args.dr_part[(((int64_t)token * args.H + h) * args.E + e) * 4 + qc] = dr2.x + dr2.y;
           dr2 = make_float2(0.f, 0.f);
         }
       }
@@ -993,7 +1027,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
       tc_fence_after();
       __nv_bfloat16* dqrow = args.dq + (int64_t)(tok_ok ? token : 0) * q_ld + h * kMhDh;
 #pragma unroll 1
-      for (int cc = hc * 64; cc < hc * 64 + 64; cc += 32) {
+      for (int cc = qc * 32; cc < qc * 32 + 32; cc += 32) {
         float ov[32];
         tmem_ld32(t_lane + cc, ov);
         tmem_ld_wait_regs(ov);
@@ -1023,7 +1057,7 @@ __global__ void __launch_bounds__(kMhThreads, 1)
 __global__ void mh_dr_reduce_kernel(const float* __restrict__ part, int64_t n, float* __restrict__ dr) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
-    dr[i] = part[2 * i] + part[2 * i + 1];
+    dr[i] = (part[4 * i] + part[4 * i + 1]) + (part[4 * i + 2] + part[4 * i + 3]);  // fixed order
 }
 
 constexpr int kMhBwdHeads = 4;  // heads per fused launch: sizes the dS / P planes of the workspace
@@ -1049,7 +1083,7 @@ MhBwdWs mh_bwd_ws(void* base, int64_t T, int64_t H, int64_t E, int64_t F, size_t
   w.hg = static_cast<int>(std::min<int64_t>(H, kMhBwdHeads));
   w.dsgu = reinterpret_cast<__nv_bfloat16*>(take((size_t)w.hg * w.tp * 2 * F * 2));
   w.p = reinterpret_cast<__nv_bfloat16*>(take((size_t)w.hg * w.tp * F * 2));
-  w.dr_part = reinterpret_cast<float*>(take((size_t)T * H * E * 2 * 4));
+  w.dr_part = reinterpret_cast<float*>(take((size_t)T * H * E * 4 * 4));
   const int64_t part = std::max(part_elems(2 * F, kMhDh, T), part_elems(F, kMhDh, T));
   w.split = reinterpret_cast<float*>(take((size_t)std::max<int64_t>(part, 4) * 4));
   if (bytes) *bytes = off;
@@ -1129,16 +1163,16 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
   for (int64_t h0 = 0; h0 < H; h0 += w.hg) {
     const int g = (int)std::min<int64_t>(w.hg, H - h0);
     {  // fused: dA, [S_g | S_u], dS_g | dS_u and P planes, router-gradient partials, dQ
-      CUtensorMap tds, tp;  // dS_g | dS_u and P planes of this launch's heads, 32 x 32 boxes
-      if (!encode_tmap_bf16(&tds, w.dsgu, 2 * F, (uint64_t)g * w.tp, 2 * F, 32, 32, 64) ||
-          !encode_tmap_bf16(&tp, w.p, F, (uint64_t)g * w.tp, F, 32, 32, 64))
+      CUtensorMap tds, tp;  // dS_g | dS_u and P planes of this launch's heads, 16 x 32 boxes
+      if (!encode_tmap_bf16(&tds, w.dsgu, 2 * F, (uint64_t)g * w.tp, 2 * F, kBwCols, 32, 32) ||
+          !encode_tmap_bf16(&tp, w.p, F, (uint64_t)g * w.tp, F, kBwCols, 32, 32))
         return SWF_ERR_LAUNCH;
       a.h0 = (int)h0;
       a.n_units = a.n_pt * g;
       const int clusters = std::min(a.n_units, ctx.num_sms / 2);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * clusters, 1, 1);
-      cfg.blockDim = dim3(kMhThreads, 1, 1);
+      cfg.blockDim = dim3(kBwThreads, 1, 1);
       cfg.dynamicSmemBytes = kBwSmemBytes;
       cfg.stream = st;
       cudaLaunchAttribute attr[1];
