@@ -38,10 +38,6 @@
 //                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
 //   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
 //                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
-//   kEpiMhGrad     (TMA epilogue only) dual [g | u] tile of a FlashFFN head with dP (TMA-loaded)
-//                  and the router weight r of the tile's sub-network: outputs dS_g = dP r u
-//                  SiLU'(g), dS_u = dP r SiLU(g), P = SiLU(g) u r, and per tile the router
-//                  gradient's partial sum_n dP SiLU(g) u -> dr_part[m][nb]
 //   kEpiHeadNormBwd C = z (the projection), heads of 128 columns, with dq (aux0, ld_aux) and the
 //                  gain (bias, nullable): dz = inv (dn - n mean(dn n)), n = z inv, dn = dq gain,
 //                  inv = 1 / sqrt(mean(z^2) + eps) -> bf16 out0; if dgain_part, per 32-row slab
@@ -78,7 +74,6 @@ enum : int {
   kEpiEnergyTopK = 10,
   kEpiHeadNorm = 11,
   kEpiRouter = 12,
-  kEpiMhGrad = 13,
   kEpiHeadNormBwd = 14,
   kEpiRouterBwd = 15
 };
@@ -120,11 +115,8 @@ struct TcGemmArgs {
   int64_t ld_grp;         // kEpiEnergy*: stride of out0 between groups (0: 1); ld_out is the
                           //   stride between tokens (1 with ld_grp = M: group-major energies)
   float eps;              // kEpiHeadNorm
-  const float* rw;        // kEpiMhGrad: router weights of the head, rw[m * ld_rw + e]
+  const float* rw;        // kEpiRouterBwd: dR, rw[m * ld_rw + n]
   int64_t ld_rw;
-  int sub_dim;            //   columns per sub-network (a multiple of the tile's BN / 2)
-  float* dr_part;         //   [M][ld_dr] partial router gradients, one per tile column block
-  int64_t ld_dr;
   float* dgain_part;      // kEpiHeadNormBwd (nullable): [M / 32 * heads][128] gain-gradient partials
   int heads;
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
@@ -143,16 +135,13 @@ struct TcGemmArgs {
 // loaded by TMA into the same kind of buffers.
 template <int EPI>
 constexpr int tma_epi_outputs() {
-  return (EPI == kEpiSwiGLU || EPI == kEpiMhGrad) ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
+  return EPI == kEpiSwiGLU ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
 }
 template <int EPI>
 constexpr int tma_epi_aux() {
-  return EPI == kEpiDGate ? 2 : ((EPI == kEpiScale || EPI == kEpiMhGrad) ? 1 : 0);
+  return EPI == kEpiDGate ? 2 : (EPI == kEpiScale ? 1 : 0);
 }
-template <int EPI>
-constexpr int aux_map0() {
-  return EPI == kEpiMhGrad ? 3 : 2;
-}
+constexpr int kEpiAuxMap = 2;  // first tensor map of the factors a TMA epilogue loads
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <int EPI, bool TMA_EPI>
 constexpr int epi_smem_bytes() {
@@ -161,7 +150,7 @@ constexpr int epi_smem_bytes() {
 }
 
 // Tensor maps of a TMA epilogue: outputs in o[0..], then the factors it loads by TMA from
-// o[aux_map0<EPI>()] on (kEpiDGate's a/b in o[2], o[3]; kEpiScale's in o[2]; kEpiMhGrad's dP in o[3]).
+// o[kEpiAuxMap] on (kEpiDGate's a/b in o[2], o[3]; kEpiScale's in o[2]).
 struct EpiMaps {
   CUtensorMap o[4];
 };
@@ -357,8 +346,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
                                                     EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
-                                                    EPI == kEpiScale || EPI == kEpiLeakySq ||
-                                                    EPI == kEpiMhGrad)) ||
+                                                    EPI == kEpiScale || EPI == kEpiLeakySq)) ||
                     (MODE == kModeRowGrouped && EPI == kEpiStore),
                 "TMA epilogue: dense bf16 outputs, or row-grouped plain stores");
 
@@ -535,7 +523,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int NOUT = tma_epi_outputs<EPI>();
     constexpr int NAUX = tma_epi_aux<EPI>();
     constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
-    constexpr bool kDual = kGLU || EPI == kEpiMhGrad;  // [g | u] accumulator halves
+    constexpr bool kDual = kGLU;  // [g | u] accumulator halves
     constexpr int NCH = (kDual ? BN / 2 : BN) / 32;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
@@ -561,7 +549,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) {
             const int db = aux_issued & 1;
             mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
-            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[aux_map0<EPI>()], n_base + c * 32, m_slab,
+            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[kEpiAuxMap], n_base + c * 32, m_slab,
                         &abar[db]);
             if constexpr (NAUX > 1)
               tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
@@ -579,10 +567,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * BN;
       const bool have_acc = t.kb > 0;
-      float mh_r = 0.f, mh_dr = 0.f;  // kEpiMhGrad: the row's router weight, gradient partial
-      if constexpr (EPI == kEpiMhGrad) {
-        if (m_slab + lane < args.M) mh_r = args.rw[(int64_t)(m_slab + lane) * args.ld_rw + n_base / args.sub_dim];
-      }
 #pragma unroll 1
       for (int c = 0; c < NCH; ++c) {
         const uint8_t* aux = nullptr;
@@ -654,32 +638,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               w[0][c4 * 4 + p] = pack_bf16x2(v0[c4 * 8 + p * 2] * bf16_lo(aw[p]),
                                              v0[c4 * 8 + p * 2 + 1] * bf16_hi(aw[p]));
           }
-        } else if constexpr (EPI == kEpiMhGrad) {
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 dv = *reinterpret_cast<const uint4*>(aux + lane * 64 + ((c4 ^ swz) * 16));
-            const uint32_t dw[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              float sg[2], su[2], pv[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int j = c4 * 8 + p * 2 + e;
-                const float g = v0[j], u = v1[j];
-                const float dp = e ? bf16_hi(dw[p]) : bf16_lo(dw[p]);
-                const float sgm = sigmoidf_(g);
-                const float a = g * sgm;
-                mh_dr = fmaf(dp, a * u, mh_dr);
-                const float dpr = dp * mh_r;
-                sg[e] = dpr * u * sgm * (1.f + g * (1.f - sgm));
-                su[e] = dpr * a;
-                pv[e] = a * u * mh_r;
-              }
-              w[0][c4 * 4 + p] = pack_bf16x2(sg[0], sg[1]);
-              w[1][c4 * 4 + p] = pack_bf16x2(su[0], su[1]);
-              w[2][c4 * 4 + p] = pack_bf16x2(pv[0], pv[1]);
-            }
-          }
         } else if constexpr (EPI == kEpiDGate) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
@@ -727,10 +685,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ++chunks;
       }
       if (!ok) break;
-      if constexpr (EPI == kEpiMhGrad) {
-        if (m_slab + lane < args.M && n_base < args.N)
-          args.dr_part[(int64_t)(m_slab + lane) * args.ld_dr + t.nb] = mh_dr;
-      }
       tc_fence_before();
       if (PAIR && rank != 0) mbar_arrive_remote(tempty_lead + buf * 8);  // TMEM read: own SM
       else mbar_arrive(&tempty[buf]);
