@@ -525,6 +525,70 @@ extern "C" swf_status flash_mhffn_fwd(const void* q, const void* w_k, const void
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 
+namespace swf {
+namespace {
+
+// Router rows of the block's prologue ("Overview": sigmoid-normalised router weights).  The
+// router GEMM leaves s = sigmoid(logits) in each token's row of N = H * E values; one warp per
+// token stages the row in shared memory, one lane per head sums its E values in index order, and
+// the row goes back out with coalesced accesses.
+constexpr int kRouterRows = 8;  // tokens (warps) per block
+
+//   R = s / sum_e s, in place
+__global__ void router_norm_kernel(float* __restrict__ r, int64_t T, int N, int E) {
+  __shared__ float sv[kRouterRows][256];
+  __shared__ float inv[kRouterRows][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kRouterRows + w;
+  if (t >= T) return;  // warp-uniform; the block never synchronises
+  float* row = r + t * N;
+  for (int j = lane; j < N; j += 32) sv[w][j] = row[j];
+  __syncwarp();
+  for (int h = lane; h < N / E; h += 32) {
+    float sum = 0.f;
+    for (int e = 0; e < E; ++e) sum += sv[w][h * E + e];
+    inv[w][h] = 1.0f / sum;
+  }
+  __syncwarp();
+  for (int j = lane; j < N; j += 32) row[j] = sv[w][j] * inv[w][j / E];
+}
+
+//   dl = s (1 - s) (dR - sum_e dR R) / S  with S = sum_e s, R = s / S  -> bf16 out (row stride
+//   ld_out), from s (rows of `sig`, N values) and dR (rows of N values)
+__global__ void router_bwd_kernel(const float* __restrict__ sig, const float* __restrict__ dr, int64_t T,
+                                  int N, int E, __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  __shared__ float sv[kRouterRows][256];
+  __shared__ float dv[kRouterRows][256];
+  __shared__ float hinv[kRouterRows][256];
+  __shared__ float hdot[kRouterRows][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kRouterRows + w;
+  if (t >= T) return;  // warp-uniform; the block never synchronises
+  for (int j = lane; j < N; j += 32) {
+    sv[w][j] = sig[t * N + j];
+    dv[w][j] = dr[t * N + j];
+  }
+  __syncwarp();
+  for (int h = lane; h < N / E; h += 32) {
+    float sum = 0.f;
+    for (int e = 0; e < E; ++e) sum += sv[w][h * E + e];
+    const float invS = 1.0f / sum;
+    float cdot = 0.f;
+    for (int e = 0; e < E; ++e) cdot = fmaf(dv[w][h * E + e], sv[w][h * E + e] * invS, cdot);
+    hinv[w][h] = invS;
+    hdot[w][h] = cdot;
+  }
+  __syncwarp();
+  __nv_bfloat16* orow = out + t * ld_out;
+  for (int j = lane; j < N; j += 32) {
+    const float s_ = sv[w][j];
+    orow[j] = __float2bfloat16_rn(s_ * (1.f - s_) * (dv[w][j] - hdot[w][j / E]) * hinv[w][j / E]);
+  }
+}
+
+}  // namespace
+}  // namespace swf
+
 // The block's prologue ("Overview": Q is the per-head RMS-normalised projection of the input, R
 // the sigmoid-normalised router weights), as two tcgen05 GEMMs with fused epilogues:
 //   q[t, h*128 + i] = z_h[i] / sqrt(mean_i z_h[i]^2 + eps) * q_gain[i],  z = x w_q^T
@@ -567,7 +631,12 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
   b.out0 = router;
   b.ld_out = nr;
   b.group_size = num_sub;
-  return launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, b, st);
+  if ((s = launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, b, st)) != SWF_OK)
+    return s;
+  ProfScope prof(SWF_K_MHFFN_PROLOGUE, st);
+  router_norm_kernel<<<(unsigned)((T + kRouterRows - 1) / kRouterRows), 32 * kRouterRows, 0, st>>>(
+      router, T, (int)nr, num_sub);
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 
 // ------------------------------------------------------------------ backward (fused per token tile)
@@ -1220,22 +1289,35 @@ extern "C" swf_status flash_mhffn_bwd(const void* q, const void* w_k, const void
 // ------------------------------------------------------------------ prologue backward
 // Gradients of the prologue given dq and drouter: the projection and router GEMMs are recomputed
 // with epilogues that apply the normalisations' backward (kEpiHeadNormBwd: dz and the gain's
-// partial sums; kEpiRouterBwd: dl), writing dz | dl side by side; then dx = [dz | dl] [W_q ; W_r]
+// partial sums; the router's sigmoid, then a row kernel for dl), writing dz | dl side by side;
+// then dx = [dz | dl] [W_q ; W_r]
 // (two K segments) and [dW_q ; dW_r] = [dz | dl]^T x (split-K weight-gradient GEMM); one kernel
 // sums the gain partials in a fixed order.
 namespace swf {
 namespace {
 
-__global__ void dgain_reduce_kernel(const float* __restrict__ part, int64_t rows, float* __restrict__ dgain) {
+// Column sums of the [rows][128] gain-gradient partials in a fixed order: block b of
+// kGainBlocks sums its contiguous range of rows (one thread per column), then one block sums
+// the kGainBlocks results in block order.
+constexpr int kGainBlocks = 256;
+__global__ void dgain_partial_kernel(const float* __restrict__ part, int64_t rows, float* __restrict__ out) {
   const int i = threadIdx.x;  // 128 columns
+  const int64_t per = (rows + kGainBlocks - 1) / kGainBlocks;
+  const int64_t r0 = blockIdx.x * per, r1 = r0 + per < rows ? r0 + per : rows;
   float s = 0.f;
-  for (int64_t r = 0; r < rows; ++r) s += part[r * 128 + i];
+  for (int64_t r = r0; r < r1; ++r) s += part[r * 128 + i];
+  out[blockIdx.x * 128 + i] = s;
+}
+__global__ void dgain_reduce_kernel(const float* __restrict__ part2, float* __restrict__ dgain) {
+  const int i = threadIdx.x;
+  float s = 0.f;
+  for (int b = 0; b < kGainBlocks; ++b) s += part2[b * 128 + i];
   dgain[i] = s;
 }
 
 struct ProBwdWs {
   __nv_bfloat16* dzl;
-  float *sig, *gain_part, *split;
+  float *sig, *gain_part, *gain_part2, *split;
   int64_t ld;
 };
 
@@ -1253,6 +1335,7 @@ ProBwdWs pro_bwd_ws(void* base, int64_t T, int64_t d_model, int64_t H, int64_t E
   w.dzl = reinterpret_cast<__nv_bfloat16*>(take((size_t)T * w.ld * 2));
   w.sig = reinterpret_cast<float*>(take((size_t)T * nr * 4));
   w.gain_part = reinterpret_cast<float*>(take((size_t)round_up(T, 256) / 32 * H * 128 * 4));
+  w.gain_part2 = reinterpret_cast<float*>(take((size_t)kGainBlocks * 128 * 4));
   w.split = reinterpret_cast<float*>(take((size_t)std::max<int64_t>(part_elems(nq + nr, d_model, T), 4) * 4));
   if (bytes) *bytes = off;
   return w;
@@ -1303,7 +1386,10 @@ extern "C" swf_status flash_mhffn_prologue_bwd(
     return SWF_ERR_LAUNCH;
   {  // dz from the recomputed projection (one-CTA tiles of one head; the gain partials are per
      // 32-row slab and head)
-    TcGemmArgs a = base_args(T, nq, 128, d_model);
+    // with an even head count, pair (cta_group::2) tiles of 256 tokens x 256 columns (two heads
+    // per epilogue row), as in the forward; otherwise one-CTA tiles of one head
+    const bool pair = nq % 256 == 0;
+    TcGemmArgs a = pair ? base_args(T, nq, 256, d_model, 2 * kTileM) : base_args(T, nq, 128, d_model);
     a.aux0 = dq;
     a.ld_aux = nq;
     a.bias = q_gain;
@@ -1312,19 +1398,21 @@ extern "C" swf_status flash_mhffn_prologue_bwd(
     a.ld_out = w.ld;
     a.dgain_part = (q_gain && dq_gain) ? w.gain_part : nullptr;
     a.heads = num_heads;
-    if ((s = launch_tc<128, false, false, false, kEpiHeadNormBwd>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st)) != SWF_OK)
-      return s;
+    s = pair ? launch_tc_pair<256, false, false, false, kEpiHeadNormBwd>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq,
+                                                                        EpiMaps{}, a, st)
+             : launch_tc<128, false, false, false, kEpiHeadNormBwd>(SWF_K_MHFFN_PROLOGUE, tx, tq, tq, a, st);
+    if (s != SWF_OK) return s;
   }
   {  // dl from the recomputed router logits, into the columns after dz
     TcGemmArgs a = base_args(T, nr, 256, d_model);
-    a.rw = drouter;
-    a.ld_rw = nr;
-    a.part = w.sig;
-    a.group_size = num_sub;
-    a.out0 = w.dzl + nq;
-    a.ld_out = w.ld;
-    if ((s = launch_tc<256, false, false, false, kEpiRouterBwd>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, a, st)) != SWF_OK)
+    a.out0 = w.sig;
+    a.ld_out = nr;
+    if ((s = launch_tc<256, false, false, false, kEpiRouter>(SWF_K_MHFFN_PROLOGUE, tx, tr, tr, a, st)) != SWF_OK)
       return s;
+    ProfScope prof(SWF_K_MHFFN_PROLOGUE, st);
+    router_bwd_kernel<<<(unsigned)((T + kRouterRows - 1) / kRouterRows), 32 * kRouterRows, 0, st>>>(
+        w.sig, drouter, T, (int)nr, num_sub, w.dzl + nq, w.ld);
+    if (cudaGetLastError() != cudaSuccess) return SWF_ERR_LAUNCH;
   }
   {  // dx = dz W_q + dl W_r: A = [dz | dl] (K = nq + nr), B segments W_q, W_r (MN-major)
     CUtensorMap ta, tbq, tbr;
@@ -1351,7 +1439,9 @@ extern "C" swf_status flash_mhffn_prologue_bwd(
   }
   if (q_gain && dq_gain) {
     ProfScope prof(SWF_K_MHFFN_PROLOGUE, st);
-    dgain_reduce_kernel<<<1, 128, 0, st>>>(w.gain_part, (int64_t)cdiv(T, 128) * 4 * H, dq_gain);
+    dgain_partial_kernel<<<kGainBlocks, 128, 0, st>>>(w.gain_part, (int64_t)cdiv(T, 128) * 4 * H,
+                                                      w.gain_part2);
+    dgain_reduce_kernel<<<1, 128, 0, st>>>(w.gain_part2, dq_gain);
     if (cudaGetLastError() != cudaSuccess) return SWF_ERR_LAUNCH;
   } else if (dq_gain) {
     if (cudaMemsetAsync(dq_gain, 0, 128 * sizeof(float), st) != cudaSuccess) return SWF_ERR_LAUNCH;

@@ -36,15 +36,12 @@
 //                  kernel sums the splits in a fixed order)
 //   kEpiHeadNorm   BN a multiple of 128, heads of 128 columns: C / sqrt(mean(C^2) + eps) * gain
 //                  -> bf16 out0 (FlashFFN's per-head RMS-normalised projection Q)
-//   kEpiRouter     N <= BN = 256 columns, heads of group_size columns: sigmoid(C) divided by its
-//                  sum over the head -> fp32 out0 (FlashFFN's sigmoid-normalised router weights)
+//   kEpiRouter     N <= BN = 256 columns: sigmoid(C) -> fp32 out0 (FlashFFN's router; a row kernel
+//                  then divides each head's values by their sum, or applies that step's backward)
 //   kEpiHeadNormBwd C = z (the projection), heads of 128 columns, with dq (aux0, ld_aux) and the
 //                  gain (bias, nullable): dz = inv (dn - n mean(dn n)), n = z inv, dn = dq gain,
 //                  inv = 1 / sqrt(mean(z^2) + eps) -> bf16 out0; if dgain_part, per 32-row slab
 //                  and head the column sums of dq n -> dgain_part[(m / 32) * heads + h][i]
-//   kEpiRouterBwd  C = router logits l (N <= BN = 256, heads of group_size columns) with dR
-//                  (rw, ld_rw): s = sigmoid(l) -> fp32 scratch (part, ld N) in a first pass, then
-//                  dl = s (1 - s) (dR - sum_e dR R) / sum_e s with R = s / sum_e s -> bf16 out0
 //   kEpiEnergyTopK the energies of a CTA's 128 tokens kept in shared memory; once the CTA has
 //                  scored every group of them (it owns all N-blocks of an M-block, `unit` =
 //                  num_n_blk) each epilogue thread adds the bias to its token's energies (-> out0
@@ -74,8 +71,7 @@ enum : int {
   kEpiEnergyTopK = 10,
   kEpiHeadNorm = 11,
   kEpiRouter = 12,
-  kEpiHeadNormBwd = 14,
-  kEpiRouterBwd = 15
+  kEpiHeadNormBwd = 14
 };
 constexpr int kTopKMaxGroups = 64;  // kEpiEnergyTopK: groups held in registers per token
 enum : int { kModeDense = 0, kModeRowGrouped = 1, kModeKGrouped = 2 };
@@ -115,8 +111,6 @@ struct TcGemmArgs {
   int64_t ld_grp;         // kEpiEnergy*: stride of out0 between groups (0: 1); ld_out is the
                           //   stride between tokens (1 with ld_grp = M: group-major energies)
   float eps;              // kEpiHeadNorm
-  const float* rw;        // kEpiRouterBwd: dR, rw[m * ld_rw + n]
-  int64_t ld_rw;
   float* dgain_part;      // kEpiHeadNormBwd (nullable): [M / 32 * heads][128] gain-gradient partials
   int heads;
   int32_t* sel_idx;       // kEpiEnergyTopK: [M][sel_k] chosen groups
@@ -791,52 +785,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else if constexpr (EPI == kEpiHeadNormBwd) {
+        // three passes over the head's 128 columns, 32 at a time (z re-read from TMEM, dq from
+        // global memory): the mean square, then sum(dn n), then dz and the gain partials; the
+        // sums run in the same column order as one pass would
         static_assert(BN % 128 == 0, "whole heads per tile");
 #pragma unroll 1
         for (int hd = 0; hd < BN / 128; ++hd) {
-          float z[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(t_acc + hd * 128 + c * 32, z[c]);
-          tmem_ld_wait_regs(z[0]);
-          pin_regs(z[1]);
-          pin_regs(z[2]);
-          pin_regs(z[3]);
           const int n0 = t.nb * BN + hd * 128;
           if (n0 >= args.N) continue;  // warp-uniform
+          const uint32_t tz = t_acc + hd * 128;
           const __nv_bfloat16* dqp = static_cast<const __nv_bfloat16*>(args.aux0) + (int64_t)m * args.ld_aux + n0;
-          float ss = 0.f, dot = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(z[c][j], z[c][j], ss);
-          const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
-          // dq of this row (zero for rows past M), kept packed
-          uint32_t dqw[4][16];
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
+          auto load_dq = [&](int c, uint32_t (&w)[16]) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const uint4 d4 = row_ok ? *reinterpret_cast<const uint4*>(dqp + c * 32 + v * 8) : make_uint4(0u, 0u, 0u, 0u);
-              dqw[c][v * 4] = d4.x, dqw[c][v * 4 + 1] = d4.y, dqw[c][v * 4 + 2] = d4.z, dqw[c][v * 4 + 3] = d4.w;
+              w[v * 4] = d4.x, w[v * 4 + 1] = d4.y, w[v * 4 + 2] = d4.z, w[v * 4 + 3] = d4.w;
             }
+          };
+          float ss = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float z[32];
+            tmem_ld32(tz + c * 32, z);
+            tmem_ld_wait_regs(z);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+            for (int j = 0; j < 32; ++j) ss = fmaf(z[j], z[j], ss);
+          }
+          const float inv = rsqrtf(ss * (1.0f / 128.0f) + args.eps);
+          float dot = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float z[32];
+            uint32_t dqw[16];
+            tmem_ld32(tz + c * 32, z);
+            load_dq(c, dqw);
+            tmem_ld_wait_regs(z);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
-              const float nv = z[c][j] * inv;
+              const float dq = (j & 1) ? bf16_hi(dqw[j >> 1]) : bf16_lo(dqw[j >> 1]);
               const float dn = dq * (args.bias ? args.bias[c * 32 + j] : 1.f);
-              dot = fmaf(dn, nv, dot);
+              dot = fmaf(dn, z[j] * inv, dot);
             }
+          }
           const float mdot = dot * (1.0f / 128.0f);
           __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out + n0;
-#pragma unroll
+          float* gp = args.dgain_part
+                          ? args.dgain_part + ((int64_t)((t.a_m + (warp & 3) * 32) / 32) * args.heads + n0 / 128) * 128
+                          : nullptr;
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
+            float z[32];
+            uint32_t dqw[16];
+            tmem_ld32(tz + c * 32, z);
+            load_dq(c, dqw);
+            tmem_ld_wait_regs(z);
             float o[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
-              const float nv = z[c][j] * inv;
+              const float dq = (j & 1) ? bf16_hi(dqw[j >> 1]) : bf16_lo(dqw[j >> 1]);
+              const float nv = z[j] * inv;
               const float dn = dq * (args.bias ? args.bias[c * 32 + j] : 1.f);
               o[j] = inv * (dn - nv * mdot);
             }
@@ -844,55 +851,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int q8 = 0; q8 < 4; ++q8) store_bf16x8(op + c * 32 + q8 * 8, o + q8 * 8);
             }
-          }
-          if (args.dgain_part) {  // column sums of dq * n over the warp's 32 rows (fixed order)
-            float* gp = args.dgain_part + ((int64_t)((t.a_m + (warp & 3) * 32) / 32) * args.heads + n0 / 128) * 128;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
+            if (gp) {  // column sums of dq * n over the warp's 32 rows (fixed order)
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                const float dq = (j & 1) ? bf16_hi(dqw[c][j >> 1]) : bf16_lo(dqw[c][j >> 1]);
-                float v = dq * z[c][j] * inv;
+                const float dq = (j & 1) ? bf16_hi(dqw[j >> 1]) : bf16_lo(dqw[j >> 1]);
+                float v = dq * z[j] * inv;
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
                 if (lane == j) gp[c * 32 + j] = v;
               }
-          }
-        }
-      } else if constexpr (EPI == kEpiRouterBwd) {
-        float* sp = args.part + (int64_t)m * args.N;  // sigmoid scratch row
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float zl[32];
-          tmem_ld32(t_acc + c, zl);
-          tmem_ld_wait_regs(zl);
-          if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) st_if(sp + c + j, sigmoidf_(zl[j]), c + j < args.N);
-          }
-        }
-        if (row_ok) {
-          const int E = args.group_size;
-          const float* drp = args.rw + (int64_t)m * args.ld_rw;
-          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(args.out0) + (int64_t)m * args.ld_out;
-#pragma unroll 1
-          for (int h0 = 0; h0 < args.N; h0 += E) {
-            float S = 0.f;
-#pragma unroll 1
-            for (int e = 0; e < E; ++e) S += sp[h0 + e];
-            const float invS = 1.0f / S;
-            float cdot = 0.f;
-#pragma unroll 1
-            for (int e = 0; e < E; ++e) cdot = fmaf(drp[h0 + e], sp[h0 + e] * invS, cdot);
-#pragma unroll 1
-            for (int e = 0; e < E; ++e) {
-              const float sv = sp[h0 + e];
-              op[h0 + e] = __float2bfloat16_rn(sv * (1.f - sv) * (drp[h0 + e] - cdot) * invS);
             }
           }
         }
       } else if constexpr (EPI == kEpiRouter) {
-        // pass 1: sigmoid of each logit into this token's output row; pass 2: per-head sums
+        // sigmoid of each logit into this token's output row
         float* rp = static_cast<float*>(args.out0) + (int64_t)m * args.ld_out;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -902,18 +874,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (row_ok) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) st_if(rp + c + j, sigmoidf_(z[j]), c + j < args.N);
-          }
-        }
-        if (row_ok) {
-          const int E = args.group_size;
-#pragma unroll 1
-          for (int h0 = 0; h0 < args.N; h0 += E) {
-            float sum = 0.f;
-#pragma unroll 1
-            for (int e = 0; e < E; ++e) sum += rp[h0 + e];
-            const float inv = 1.0f / sum;
-#pragma unroll 1
-            for (int e = 0; e < E; ++e) rp[h0 + e] *= inv;
           }
         }
       } else if constexpr (EPI == kEpiEnergy || EPI == kEpiEnergyTopK) {
