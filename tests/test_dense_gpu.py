@@ -93,6 +93,21 @@ def test_workload2_full_size_sampled():
     assert_close("dw_down[:,cols]", f64(out["dw_down"])[:, cols], sub["dw_down"], torch.bfloat16)
 
 
+def test_workload4_inference_full_size_sampled():
+    """The inference forward at 262144 tokens x 2048 x 5504, the launch configuration of the
+    bench's inference line: sampled token rows against the oracle."""
+    w = synth.WORKLOADS[4]
+    inp = synth.workload_inputs(4)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    y = api.swiglu_ffn_fwd_infer(dev["x"], dev["w_gate"], dev["w_up"], dev["w_down"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    rng = np.random.default_rng(4)
+    rows = np.sort(np.concatenate([rng.choice(w["M"], 32, replace=False), [0, w["M"] - 1]]))
+    x, wg, wu, wd = (f64(inp[k]) for k in ("x", "w_gate", "w_up", "w_down"))
+    assert_close("y[rows]", f64(y)[rows], O.dense_forward(x[rows], wg, wu, wd)["y"], torch.bfloat16)
+
+
 def test_repeat_calls_are_bitwise_identical():
     inp = synth.dense_inputs(1000, 256, 512, seed=7, dtype=torch.bfloat16)
     o1 = run_dense(inp, torch.bfloat16)

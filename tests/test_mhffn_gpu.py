@@ -194,6 +194,35 @@ def test_prologue_backward(T, d_model, H, E, use_gain):
         assert_close("dq_gain", f64(dg), ref["dgain"], torch.float32)
 
 
+def test_prologue_full_size_sampled():
+    """The prologue forward and backward at the bench's block configuration (32768 tokens,
+    d_model 2048, 16 heads, E = 15): q and router rows and dx on sampled tokens; the dW_q and dW_r
+    rows of two heads, each a sum over all tokens that the oracle computes from that head alone."""
+    T, d_model, H, E = 32768, 2048, 16, 15
+    pro = synth.mhffn_prologue_inputs(T, d_model, H, 128, E, seed=6)
+    dq = synth.normal((T, H, 128), 0.1, 6, "do")
+    dr = synth.normal((T, H, E), 0.1, 6, "dy", torch.float32)
+    g = {k: v.cuda() for k, v in pro.items()}
+    q, r = api.flash_mhffn_prologue(g["x"], g["w_q"], g["w_r"], H, E, q_gain=g["q_gain"], eps=1e-6)
+    dx, dwq, dwr, _ = api.flash_mhffn_prologue_bwd(g["x"], g["w_q"], g["w_r"], H, E, dq.cuda(), dr.cuda(),
+                                                   q_gain=g["q_gain"])
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    x, wq, wr, gain = (f64(pro[k]) for k in ("x", "w_q", "w_r", "q_gain"))
+    rng = np.random.default_rng(6)
+    tokens = np.sort(np.concatenate([rng.choice(T, 24, replace=False), [T - 1]]))
+    fw = O.mhffn_prologue_forward(x[tokens], wq, wr, H, E, gain, 1e-6)
+    assert_close("q[tokens]", f64(q)[tokens], fw["q"], torch.bfloat16)
+    assert_close("router[tokens]", f64(r)[tokens], fw["r"], torch.float32)
+    bw = O.mhffn_prologue_backward(x[tokens], wq, wr, H, E, f64(dq)[tokens], f64(dr)[tokens], gain, 1e-6)
+    assert_close("dx[tokens]", f64(dx)[tokens], bw["dx"], torch.bfloat16)
+    for h in (0, 11):
+        qs, rs = slice(h * 128, (h + 1) * 128), slice(h * E, (h + 1) * E)
+        sub = O.mhffn_prologue_backward(x, wq[qs], wr[rs], 1, E, f64(dq)[:, [h]], f64(dr)[:, [h]], gain, 1e-6)
+        assert_close(f"dw_q[head {h}]", f64(dwq)[qs], sub["dw_q"], torch.bfloat16)
+        assert_close(f"dw_r[head {h}]", f64(dwr)[rs], sub["dw_r"], torch.bfloat16)
+
+
 def test_block_training_step_end_to_end():
     """x -> prologue -> fused core -> O, then dO back to dx and every weight gradient, against
     the oracle's block (prologue and core chained)."""
