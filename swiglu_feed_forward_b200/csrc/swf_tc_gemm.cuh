@@ -136,11 +136,19 @@ constexpr int tma_epi_aux() {
   return EPI == kEpiDGate ? 2 : (EPI == kEpiScale ? 1 : 0);
 }
 constexpr int kEpiAuxMap = 2;  // first tensor map of the factors a TMA epilogue loads
+// Buffers per epilogue warp for the factor boxes a TMA epilogue loads: kEpiScale's short-K tiles
+// (the activation gradient of a 512-deep product) prefetch three 32-column chunks ahead.
+template <int EPI>
+constexpr int tma_epi_aux_bufs() {
+  return EPI == kEpiScale ? 4 : 2;
+}
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <int EPI, bool TMA_EPI>
 constexpr int epi_smem_bytes() {
   return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
-                               : (TMA_EPI ? 4 * (tma_epi_outputs<EPI>() + tma_epi_aux<EPI>()) * 2 * kEpiBox : 0);
+                               : (TMA_EPI ? 4 * (2 * tma_epi_outputs<EPI>() + tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>()) *
+                                                kEpiBox
+                                          : 0);
 }
 
 // Tensor maps of a TMA epilogue: outputs in o[0..], then the factors it loads by TMA from
@@ -352,8 +360,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* auxbar = drain + 1;  // [4 epilogue warps][2 buffers]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 8);
+  uint64_t* auxbar = drain + 1;  // [4 epilogue warps][up to 4 buffers]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -376,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[b], PAIR ? 256 : 128);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&auxbar[i], 1);
+    for (int i = 0; i < 16; ++i) mbar_init(&auxbar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -521,9 +529,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int NCH = (kDual ? BN / 2 : BN) / 32;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
-    uint8_t* ebase = smem + L::kEpiOffset + ew * (NOUT + NAUX) * 2 * kEpiBox;
-    uint8_t* abase = ebase + NOUT * 2 * kEpiBox;  // aux buffers [2][NAUX]
-    uint64_t* abar = auxbar + ew * 2;
+    constexpr int AB = tma_epi_aux_bufs<EPI>();
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (2 * NOUT + AB * NAUX) * kEpiBox;
+    uint8_t* abase = ebase + NOUT * 2 * kEpiBox;  // aux buffers [AB][NAUX]
+    uint64_t* abar = auxbar + ew * AB;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this lane's staging row
     uint32_t aux_issued = 0, aux_done = 0, chunks = 0;
@@ -541,7 +550,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       auto issue_aux = [&](int c) {
         if constexpr (NAUX > 0) {
           if (lane == 0) {
-            const int db = aux_issued & 1;
+            const int db = aux_issued % AB;
             mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
             tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[kEpiAuxMap], n_base + c * 32, m_slab,
                         &abar[db]);
@@ -551,7 +560,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++aux_issued;
         }
       };
-      issue_aux(0);  // the factors do not depend on the accumulator: fetch them early
+      // the factors do not depend on the accumulator: fetch the first chunks' early
+      for (int c = 0; c < AB - 1 && c < NCH; ++c) issue_aux(c);
       const bool ready = mbar_wait(&tfull[buf], use & 1u, ctl);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ready)) {
@@ -565,9 +575,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c = 0; c < NCH; ++c) {
         const uint8_t* aux = nullptr;
         if constexpr (NAUX > 0) {
-          if (c + 1 < NCH) issue_aux(c + 1);
-          const int db = aux_done & 1;
-          const bool got = mbar_wait(&abar[db], (aux_done >> 1) & 1u, ctl);
+          if (c + AB - 1 < NCH) issue_aux(c + AB - 1);
+          const int db = aux_done % AB;
+          const bool got = mbar_wait(&abar[db], (aux_done / AB) & 1u, ctl);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) {
             ok = false;
@@ -688,7 +698,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       WaitCtl quick{abort_flag, args.status, 100000000ull};
       volatile int no_abort = 0;
       quick.abort = &no_abort;
-      for (; aux_done < aux_issued; ++aux_done) mbar_wait(&abar[aux_done & 1], (aux_done >> 1) & 1u, quick);
+      for (; aux_done < aux_issued; ++aux_done) mbar_wait(&abar[aux_done % AB], (aux_done / AB) & 1u, quick);
       bulk_wait_all();
     }
   } else {
