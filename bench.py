@@ -408,7 +408,8 @@ def secondary_mhffn(api, steps, warmup, world, peak):
         block()
     ms_b = timed(block, steps, world)
     flops_b = flops + 2.0 * T * d_model * (H * dh + H * E)
-    # backward (per-head GEMMs; writes the head's activations to a workspace)
+    # backward (one fused kernel per group of four heads, then split-K weight-gradient GEMMs over
+    # the dS and P planes it leaves in the workspace)
     dout = synth.normal((T, H, dh), synth.DY_STD, w["seed"], "do").to(dev)
     gq, gk, gu, gv, gr = (torch.empty_like(t[k]) for k in ("q", "w_k", "w_u", "w_v", "router"))
     ws = torch.empty(max(16, api.flash_mhffn_bwd_workspace_bytes(T, H, dh, E, de)), device=dev,
