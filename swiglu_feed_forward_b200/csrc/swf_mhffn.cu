@@ -664,9 +664,9 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
 // rows (32 per CTA) for dA.  Shared memory: Q and dO 64 KB, S ring 2 x 16, V ring 2 x 8, dQ ring
 // 2 x 16, two dS buffers of 32 KB, P staging 16 KB = 224 KB.
 //
-// Threads (384 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 3 lane 0
-// the V ring and, in the even CTA, issues the dA products; warp 2 lane 0 the dQ ring and, in the
-// even CTA, issues the dQ products; warp 1 owns TMEM and, in the even CTA, issues the S products
+// Threads (672 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 20 lane 0
+// the V ring; warp 3 lane 0 (even CTA) issues the dA products; warp 2 lane 0 the dQ ring and, in
+// the even CTA, issues the dQ products; warp 1 owns TMEM and, in the even CTA, issues the S products
 // (one issuing thread per product stream: a thread issues about one tcgen05.mma per 60-90
 // cycles); warps 4..11 form dS_g, dS_u, P for every chunk (warp (q, hc): token rows 32q..32q+31,
 // the chunk's columns 32hc..32hc+31; chunk c uses TMEM buffer c & 1 and dS buffer c & 1), and at
@@ -680,7 +680,8 @@ constexpr int kBwDqStages = 2;
 constexpr int kBwVBox = 32 * 64 * 2;          // 32 V rows x 64 d_h (4 KB)
 constexpr int kBwVBytes = 2 * kBwVBox;        // this CTA's 32 rows of V_c
 constexpr int kBwEpiWarps = 16;              // four per TMEM lane quadrant, 16 columns each
-constexpr int kBwThreads = 128 + 32 * kBwEpiWarps;
+constexpr int kBwVWarp = 4 + kBwEpiWarps;    // the V-ring producer, after the epilogue warps
+constexpr int kBwThreads = 32 * (kBwVWarp + 1);
 constexpr int kBwCols = kMhChunk / 4;         // columns of a chunk per epilogue warp
 constexpr int kBwDsAtom = 128 * kBwCols * 2;  // 128 rows x 16 bf16 (32-byte rows): one K16 atom
 constexpr int kBwDsBytes = 8 * kBwDsAtom;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
@@ -779,7 +780,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tma_prefetch_desc(&tmDO);
     tma_prefetch_desc(rank == 0 ? &tmK : &tmU);
   }
-  if (warp == 3 && lane == 0) tma_prefetch_desc(&tmV);
+  if (warp == kBwVWarp && lane == 0) tma_prefetch_desc(&tmV);
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmDS);
     tma_prefetch_desc(&tmP);
@@ -826,47 +827,41 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
       }
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ V ring and dA issuer
-    // The loads run at most kBwVStages - 1 chunks ahead of the dA products (in the even CTA this
-    // thread issues the products that free the stages).
+  } else if (warp == kBwVWarp) {
+    // ------------------------------------------------------------ V-ring producer (both CTAs)
+    // A thread of its own, so the loads run ahead as soon as the dA products free a stage.
     if (lane == 0) {
       const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
-      const int my_units = cl < args.n_units ? (args.n_units - cl + n_cl - 1) / n_cl : 0;
-      const uint32_t total = static_cast<uint32_t>(my_units) * static_cast<uint32_t>(args.nch);
-      uint32_t nl = 0;  // chunks whose V rows were requested
+      uint32_t gc = 0;
+      bool ok = true;
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl) {
+        const int h = args.h0 + unit / args.n_pt;
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const int row = h * rows_per_head + c * kMhChunk + static_cast<int>(rank) * 32;
+          const uint32_t sv = gc % kBwVStages;
+          if (!mbar_wait(&v_empty[sv], ((gc / kBwVStages) & 1u) ^ 1u, ctl)) { ok = false; break; }
+          uint8_t* vb = smem + kBwVOff + sv * kBwVBytes;
+          if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kBwVBytes);
+          tma_load_2d_pair(vb, &tmV, 0, row, v_full_lead + sv * 8);
+          tma_load_2d_pair(vb + kBwVBox, &tmV, 64, row, v_full_lead + sv * 8);
+        }
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ dA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);
+      const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
+      uint32_t gc = 0;
+      int lu = 0;
       bool ok = true, issued = false;
-      auto load_next = [&]() -> bool {
-        const int unit = cl + static_cast<int>(nl / args.nch) * n_cl;
-        const int c = static_cast<int>(nl % args.nch);
-        const int row = (args.h0 + unit / args.n_pt) * rows_per_head + c * kMhChunk +
-                        static_cast<int>(rank) * 32;
-        const uint32_t sv = nl % kBwVStages;
-        if (!mbar_wait(&v_empty[sv], ((nl / kBwVStages) & 1u) ^ 1u, ctl)) return false;
-        uint8_t* vb = smem + kBwVOff + sv * kBwVBytes;
-        if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * kBwVBytes);
-        tma_load_2d_pair(vb, &tmV, 0, row, v_full_lead + sv * 8);
-        tma_load_2d_pair(vb + kBwVBox, &tmV, 64, row, v_full_lead + sv * 8);
-        ++nl;
-        return true;
-      };
-      if (rank != 0) {
-        while (ok && nl < total) ok = load_next();
-      } else {
-        constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);
-        const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
-        const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
-        while (ok && nl < total && nl < static_cast<uint32_t>(kBwVStages)) ok = load_next();
-        int lu = -1;
-        for (uint32_t i = 0; ok && i < total; ++i) {
-          const int c = static_cast<int>(i % args.nch);
-          if (c == 0) {
-            ++lu;
-            if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
-          }
-          const uint32_t sv = i % kBwVStages, b = i & 1u;
-          if (!mbar_wait(&v_full[sv], (i / kBwVStages) & 1u, ctl)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[b], ((i >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
+      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
+        if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
+        for (int c = 0; c < args.nch; ++c, ++gc) {
+          const uint32_t sv = gc % kBwVStages, b = gc & 1u;
+          if (!mbar_wait(&v_full[sv], (gc / kBwVStages) & 1u, ctl)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem_base + kMhDh + b * kBwBufCols + 2 * kMhChunk;
           const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
@@ -881,10 +876,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           umma_commit_pair(&v_empty[sv], 3);
           if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // dO no longer read in this unit
           issued = true;
-          while (ok && nl < total && nl < i + kBwVStages) ok = load_next();
         }
-        if (!ok && issued) drain_mma(&drain[2], abort_flag, args.status);
       }
+      if (!ok && issued) drain_mma(&drain[2], abort_flag, args.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer (even CTA)
