@@ -664,13 +664,13 @@ extern "C" swf_status flash_mhffn_prologue(const void* x, const void* w_q, const
 // rows (32 per CTA) for dA.  Shared memory: Q and dO 64 KB, S ring 2 x 16, V ring 2 x 8, dQ ring
 // 2 x 16, two dS buffers of 32 KB, P staging 16 KB = 224 KB.
 //
-// Threads (672 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 20 lane 0
-// the V ring; warp 3 lane 0 (even CTA) issues the dA products; warp 2 lane 0 the dQ ring and, in
-// the even CTA, issues the dQ products; warp 1 owns TMEM and, in the even CTA, issues the S products
-// (one issuing thread per product stream: a thread issues about one tcgen05.mma per 60-90
-// cycles); warps 4..11 form dS_g, dS_u, P for every chunk (warp (q, hc): token rows 32q..32q+31,
-// the chunk's columns 32hc..32hc+31; chunk c uses TMEM buffer c & 1 and dS buffer c & 1), and at
-// the end of a unit they drain dQ.  Every wait is bounded.
+// Threads (640 per CTA): warp 0 lane 0 loads Q, dO (once per unit) and the S ring; warp 3 lane 0
+// the V ring; warp 2 lane 0 the dQ ring and, in the even CTA, issues the dQ products; warp 1 owns
+// TMEM and, in the even CTA, issues the S and dA products (a thread issues about one tcgen05.mma
+// per 60-90 cycles, so the dQ products come from a second thread); warps 4..19 form dS_g, dS_u, P
+// for every chunk (warp (q, qc): token rows 32q..32q+31, the chunk's columns 16qc..16qc+15;
+// chunk c uses TMEM buffer c & 1 and dS buffer c & 1), and at the end of a unit they drain dQ.
+// Every wait is bounded.
 namespace swf {
 namespace {
 
@@ -680,8 +680,8 @@ constexpr int kBwDqStages = 2;
 constexpr int kBwVBox = 32 * 64 * 2;          // 32 V rows x 64 d_h (4 KB)
 constexpr int kBwVBytes = 2 * kBwVBox;        // this CTA's 32 rows of V_c
 constexpr int kBwEpiWarps = 16;              // four per TMEM lane quadrant, 16 columns each
-constexpr int kBwVWarp = 4 + kBwEpiWarps;    // the V-ring producer, after the epilogue warps
-constexpr int kBwThreads = 32 * (kBwVWarp + 1);
+constexpr int kBwVWarp = 3;                  // the V-ring producer
+constexpr int kBwThreads = 128 + 32 * kBwEpiWarps;
 constexpr int kBwCols = kMhChunk / 4;         // columns of a chunk per epilogue warp
 constexpr int kBwDsAtom = 128 * kBwCols * 2;  // 128 rows x 16 bf16 (32-byte rows): one K16 atom
 constexpr int kBwDsBytes = 8 * kBwDsAtom;     // dS_g and dS_u of one chunk (2 x 128 x 64 bf16)
@@ -750,7 +750,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     // arrival counts are those of the even CTA's barriers, the only ones waited on with them
     // (the dQ-ring and dS barriers are also waited on in the odd CTA: commit arrivals only)
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 2);  // the S and the dA issuer each release Q / dO
+    mbar_init(q_empty, 1);  // released by the S / dA issuer
     for (int s = 0; s < kBwSuStages; ++s) {
       mbar_init(&su_full[s], 1);
       mbar_init(&su_empty[s], 1);
@@ -764,7 +764,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       mbar_init(&w_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 2);                   // S products and dA products
+      mbar_init(&s_full[b], 1);                   // the S and dA products of a chunk
       mbar_init(&s_empty[b], 2 * kBwEpiWarps);    // one arrival per epilogue warp, both CTAs
       mbar_init(&ds_full[b], 2 * kBwEpiWarps);
       mbar_init(&ds_empty[b], 1);
@@ -829,7 +829,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
   } else if (warp == kBwVWarp) {
     // ------------------------------------------------------------ V-ring producer (both CTAs)
-    // A thread of its own, so the loads run ahead as soon as the dA products free a stage.
+    // A thread of its own, so the loads run ahead as soon as the dA products free a stage (an
+    // issuing thread that also refilled the ring waited a whole load latency every chunk).
     if (lane == 0) {
       const uint32_t v_full_lead = map_to_rank(smem_u32(v_full), 0);
       uint32_t gc = 0;
@@ -847,41 +848,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
       }
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ dA issuer (even CTA)
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);
-      const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
-      uint32_t gc = 0;
-      int lu = 0;
-      bool ok = true, issued = false;
-      for (int unit = cl; ok && unit < args.n_units; unit += n_cl, ++lu) {
-        if (!mbar_wait(q_full, lu & 1, ctl)) { ok = false; break; }
-        for (int c = 0; c < args.nch; ++c, ++gc) {
-          const uint32_t sv = gc % kBwVStages, b = gc & 1u;
-          if (!mbar_wait(&v_full[sv], (gc / kBwVStages) & 1u, ctl)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[b], ((gc >> 1) & 1u) ^ 1u, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem_base + kMhDh + b * kBwBufCols + 2 * kMhChunk;
-          const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16_pair(d, desc_add(do_desc, kb * (kMhQBytes / 2) + k * 32),
-                             desc_add(vd, kb * kBwVBox + k * 32), kIdescA, (kb | k) != 0 ? 1u : 0u);
-          }
-          umma_commit_pair(&s_full[b], 3);
-          umma_commit_pair(&v_empty[sv], 3);
-          if (c == args.nch - 1) umma_commit_pair(q_empty, 3);  // dO no longer read in this unit
-          issued = true;
-        }
-      }
-      if (!ok && issued) drain_mma(&drain[2], abort_flag, args.status);
-    }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ S issuer (even CTA)
+    // ------------------------------------------------------------ S and dA issuer (even CTA)
+    // 16 products per chunk from one thread (about 1600 cycles of issue against a chunk's 3000 or
+    // more), so the V ring can have a producer thread of its own.
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(2 * kMhTile, 2 * kMhChunk, 0, 0);  // [g | u]
       const uint64_t q_desc = smem_desc_sw128(smem_u32(smem), 16, 1024);
@@ -905,6 +875,23 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             for (int k = 0; k < 4; ++k)
               umma_bf16_pair(d, desc_add(q_desc, kb * (kMhQBytes / 2) + k * 32),
                              desc_add(sd, kb * kMhBox + k * 32), kIdescS, (kb | k) != 0 ? 1u : 0u);
+          }
+          {
+            constexpr uint32_t kIdescA = idesc_bf16(2 * kMhTile, kMhChunk, 0, 0);
+            const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + kBwDoOff), 16, 1024);
+            const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kBwVOff), 16, 1024);
+            const uint32_t sv = gc % kBwVStages;
+            if (!mbar_wait(&v_full[sv], (gc / kBwVStages) & 1u, ctl)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t vd = desc_add(v_desc, sv * kBwVBytes);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                umma_bf16_pair(d + 2 * kMhChunk, desc_add(do_desc, kb * (kMhQBytes / 2) + k * 32),
+                               desc_add(vd, kb * kBwVBox + k * 32), kIdescA, (kb | k) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&v_empty[sv], 3);
           }
           umma_commit_pair(&s_full[b], 3);
           umma_commit_pair(&su_empty[s], 3);
