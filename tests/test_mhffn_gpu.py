@@ -122,6 +122,7 @@ def test_block_prologue_then_fused_forward():
     (300, 1, 2, 256),    # two 128-column blocks per sub-network
     (700, 3, 2, 384),    # the 1.3B sub-network width, odd head count
     (4000, 5, 1, 128),   # two launches (four heads, then one), more units than clusters
+    (333, 2, 2, 512),    # eight 64-column chunks per sub-network, ragged tokens
 ])
 def test_backward(T, H, E, de):
     inp = synth.mhffn_inputs(T, H, 128, E, de, seed=T + 3 * E)
