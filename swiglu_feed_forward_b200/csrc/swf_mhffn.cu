@@ -43,7 +43,6 @@ constexpr int kMhKuStages = 4;   // K|U chunk stages (free once the chunk's S pr
 constexpr int kMhVStages = 6;    // V chunk stages (free once its PV product is done)
 constexpr int kMhEpiWarps = 8;   // two sets of four (one warp per TMEM lane quadrant each)
 constexpr int kMhThreads = 128 + 32 * kMhEpiWarps;  // 2 producers, S and PV issuers, epilogue
-constexpr int kMhEpiThreads = 32 * kMhEpiWarps;
 constexpr int kMhBox = 64 * 64 * 2;                 // one 64 x 64 bf16 TMA box (8 KB)
 constexpr int kMhQBytes = 2 * kMhTile * 64 * 2;     // Q tile: two 128 x 64 boxes
 constexpr int kMhKuBytes = 2 * kMhBox;              // this CTA's half of [K; U]: two d_h boxes
@@ -78,21 +77,14 @@ __device__ __forceinline__ uint32_t p_offset(int row, int c16) {
   return static_cast<uint32_t>(row * 128 + ((c16 ^ (row & 7)) << 4));
 }
 
-// SiLU(z) = z * sigmoid(z) with sigmoid(z) = (1 + tanh(z / 2)) / 2: one MUFU operation
-// (tanh.approx.f32, relative error about 2^-11) instead of an exponential and a reciprocal.  The
-// epilogue is bound by the MUFU pipe, and P is rounded to bf16 (2^-9) right after.
-__device__ __forceinline__ float silu_tanh(float z) {
-  const float hz = 0.5f * z;
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hz));
-  return fmaf(hz, t, hz);
-}
-
 __device__ constexpr float2 kHalf2 = {0.5f, 0.5f};
 __device__ constexpr float2 kMinusHalf2 = {-0.5f, -0.5f};
 
-// SiLU(g) * u * r for two columns with Blackwell's paired fp32 operations (mul/fma .f32x2, IEEE
-// round-to-nearest like the scalar forms, so the result equals silu_tanh(g) * u * r), as bf16x2.
+// SiLU(g) * u * r for two columns, as bf16x2.  SiLU(g) = g sigmoid(g) with sigmoid(g) =
+// (1 + tanh(g / 2)) / 2, i.e. h + h tanh(h) with h = g / 2: one MUFU operation (tanh.approx.f32,
+// relative error about 2^-11) instead of an exponential and a reciprocal, the rest in Blackwell's
+// paired fp32 operations (mul/fma .f32x2, IEEE round-to-nearest like the scalar forms).  The
+// result is rounded to bf16 (2^-9) right after.
 __device__ __forceinline__ uint32_t silu_mul_pair(float ga, float gb, float ua, float ub, float2 r2) {
   const float2 h2 = __fmul2_rn(make_float2(ga, gb), kHalf2);
   float2 th;
@@ -120,24 +112,11 @@ __device__ __forceinline__ void warp_arrive_lead(uint64_t* bar, uint32_t rank, i
   }
 }
 
-// UMMA shared-memory descriptor (sm_100 format) of a K-major operand in the 64-byte-swizzle
-// layout: rows of 64 bytes (32 bf16 of K), 16-byte chunk c of row r at chunk position
-// c ^ ((r >> 1) & 3), 8-row groups `sbo_bytes` apart (layout type 4 at bits 61..63; the leading
-// byte offset is not used by swizzled K-major layouts).  Tiles are 512-byte aligned so the
-// swizzle phase is that of the address.
-__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;
-  d |= 4ull << 61;
-  return d;
-}
-
-// The same for the 32-byte-swizzle layout: rows of 32 bytes (16 bf16 of K, one K16 step), 16-byte
-// chunk c of row r at chunk position c ^ ((r >> 2) & 1), 8-row groups `sbo_bytes` apart (layout
-// type 6).  Tiles are 256-byte aligned.
+// UMMA shared-memory descriptor (sm_100 format) of a K-major operand in the 32-byte-swizzle
+// layout: rows of 32 bytes (16 bf16 of K, one K16 step), 16-byte chunk c of row r at chunk
+// position c ^ ((r >> 2) & 1), 8-row groups `sbo_bytes` apart (layout type 6 at bits 61..63; the
+// leading byte offset is not used by swizzled K-major layouts).  Tiles are 256-byte aligned so
+// the swizzle phase is that of the address.
 __device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
