@@ -307,6 +307,26 @@ def secondary_infer(api, steps, warmup, world):
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
+def sparse_step_hbm_bytes(M, d, f, G, K, spg, R):
+    """HBM bytes the group-sparse step's kernels must move in this design (bf16 data, int32
+    indices), with R the padded pair rows: selection (x, the sampled gate rows, the chosen
+    groups), the gathers (x and dY rows written group-major; the token rows come from L2), the
+    row-grouped GEMMs (gathered rows, the group's weights, h, a, b, [dG | dU]), the per-pair y and
+    dx contributions written and summed, and the grouped weight gradients."""
+    b, ng = 2, f // G
+    P = 1 << max(0, (spg - 1).bit_length())
+    select = b * M * d + b * ng * P * d + 4 * M * K
+    buckets = 3 * 4 * M * K
+    gather = b * R * d + b * M * d                               # one of x, dY
+    up = b * R * d + 2 * b * f * d + 3 * b * R * G
+    down = b * R * G + b * d * f + b * R * d
+    pair_sum = b * R * d + b * M * d + 4 * M * K                 # one of y, dx
+    dgate = b * R * d + b * d * f + 2 * b * R * G + b * R * 128
+    dxg = b * R * 128 + 2 * b * f * d + b * R * d
+    dw = (b * R * 128 + b * R * d + 2 * b * f * d) + (b * R * d + b * R * G + b * d * f)
+    return select + buckets + 2 * gather + up + down + 2 * pair_sum + dgate + dxg + dw
+
+
 def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     w = synth.WORKLOADS[3]
     M, d, f, G, K, spg = (w[k] for k in ("M", "d_model", "d_ff", "group_size", "num_active_groups",
@@ -347,6 +367,10 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     useful = 2.0 * M * d * ng * spg + 18.0 * M * d * K * G
     tf = useful * steps / (ms / 1e3) / 1e12
     per_group = torch.bincount(idx.flatten().long(), minlength=ng)
+    R = int(((per_group + 127) // 128 * 128).sum())
+    hbm_bytes = sparse_step_hbm_bytes(M, d, f, G, K, spg, R)
+    hbm_peak = float(load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    hbm_gbs = hbm_bytes / (ms_graph / steps / 1e3) / 1e9
     return {"workload": w["name"] + (" (skewed bias: +0.5 on 2 groups, -0.5 on 2)" if skewed else ""),
             "useful_tflops": round(tf * world, 3),
             "pct_of_peak": round(100 * tf / peak, 2), "ms_per_step": round(ms / steps, 3),
@@ -354,7 +378,12 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
             "cuda_graph": {"ms_per_step": round(ms_graph / steps, 3),
                            "useful_tflops": round(useful * steps / (ms_graph / 1e3) / 1e12 * world, 3)},
             "tokens_per_group": {"max": int(per_group.max()), "mean": round(M * K / ng, 1),
-                                 "min": int(per_group.min())}}
+                                 "min": int(per_group.min())},
+            "roofline": {"bound": "hbm", "achieved": round(hbm_gbs * world, 1), "peak": hbm_peak,
+                         "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4), "traffic": None,
+                         "bytes_per_step": hbm_bytes, "padded_pair_rows": R,
+                         "basis": "the step's design traffic (sparse_step_hbm_bytes) over the CUDA-graph "
+                                  "step time"}}
 
 
 def secondary_mlp2(api, steps, warmup, world, peak):
