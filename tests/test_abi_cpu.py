@@ -111,6 +111,10 @@ def test_mhffn_argument_errors(lib):
     assert b(p, p, p, p, p, p, p, p, p, p, p, None, 0, 256, 16, 128, 15, 384, BF, None) == 4        # no workspace
     assert lib.flash_mhffn_bwd_workspace_bytes(256, 16, 128, 15, 384, BF) > 256 * 5760 * 8
     assert lib.flash_mhffn_bwd_workspace_bytes(256, 16, 64, 15, 384, BF) == 0
+    # the dS_g | dS_u and P planes are held for at most four heads at a time
+    planes = lambda g: g * 4096 * 5760 * 2 * 3
+    w2, w4, w8 = (lib.flash_mhffn_bwd_workspace_bytes(4096, h, 128, 15, 384, BF) for h in (2, 4, 8))
+    assert planes(2) <= w2 < planes(4) <= w4 and w8 - w4 < planes(1)
     g = lib.flash_mhffn_prologue
     assert g(None, p, None, p, p, p, 256, 2048, 16, 128, 15, 1e-6, BF, None) == 1  # null x
     assert g(p, p, None, p, p, p, 256, 2048, 16, 128, 15, -1.0, BF, None) == 1     # eps < 0
