@@ -146,9 +146,14 @@ swf_status dense_fwd_bf16(const void* x, const void* wg, const void* wu, const v
   k1.aux0 = a;
   k1.aux1 = b;
   k1.ld_aux = f;
+  // h (and a, b) leave through per-warp staging boxes and TMA stores
+  EpiMaps e1{};
+  if (!epi_map(&e1.o[0], h, f, M, f) ||
+      (!infer && (!epi_map(&e1.o[1], a, f, M, f) || !epi_map(&e1.o[2], b, f, M, f))))
+    return SWF_ERR_LAUNCH;
   swf_status s =
-      infer ? launch_tc_pair<256, false, false, true, kEpiSwiGLUInf>(SWF_K_GATE_UP_INFER, tx, twg, twu, EpiMaps{}, k1, st)
-            : launch_tc_pair<256, false, false, true, kEpiSwiGLU>(SWF_K_GATE_UP, tx, twg, twu, EpiMaps{}, k1, st);
+      infer ? launch_tc_pair<256, false, false, true, kEpiSwiGLUInf, true>(SWF_K_GATE_UP_INFER, tx, twg, twu, e1, k1, st)
+            : launch_tc_pair<256, false, false, true, kEpiSwiGLU, true>(SWF_K_GATE_UP, tx, twg, twu, e1, k1, st);
   if (s != SWF_OK) return s;
   // K2: y = h W_d^T
   TcGemmArgs k2 = base_args(M, d, 256, f, 2 * kTileM);

@@ -27,7 +27,7 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE, false, TMA_EPI>;
-  constexpr int smem = TcSmem<BN, false, epi_smem_bytes<EPI, TMA_EPI>()>::kBytes;
+  constexpr int smem = TcSmem<BN, false, epi_smem_bytes<EPI, TMA_EPI, false>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int64_t units = args.unit > 1 ? (tiles + args.unit - 1) / args.unit : tiles;
@@ -54,7 +54,7 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, kModeDense, true, TMA_EPI>;
-  constexpr int smem = TcSmem<BN, true, epi_smem_bytes<EPI, TMA_EPI>()>::kBytes;
+  constexpr int smem = TcSmem<BN, true, epi_smem_bytes<EPI, TMA_EPI, true>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int clusters = (int)std::min<int64_t>(tiles, ctx.num_sms / 2);

@@ -125,8 +125,14 @@ struct TcGemmArgs {
 };
 
 // Epilogues that move their tiles with TMA: bf16 outputs staged per warp in shared memory
-// (32 x 32 boxes, 64-byte swizzle, double-buffered) and, for kEpiDGate, the a/b factor tiles
-// loaded by TMA into the same kind of buffers.
+// (32 x 32 boxes, 64-byte swizzle) and, for kEpiDGate, the a/b factor tiles loaded by TMA into
+// the same kind of buffers.  Pair-mode (dense) kernels keep one box per output, which a warp
+// overwrites once the previous chunk's store has read it (the chunk's TMEM load and arithmetic
+// cover that); this leaves the gate|up kernel its six ring stages.  Measured with a %clock64
+// probe of the MMA issuer on B200, its k-blocks then take about 605 cycles, against about 690
+// with per-thread 16-byte row stores and 613 with two boxes per output and five stages.  The
+// 1-CTA row-grouped tiles of the sparse path keep two boxes per output (one box: sparse dx
+// 6% slower).
 template <int EPI>
 constexpr int tma_epi_outputs() {
   return EPI == kEpiSwiGLU ? 3 : ((EPI == kEpiDGate || EPI == kEpiLeakySq) ? 2 : 1);
@@ -143,10 +149,15 @@ constexpr int tma_epi_aux_bufs() {
   return EPI == kEpiScale ? 4 : 2;
 }
 constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
-template <int EPI, bool TMA_EPI>
+template <bool PAIR>
+constexpr int tma_epi_out_bufs() {
+  return PAIR ? 1 : 2;
+}
+template <int EPI, bool TMA_EPI, bool PAIR>
 constexpr int epi_smem_bytes() {
   return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
-                               : (TMA_EPI ? 4 * (2 * tma_epi_outputs<EPI>() + tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>()) *
+                               : (TMA_EPI ? 4 * (tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>() +
+                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>()) *
                                                 kEpiBox
                                           : 0);
 }
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ EpiMaps emaps,
                    const TcGemmArgs args) {
-  using L = TcSmem<BN, PAIR, epi_smem_bytes<EPI, TMA_EPI>()>;
+  using L = TcSmem<BN, PAIR, epi_smem_bytes<EPI, TMA_EPI, PAIR>()>;
   constexpr int S = L::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(PAIR ? 2 * kTileM : kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
   constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
@@ -530,8 +541,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
     constexpr int AB = tma_epi_aux_bufs<EPI>();
-    uint8_t* ebase = smem + L::kEpiOffset + ew * (2 * NOUT + AB * NAUX) * kEpiBox;
-    uint8_t* abase = ebase + NOUT * 2 * kEpiBox;  // aux buffers [AB][NAUX]
+    constexpr int OB = tma_epi_out_bufs<PAIR>();
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT + AB * NAUX) * kEpiBox;  // boxes [NOUT][OB]
+    uint8_t* abase = ebase + OB * NOUT * kEpiBox;  // aux buffers [AB][NAUX]
     uint64_t* abar = auxbar + ew * AB;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this lane's staging row
@@ -659,12 +671,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         // stage this warp's 32 x 32 box of every output, then one lane stores them with TMA
-        const int db = chunks & 1;
-        if (lane == 0) bulk_wait_read<1>();  // the store that last used buffer db has read it
+        const int db = OB > 1 ? static_cast<int>(chunks & 1u) : 0;
+        if (lane == 0) bulk_wait_read<OB - 1>();  // the store that last used box db has read it
         __syncwarp();
 #pragma unroll
         for (int o = 0; o < NOUT; ++o) {
-          uint8_t* ob = ebase + (o * 2 + db) * kEpiBox;
+          uint8_t* ob = ebase + (o * OB + db) * kEpiBox;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4)
             *reinterpret_cast<uint4*>(ob + lane * 64 + ((c4 ^ swz) * 16)) =
@@ -682,7 +694,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
 #pragma unroll
             for (int o = 0; o < NOUT; ++o)
-              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * 2 + db) * kEpiBox);
+              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * OB + db) * kEpiBox);
           }
           bulk_commit();
         }
