@@ -479,11 +479,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
+    // This one thread's issue loop bounds the dense GEMMs (a %clock64 probe on B200: precomputed
+    // descriptors took dx from 542 to 528 cycles per k-block), so it does as little as it can:
+    // the smem descriptors of stage 0 are built once and a stage / K step adds its byte offset
+    // / 16 to the address field (the whole ring lies below 256 KB, so the 14-bit field cannot
+    // carry), and the stage index and phase advance by increment.
     if (lane == 0 && rank == 0) {
-      uint32_t it = 0;
+      int s = 0;        // ring stage of the next k-block
+      uint32_t ph = 0;  // parity of its full barrier
       int local = 0;
       bool ok = true;
       bool issued = false;
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t a_desc0 = A_MN ? smem_desc_sw128(sbase, 8192, 1024) : smem_desc_sw128(sbase, 16, 1024);
+      const uint64_t b_desc0 = B_MN ? smem_desc_sw128(sbase + L::kABytes, 8192, 1024)
+                                    : smem_desc_sw128(sbase + L::kABytes, 16, 1024);
+      constexpr uint64_t kAStep = A_MN ? 2048 / 16 : 32 / 16;  // one K step of 16
+      constexpr uint64_t kBStep = B_MN ? 2048 / 16 : 32 / 16;
+      static_assert(L::kTileBytes + 2048 < (1 << 18), "descriptor address field");
       for (int i_ = 0, tile = tile0 * unit_; ok && tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
         const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
         if (t.grp < 0) continue;
@@ -493,24 +506,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
-        for (int kb = 0; kb < t.kb; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1u;
+        for (int kb = 0; kb < t.kb; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + s * L::kStageBytes);
-          const uint32_t b0 = a0 + L::kABytes;
+          const uint64_t so = static_cast<uint64_t>(s) * (L::kStageBytes / 16);
 #pragma unroll
           for (int k = 0; k < kTileK / kUmmaK; ++k) {
-            const uint64_t ad = A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
-                                     : smem_desc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
-                                     : smem_desc_sw128(b0 + k * 32, 16, 1024);
+            const uint64_t ad = a_desc0 + so + k * kAStep;
+            const uint64_t bd = b_desc0 + so + k * kBStep;
             if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
             else umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
           if constexpr (PAIR) umma_commit_pair(&empty[s], 3);
           else umma_commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
           issued = true;
         }
         if (!ok) break;
