@@ -806,7 +806,7 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 256))
       return SWF_ERR_LAUNCH;
     EpiMaps em{};
-    if (!encode_tmap_bf16(&em.o[0], w.yc, d, sd.rmax, d, 32, 32, 64)) return SWF_ERR_LAUNCH;
+    if (!encode_tmap_bf16(&em.o[0], w.yc, d, sd.rmax, d, 64, 32, 128)) return SWF_ERR_LAUNCH;  // 32 x 64 boxes
     TcGemmArgs a = base_args(sd.rmax, d, 256, G);
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
@@ -869,7 +869,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
     EpiMaps em{};
-    if (!encode_tmap_bf16(&em.o[0], w.dxc, d, sd.rmax, d, 32, 32, 64)) return SWF_ERR_LAUNCH;
+    if (!encode_tmap_bf16(&em.o[0], w.dxc, d, sd.rmax, d, 64, 32, 128)) return SWF_ERR_LAUNCH;  // 32 x 64 boxes
     s = launch_tc<256, false, true, false, kEpiStore, kModeRowGrouped, true>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st, em);
     if (s != SWF_OK) return s;
   }

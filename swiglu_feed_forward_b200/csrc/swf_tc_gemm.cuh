@@ -153,12 +153,20 @@ template <bool PAIR>
 constexpr int tma_epi_out_bufs() {
   return PAIR ? 1 : 2;
 }
+// Columns of one output staging box (rows: 32, one per lane).  The plain-store epilogue of the
+// row-grouped sparse GEMMs moves 64 columns per chunk through 32 x 64 boxes (128-byte swizzle):
+// their K is one or two k-blocks, so each tile is mostly epilogue and half the chunks means half
+// the TMEM-load waits, proxy fences and TMA stores.  The others keep 32 x 32 boxes (64-byte
+// swizzle), which their register budget needs.
+template <int EPI>
+constexpr int tma_epi_cols() {
+  return EPI == kEpiStore ? 64 : 32;
+}
 template <int EPI, bool TMA_EPI, bool PAIR>
 constexpr int epi_smem_bytes() {
   return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
-                               : (TMA_EPI ? 4 * (tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>() +
-                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>()) *
-                                                kEpiBox
+                               : (TMA_EPI ? 4 * (tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>() * 64 * tma_epi_cols<EPI>() +
+                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>() * kEpiBox)
                                           : 0);
 }
 
@@ -549,13 +557,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int NAUX = tma_epi_aux<EPI>();
     constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
     constexpr bool kDual = kGLU;  // [g | u] accumulator halves
-    constexpr int NCH = (kDual ? BN / 2 : BN) / 32;
+    constexpr int CWO = tma_epi_cols<EPI>();  // output columns per chunk
+    static_assert(CWO == 32 || (CWO == 64 && !kDual && NAUX == 0 && NOUT == 1), "64-column chunks");
+    constexpr int kOutBox = 64 * CWO;         // bytes of one 32-row output box
+    constexpr int NCH = (kDual ? BN / 2 : BN) / CWO;
+    static_assert((kDual ? BN / 2 : BN) % CWO == 0, "whole chunks");
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
     constexpr int AB = tma_epi_aux_bufs<EPI>();
     constexpr int OB = tma_epi_out_bufs<PAIR>();
-    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT + AB * NAUX) * kEpiBox;  // boxes [NOUT][OB]
-    uint8_t* abase = ebase + OB * NOUT * kEpiBox;  // aux buffers [AB][NAUX]
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT * kOutBox + AB * NAUX * kEpiBox);  // boxes [NOUT][OB]
+    uint8_t* abase = ebase + OB * NOUT * kOutBox;  // aux buffers [AB][NAUX]
     uint64_t* abar = auxbar + ew * AB;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this lane's staging row
@@ -610,20 +622,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ++aux_done;
           aux = abase + (db * NAUX) * kEpiBox;
         }
-        float v0[32], v1[32];
+        float v0[32], v1[32];  // kDual: g | u columns; 64-column chunks: the chunk's two halves
         if (have_acc) {
-          tmem_ld32(t_acc + c * 32, v0);
+          tmem_ld32(t_acc + c * CWO, v0);
           if constexpr (kDual) tmem_ld32(t_acc + BN / 2 + c * 32, v1);
+          else if constexpr (CWO == 64) tmem_ld32(t_acc + c * CWO + 32, v1);
           tmem_ld_wait_regs(v0);
-          if constexpr (kDual) pin_regs(v1);
+          if constexpr (kDual || CWO == 64) pin_regs(v1);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0.f;
         }
-        uint32_t w[NOUT][16];
+        uint32_t w[NOUT][CWO / 2];
         if constexpr (EPI == kEpiStore) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[0][i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+          for (int i = 0; i < 16; ++i) {
+            w[0][i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+            w[0][16 + i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
+          }
         } else if constexpr (kGLU) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -688,25 +704,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
 #pragma unroll
         for (int o = 0; o < NOUT; ++o) {
-          uint8_t* ob = ebase + (o * OB + db) * kEpiBox;
+          uint8_t* ob = ebase + (o * OB + db) * kOutBox;
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            *reinterpret_cast<uint4*>(ob + lane * 64 + ((c4 ^ swz) * 16)) =
+          for (int c4 = 0; c4 < CWO / 8; ++c4) {  // 16-byte pieces of this lane's row, swizzled
+            const int phys = CWO == 64 ? (c4 ^ (lane & 7)) : (c4 ^ swz);
+            *reinterpret_cast<uint4*>(ob + lane * (2 * CWO) + phys * 16) =
                 make_uint4(w[o][c4 * 4], w[o][c4 * 4 + 1], w[o][c4 * 4 + 2], w[o][c4 * 4 + 3]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
-        const int n0 = n_base + c * 32;
+        const int n0 = n_base + c * CWO;
         // A box that starts inside its tensor is clipped by TMA at the far edges; boxes that
         // start past the last row or column are not issued at all.
         if (lane == 0 && m_slab < args.M && n0 < args.N) {
           if constexpr (EPI == kEpiStore) {
-            if (m_slab < args.row_split) tma_store_2d(&emaps.o[0], n0, m_slab, ebase + db * kEpiBox);
-            else tma_store_2d(&emaps.o[1], n0, m_slab - args.row_split, ebase + db * kEpiBox);
+            if (m_slab < args.row_split) tma_store_2d(&emaps.o[0], n0, m_slab, ebase + db * kOutBox);
+            else tma_store_2d(&emaps.o[1], n0, m_slab - args.row_split, ebase + db * kOutBox);
           } else {
 #pragma unroll
             for (int o = 0; o < NOUT; ++o)
-              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * OB + db) * kEpiBox);
+              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * OB + db) * kOutBox);
           }
           bulk_commit();
         }
