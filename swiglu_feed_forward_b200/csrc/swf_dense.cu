@@ -19,8 +19,11 @@ namespace swf {
 
 namespace {
 // 32 x 32 box with 64-byte swizzle: the staging box of the TMA epilogue.
-bool epi_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t row_elems) {
-  return encode_tmap_bf16(m, base, cols, rows, row_elems, 32, 32, 64);
+// Tensor map of a TMA epilogue's output or factor plane: 32-row boxes of 32 columns (64-byte
+// swizzle) or 64 columns (128-byte swizzle), as the epilogue's staging boxes are laid out.
+bool epi_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t row_elems,
+             int box_cols = 32) {
+  return encode_tmap_bf16(m, base, cols, rows, row_elems, box_cols, 32, box_cols == 64 ? 128 : 64);
 }
 
 // out[m, n] = bf16(sum over splits s = 0, 1, ... of part[s][m][n]) in that fixed order; rows at
@@ -296,7 +299,9 @@ swf_status mlp2_fwd_bf16(const void* x, const void* wu, const void* wd, void* y,
     return SWF_ERR_LAUNCH;
   // post and act_grad leave through TMA stores (K = d_model is short, the epilogue dominates)
   EpiMaps e1{};
-  if (!epi_map(&e1.o[0], post, f, M, f) || !epi_map(&e1.o[1], act_grad, f, M, f)) return SWF_ERR_LAUNCH;
+  if (!epi_map(&e1.o[0], post, f, M, f, tma_epi_cols<kEpiLeakySq>()) ||
+      !epi_map(&e1.o[1], act_grad, f, M, f, tma_epi_cols<kEpiLeakySq>()))
+    return SWF_ERR_LAUNCH;
   TcGemmArgs u1 = base_args(M, f, 256, d, 2 * kTileM);
   swf_status s = launch_tc_pair<256, false, false, false, kEpiLeakySq, true>(SWF_K_MLP2_UP, tx, twu, twu, e1, u1, st);
   if (s != SWF_OK) return s;
