@@ -319,7 +319,8 @@ swf_status mlp2_bwd_bf16(const void* dy, const void* x, const void* wu, const vo
     CUtensorMap tdy, twd;
     EpiMaps e{};
     if (!encode_tmap_bf16(&tdy, dy, d, M, d, 64, 128) || !encode_tmap_bf16(&twd, wd, f, d, f, 64, 64) ||
-        !epi_map(&e.o[0], dpre, f, M, f) || !epi_map(&e.o[2], act_grad, f, M, f))
+        !epi_map(&e.o[0], dpre, f, M, f, tma_epi_cols<kEpiScale>()) ||
+        !epi_map(&e.o[2], act_grad, f, M, f, tma_epi_cols<kEpiScale>()))
       return SWF_ERR_LAUNCH;
     TcGemmArgs u3 = base_args(M, f, 256, d, 2 * kTileM);
     s = launch_tc_pair<256, false, true, false, kEpiScale, true>(SWF_K_MLP2_DPRE, tdy, twd, twd, e, u3, st);

@@ -143,30 +143,30 @@ constexpr int tma_epi_aux() {
 }
 constexpr int kEpiAuxMap = 2;  // first tensor map of the factors a TMA epilogue loads
 // Buffers per epilogue warp for the factor boxes a TMA epilogue loads: kEpiScale's short-K tiles
-// (the activation gradient of a 512-deep product) prefetch three 32-column chunks ahead.
+// (the activation gradient of a 512-deep product) prefetch two 64-column chunks ahead.
 template <int EPI>
 constexpr int tma_epi_aux_bufs() {
-  return EPI == kEpiScale ? 4 : 2;
+  return EPI == kEpiScale ? 3 : 2;
 }
-constexpr int kEpiBox = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
 template <bool PAIR>
 constexpr int tma_epi_out_bufs() {
   return PAIR ? 1 : 2;
 }
-// Columns of one output staging box (rows: 32, one per lane).  The plain-store epilogue of the
-// row-grouped sparse GEMMs and the LeakyReLU^2 epilogue move 64 columns per chunk through
-// 32 x 64 boxes (128-byte swizzle): their K is one, two or eight k-blocks, so each tile is mostly
-// epilogue, and half the chunks means half the TMEM-load waits, proxy fences and TMA stores
-// (sparse down 84 -> 62 us on B200).  The others keep 32 x 32 boxes (64-byte swizzle).
+// Columns of one output (and factor) staging box (rows: 32, one per lane).  The plain-store
+// epilogue of the row-grouped sparse GEMMs and the LeakyReLU^2 up / activation-gradient
+// epilogues move 64 columns per chunk through 32 x 64 boxes (128-byte swizzle): their K is one,
+// two or eight k-blocks, so each tile is mostly epilogue, and half the chunks means half the
+// TMEM-load waits, proxy fences and TMA copies (sparse down 84 -> 62 us, LeakyReLU^2 up 186 ->
+// 167 us on B200).  The others keep 32 x 32 boxes (64-byte swizzle).
 template <int EPI>
 constexpr int tma_epi_cols() {
-  return (EPI == kEpiStore || EPI == kEpiLeakySq) ? 64 : 32;
+  return (EPI == kEpiStore || EPI == kEpiLeakySq || EPI == kEpiScale) ? 64 : 32;
 }
 template <int EPI, bool TMA_EPI, bool PAIR>
 constexpr int epi_smem_bytes() {
   return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
                                : (TMA_EPI ? 4 * (tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>() * 64 * tma_epi_cols<EPI>() +
-                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>() * kEpiBox)
+                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>() * 64 * tma_epi_cols<EPI>())
                                           : 0);
 }
 
@@ -558,15 +558,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
     constexpr bool kDual = kGLU;  // [g | u] accumulator halves
     constexpr int CWO = tma_epi_cols<EPI>();  // output columns per chunk
-    static_assert(CWO == 32 || (CWO == 64 && !kDual && NAUX == 0), "64-column chunks");
-    constexpr int kOutBox = 64 * CWO;         // bytes of one 32-row output box
+    static_assert(CWO == 32 || (CWO == 64 && !kDual && NAUX <= 1), "64-column chunks");
+    constexpr int kOutBox = 64 * CWO;         // bytes of one 32-row output (or factor) box
     constexpr int NCH = (kDual ? BN / 2 : BN) / CWO;
     static_assert((kDual ? BN / 2 : BN) % CWO == 0, "whole chunks");
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int ew = warp - 2;
     constexpr int AB = tma_epi_aux_bufs<EPI>();
     constexpr int OB = tma_epi_out_bufs<PAIR>();
-    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT * kOutBox + AB * NAUX * kEpiBox);  // boxes [NOUT][OB]
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT + AB * NAUX) * kOutBox;  // boxes [NOUT][OB]
     uint8_t* abase = ebase + OB * NOUT * kOutBox;  // aux buffers [AB][NAUX]
     uint64_t* abar = auxbar + ew * AB;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
@@ -587,11 +587,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if constexpr (NAUX > 0) {
           if (lane == 0) {
             const int db = aux_issued % AB;
-            mbar_arrive_expect_tx(&abar[db], NAUX * kEpiBox);
-            tma_load_2d(abase + (db * NAUX) * kEpiBox, &emaps.o[kEpiAuxMap], n_base + c * 32, m_slab,
+            mbar_arrive_expect_tx(&abar[db], NAUX * kOutBox);
+            tma_load_2d(abase + (db * NAUX) * kOutBox, &emaps.o[kEpiAuxMap], n_base + c * CWO, m_slab,
                         &abar[db]);
             if constexpr (NAUX > 1)
-              tma_load_2d(abase + (db * NAUX + 1) * kEpiBox, &emaps.o[3], n_base + c * 32, m_slab, &abar[db]);
+              tma_load_2d(abase + (db * NAUX + 1) * kOutBox, &emaps.o[3], n_base + c * CWO, m_slab, &abar[db]);
           }
           ++aux_issued;
         }
@@ -620,7 +620,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           ++aux_done;
-          aux = abase + (db * NAUX) * kEpiBox;
+          aux = abase + (db * NAUX) * kOutBox;
         }
         float v0[32], v1[32];  // kDual: g | u columns; 64-column chunks: the chunk's two halves
         if (have_acc) {
@@ -675,20 +675,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         } else if constexpr (EPI == kEpiScale) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 av = *reinterpret_cast<const uint4*>(aux + lane * 64 + ((c4 ^ swz) * 16));
+          for (int c4 = 0; c4 < CWO / 8; ++c4) {  // 16-byte pieces of the factor row
+            const int phys = CWO == 64 ? (c4 ^ (lane & 7)) : (c4 ^ swz);
+            const uint4 av = *reinterpret_cast<const uint4*>(aux + lane * (2 * CWO) + phys * 16);
             const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+            const float* vh = c4 < 4 ? v0 : v1;  // resolved at compile time (unrolled)
 #pragma unroll
             for (int p = 0; p < 4; ++p)
-              w[0][c4 * 4 + p] = pack_bf16x2(v0[c4 * 8 + p * 2] * bf16_lo(aw[p]),
-                                             v0[c4 * 8 + p * 2 + 1] * bf16_hi(aw[p]));
+              w[0][c4 * 4 + p] = pack_bf16x2(vh[(c4 & 3) * 8 + p * 2] * bf16_lo(aw[p]),
+                                             vh[(c4 & 3) * 8 + p * 2 + 1] * bf16_hi(aw[p]));
           }
         } else if constexpr (EPI == kEpiDGate) {
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
             const int off = lane * 64 + ((c4 ^ swz) * 16);
             const uint4 av = *reinterpret_cast<const uint4*>(aux + off);
-            const uint4 bv = *reinterpret_cast<const uint4*>(aux + kEpiBox + off);
+            const uint4 bv = *reinterpret_cast<const uint4*>(aux + kOutBox + off);
             const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
