@@ -47,6 +47,7 @@ KERNEL_FLOP_UNITS = {"gate_up_swiglu": 4, "gate_up_swiglu_infer": 4, "down_proj"
                      "dx": 4, "dw_gate_up": 4, "dw_down": 2}
 KERNEL_SOURCES = ["swiglu_feed_forward_b200/csrc/swf_tc_gemm.cuh",
                   "swiglu_feed_forward_b200/csrc/swf_ptx.cuh",
+                  "swiglu_feed_forward_b200/csrc/swf_launch.cuh",
                   "swiglu_feed_forward_b200/csrc/swf_dense.cu"]
 
 
@@ -63,11 +64,35 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha():
+def code_lines(text):
+    """The lines of a C++/CUDA source with // comments, trailing blanks and empty lines removed
+    (string literals kept whole), so that edits to comments alone leave its hash unchanged."""
+    out = []
+    for line in text.splitlines():
+        in_str, cut = False, len(line)
+        for i, ch in enumerate(line):
+            if ch == '"' and (i == 0 or line[i - 1] != "\\"):
+                in_str = not in_str
+            elif not in_str and line.startswith("//", i):
+                cut = i
+                break
+        code = line[:cut].rstrip()
+        if code:
+            out.append(code)
+    return out
+
+
+def source_sha(read=None):
+    """Hash of the code (comments aside) of the sources the dense kernels are built from; the
+    ncu traffic figures are valid while it is unchanged.  `read(rel)` overrides file reading."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as fh:
-            h.update(fh.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel)) as fh:
+                text = fh.read()
+        else:
+            text = read(rel)
+        h.update("\n".join(code_lines(text)).encode())
     return h.hexdigest()[:16]
 
 

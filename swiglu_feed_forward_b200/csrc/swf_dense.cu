@@ -18,7 +18,6 @@
 namespace swf {
 
 namespace {
-// 32 x 32 box with 64-byte swizzle: the staging box of the TMA epilogue.
 // Tensor map of a TMA epilogue's output or factor plane: 32-row boxes of 32 columns (64-byte
 // swizzle) or 64 columns (128-byte swizzle), as the epilogue's staging boxes are laid out.
 bool epi_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t row_elems,

@@ -125,8 +125,8 @@ struct TcGemmArgs {
 };
 
 // Epilogues that move their tiles with TMA: bf16 outputs staged per warp in shared memory
-// (32 x 32 boxes, 64-byte swizzle) and, for kEpiDGate, the a/b factor tiles loaded by TMA into
-// the same kind of buffers.  Pair-mode (dense) kernels keep one box per output, which a warp
+// (32-row boxes, 32 or 64 columns wide: see tma_epi_cols) and, for kEpiDGate and kEpiScale,
+// the factor tiles loaded by TMA into the same kind of buffers.  Pair-mode (dense) kernels keep one box per output, which a warp
 // overwrites once the previous chunk's store has read it (the chunk's TMEM load and arithmetic
 // cover that); this leaves the gate|up kernel its six ring stages.  Measured with a %clock64
 // probe of the MMA issuer on B200, its k-blocks then take about 605 cycles, against about 690
@@ -701,7 +701,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        // stage this warp's 32 x 32 box of every output, then one lane stores them with TMA
+        // stage this warp's 32-row box of every output, then one lane stores them with TMA
         const int db = OB > 1 ? static_cast<int>(chunks & 1u) : 0;
         if (lane == 0) bulk_wait_read<OB - 1>();  // the store that last used box db has read it
         __syncwarp();
