@@ -19,6 +19,11 @@ namespace swf {
 namespace {
 
 constexpr int kBucketSmemBytes = 98304;
+// The plain-store TMA epilogue's staging boxes: 32 rows x kStoreBoxCols columns, swizzled by
+// the width in bytes (the tensor maps of its outputs must match them).
+constexpr int kStoreBoxCols = tma_epi_cols<kEpiStore>();
+constexpr int kStoreBoxSwizzle = kStoreBoxCols * 2;
+static_assert(kStoreBoxSwizzle == 64 || kStoreBoxSwizzle == 128, "box row = swizzle span");
 
 struct SparseDims {
   int64_t M, d, f;
@@ -806,7 +811,7 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 256))
       return SWF_ERR_LAUNCH;
     EpiMaps em{};
-    if (!encode_tmap_bf16(&em.o[0], w.yc, d, sd.rmax, d, 64, 32, 128)) return SWF_ERR_LAUNCH;  // 32 x 64 boxes
+    if (!encode_tmap_bf16(&em.o[0], w.yc, d, sd.rmax, d, kStoreBoxCols, 32, kStoreBoxSwizzle)) return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, d, 256, G);
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
@@ -869,7 +874,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.tile_group = v.tile_group;
     a.grp_b_k = G;
     EpiMaps em{};
-    if (!encode_tmap_bf16(&em.o[0], w.dxc, d, sd.rmax, d, 64, 32, 128)) return SWF_ERR_LAUNCH;  // 32 x 64 boxes
+    if (!encode_tmap_bf16(&em.o[0], w.dxc, d, sd.rmax, d, kStoreBoxCols, 32, kStoreBoxSwizzle)) return SWF_ERR_LAUNCH;
     s = launch_tc<256, false, true, false, kEpiStore, kModeRowGrouped, true>(SWF_K_SPARSE_DX, tdgu, twg, twu, a, st, em);
     if (s != SWF_OK) return s;
   }
