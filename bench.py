@@ -64,6 +64,37 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The B200's dense bf16 tensor-core rate: 2.25 PFLOP/s nominal (NVIDIA's 4.5 PFLOP/s is the 2:4
+# sparse figure), i.e. 8192 FLOP per SM per clock (148 SMs at about 1.855 GHz).
+NOMINAL_BF16_TFLOPS = 2250.0
+NUM_SMS = 148
+BF16_FLOP_PER_SM_CLOCK = 8192.0
+# A timed region shorter than this runs at burst clocks: its kernels are held against the burst
+# peak (the sustained one describes seconds of back-to-back GEMMs under the power cap).
+SUSTAINED_AFTER_S = 3.0
+
+
+def choose_peak(region_s, peak_burst, peak_sus, src):
+    """The bf16 peak a kernel timed inside a region of region_s seconds is held against."""
+    if region_s >= SUSTAINED_AFTER_S:
+        return peak_sus, f"{src} bf16 sustained (timed region {region_s:.2f} s >= {SUSTAINED_AFTER_S} s)"
+    return peak_burst, f"{src} bf16 burst (timed region {region_s:.2f} s < {SUSTAINED_AFTER_S} s)"
+
+
+def pct_of_peak(tflops, peak_burst, peak_sus, src, clk):
+    """The step's rate as a percentage of each bf16 peak: the measured burst and sustained
+    cuBLAS figures, the nominal 2.25 PFLOP/s, and the tensor cores' rate at the SM clock
+    sampled during the timed region (148 SMs x 8192 FLOP per clock)."""
+    out = {"burst": round(100 * tflops / peak_burst, 2), "sustained": round(100 * tflops / peak_sus, 2),
+           "nominal": round(100 * tflops / NOMINAL_BF16_TFLOPS, 2), "source": src,
+           "nominal_tflops": NOMINAL_BF16_TFLOPS}
+    if clk and clk.get("sm_mhz"):
+        at_clock = NUM_SMS * BF16_FLOP_PER_SM_CLOCK * clk["sm_mhz"] * 1e6 / 1e12
+        out["at_sampled_clock"] = round(100 * tflops / at_clock, 2)
+        out["at_sampled_clock_tflops"] = round(at_clock, 1)
+    return out
+
+
 def code_lines(text):
     """The lines of a C++/CUDA source with // comments, trailing blanks and empty lines removed
     (string literals kept whole), so that edits to comments alone leave its hash unchanged."""
@@ -82,11 +113,12 @@ def code_lines(text):
     return out
 
 
-def source_sha(read=None):
-    """Hash of the code (comments aside) of the sources the dense kernels are built from; the
-    ncu traffic figures are valid while it is unchanged.  `read(rel)` overrides file reading."""
+def source_sha(read=None, files=None):
+    """Hash of the code (comments aside) of the sources the dense kernels (or `files`) are built
+    from; the ncu traffic figures are valid while it is unchanged.  `read(rel)` overrides file
+    reading."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in (files or KERNEL_SOURCES):
         if read is None:
             with open(os.path.join(ROOT, rel)) as fh:
                 text = fh.read()
@@ -111,27 +143,78 @@ def ncu_traffic(kernel):
 
 
 # ------------------------------------------------------------------ clocks
+def parse_smi_time(text):
+    """nvidia-smi's local timestamp ("2026/12/02 16:15:00.123") as seconds since the epoch."""
+    import datetime
+    for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+        try:
+            return datetime.datetime.strptime(text.strip(), fmt).timestamp()
+        except ValueError:
+            continue
+    return None
+
+
+def summarize_clocks(rows, t0=None, t1=None):
+    """Median SM clock, max power and the throttle reasons seen in the samples whose timestamp
+    lies in [t0, t1] (the timed region), or in all samples when no window is given."""
+    if t0 is not None:
+        inside = [r for r in rows if r["ts"] is not None and t0 <= r["ts"] <= t1]
+    else:
+        inside = list(rows)
+    if not inside:
+        return None
+    sms = sorted(r["sm"] for r in inside)
+    reasons = set()
+    for r in inside:
+        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                          ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+            if r[key].lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": inside[0]["smax"],
+            "power_w_max": max(r["power"] for r in inside), "samples": len(inside),
+            "reasons": sorted(reasons)}
+
+
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 20 ms in the background; stop() keeps only the samples taken
+    inside the window mark_start() .. mark_end() (the timed region)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, interval_ms=20):
         self.proc = None
         self.path = None
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
+        self.t0 = self.t1 = None
 
-    def start(self):
+    def start(self, wait_first_s=3.0):
+        """Starts nvidia-smi and waits (bounded) until it has written its first sample, so
+        that the timed region that follows is covered from its start."""
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        deadline = time.time() + wait_first_s
+        while time.time() < deadline and self.proc.poll() is None:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
@@ -146,26 +229,26 @@ class ClockSampler:
         with open(self.path) as fh:
             for line in fh:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                     hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                    rows.append(dict(ts=parse_smi_time(parts[0]), sm=float(parts[2]), smax=float(parts[3]),
+                                     power=float(parts[4]), hw=parts[6], hwt=parts[7], swt=parts[8],
+                                     swp=parts[9]))
                 except ValueError:
                     continue
         os.unlink(self.path)
         if not rows:
             return None
-        sms = sorted(r["sm"] for r in rows)
-        reasons = set()
-        for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
-                if r[key].lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": rows[0]["smax"],
-                "power_w_max": max(r["power"] for r in rows), "samples": len(rows),
-                "reasons": sorted(reasons)}
+        # nvidia-smi stamps to the millisecond; allow one sampling interval of slack each side
+        slack = self.interval_ms / 1e3
+        out = summarize_clocks(rows, self.t0 - slack, self.t1 + slack) if self.t0 is not None else None
+        if out is None:  # no sample fell inside the region: report all, flagged
+            out = summarize_clocks(rows)
+            out["window"] = "no sample inside the timed region; all samples of the run"
+        else:
+            out["window"] = "samples inside the timed region only"
+        return out
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -226,6 +309,53 @@ def oracle_sample_time(tokens, min_seconds=10.0, max_seconds=30.0):
             f"{w['M']} tokens (d_model {w['d_model']}, d_ff {w['d_ff']}), {reps} pass(es), "
             f"{el:.1f} s")
     return flops / el / 1e12, int(threads), desc, reps, el
+
+
+def selection_check(idx_gpu, tie_rel=1e-3):
+    """The GPU's group indices at workload 3 against the fp64 oracle's top-k on all M tokens:
+    rows whose chosen set differs, rows whose K-th and (K+1)-th oracle scores lie within
+    tie_rel (relative) of each other, and differing rows outside those near-ties (which must
+    be none)."""
+    import numpy as np
+
+    import oracle as O
+    w = synth.WORKLOADS[3]
+    M, f, G, K, spg = (w[k] for k in ("M", "d_ff", "group_size", "num_active_groups", "samples_per_group"))
+    inp = synth.workload_inputs(3, with_dy=False)
+    x, wg = (inp[k].to(torch.float64).numpy() for k in ("x", "w_gate"))
+    sub = O.make_subsample_index(f, G, spg, w["seed"])
+    bias = synth.balance_bias(f // G, w["seed"]).to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    E_ref = O.group_energy(x, wg, G, sub, bias)
+    ref = O.topk_groups(E_ref, K)
+    gap = O.topk_gap(E_ref, K)
+    idx = np.sort(idx_gpu.numpy(), axis=1)
+    differ = ~np.all(idx == ref, axis=1)
+    ties = gap < tie_rel
+    return {"tokens": int(M), "rows_differing": int(differ.sum()), "near_tie_rows": int(ties.sum()),
+            "rows_differing_outside_near_ties": int((differ & ~ties).sum()), "tie_rel": tie_rel,
+            "checker": "fp64 numpy oracle group_energy + topk_groups on the same bf16 inputs",
+            "seconds": round(time.perf_counter() - t0, 2)}
+
+
+SPARSE_SOURCES = ["swiglu_feed_forward_b200/csrc/swf_tc_gemm.cuh",
+                  "swiglu_feed_forward_b200/csrc/swf_ptx.cuh",
+                  "swiglu_feed_forward_b200/csrc/swf_launch.cuh",
+                  "swiglu_feed_forward_b200/csrc/swf_sparse.cu"]
+
+
+def ncu_sparse_traffic():
+    """DRAM bytes of one group-sparse step summed over its kernels' one-kernel ncu captures
+    (committed under profiles/), or None when absent or taken on other sparse sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    e = d.get("group_sparse_step")
+    if not e or e.get("source_sha") != source_sha(files=SPARSE_SOURCES):
+        return None
+    return {"dram_bytes_per_step": e["dram_bytes_per_step"], "from": e["from"]}
 
 
 def run_reference(args, world, rank):
@@ -332,12 +462,26 @@ def secondary_infer(api, steps, warmup, world):
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
-def sparse_step_hbm_bytes(M, d, f, G, K, spg, R):
-    """HBM bytes the group-sparse step's kernels must move in this design (bf16 data, int32
+def sparse_step_algorithmic_bytes(M, d, f, G, K, spg):
+    """The least HBM traffic of one group-sparse step (selection + forward + backward, bf16
+    tensors, int32 indices): every input read once and every output written once.
+    selection: x, the sampled gate rows, the chosen groups; forward: x, the three weights, the
+    chosen groups, y, and the per-pair h, a, b kept for the backward; backward: dY, x, the three
+    weights, h, a, b, the chosen groups, dx and the three weight gradients."""
+    b, ng = 2, f // G
+    select = b * M * d + b * ng * spg * d + 4 * M * K
+    fwd = 2 * b * M * d + 3 * b * f * d + 4 * M * K + 3 * b * M * K * G
+    bwd = 3 * b * M * d + 6 * b * f * d + 4 * M * K + 3 * b * M * K * G
+    return select + fwd + bwd
+
+
+def sparse_step_design_bytes(M, d, f, G, K, spg, R):
+    """HBM bytes the group-sparse step's kernels move in this design (bf16 data, int32
     indices), with R the padded pair rows: selection (x, the sampled gate rows, the chosen
     groups), the gathers (x and dY rows written group-major; the token rows come from L2), the
     row-grouped GEMMs (gathered rows, the group's weights, h, a, b, [dG | dU]), the per-pair y and
-    dx contributions written and summed, and the grouped weight gradients."""
+    dx contributions written and summed, and the grouped weight gradients.  The [dG | dU] rows
+    are 128 columns wide for every group size (each half padded to 64 columns)."""
     b, ng = 2, f // G
     P = 1 << max(0, (spg - 1).bit_length())
     select = b * M * d + b * ng * P * d + 4 * M * K
@@ -352,12 +496,15 @@ def sparse_step_hbm_bytes(M, d, f, G, K, spg, R):
     return select + buckets + 2 * gather + up + down + 2 * pair_sum + dgate + dxg + dw
 
 
-def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
+def secondary_sparse(api, steps, warmup, world, peaks, skewed=False):
+    """Selection + sparse forward + sparse backward at workload 3.  Returns the line and the
+    selected group indices (host copy) for the CPU leg's check against the oracle."""
+    peak_burst, peak_sus = peaks
     w = synth.WORKLOADS[3]
     M, d, f, G, K, spg = (w[k] for k in ("M", "d_model", "d_ff", "group_size", "num_active_groups",
                                           "samples_per_group"))
     if api.supported("sparse_fwd", M, d, f, G, K, spg) != 0:
-        return {"workload": w["name"], "unavailable": "sparse path not supported for this shape"}
+        return {"workload": w["name"], "unavailable": "sparse path not supported for this shape"}, None
     dev = torch.device("cuda")
     inp = synth.workload_inputs(3)
     t = {k: v.to(dev) for k, v in inp.items()}
@@ -384,6 +531,11 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     for _ in range(warmup):
         fn()
     ms = timed(fn, steps, world)
+    # per-kernel split from the library's event hooks, in a separate pass (the hooks add events)
+    api.profile_enable(True)
+    timed(fn, steps, world)
+    kern = api.profile_read()
+    api.profile_enable(False)
     # the same step as one CUDA graph: about 20 short launches, so launch gaps show
     g = graph_of(fn)
     for _ in range(warmup):
@@ -391,28 +543,57 @@ def secondary_sparse(api, steps, warmup, world, peak, skewed=False):
     ms_graph = timed(g.replay, steps, world)
     useful = 2.0 * M * d * ng * spg + 18.0 * M * d * K * G
     tf = useful * steps / (ms / 1e3) / 1e12
+    tf_graph = useful * steps / (ms_graph / 1e3) / 1e12
     per_group = torch.bincount(idx.flatten().long(), minlength=ng)
     R = int(((per_group + 127) // 128 * 128).sum())
-    hbm_bytes = sparse_step_hbm_bytes(M, d, f, G, K, spg, R)
+    alg_bytes = sparse_step_algorithmic_bytes(M, d, f, G, K, spg)
+    design_bytes = sparse_step_design_bytes(M, d, f, G, K, spg, R)
     hbm_peak = float(load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    hbm_gbs = hbm_bytes / (ms_graph / steps / 1e3) / 1e9
-    return {"workload": w["name"] + (" (skewed bias: +0.5 on 2 groups, -0.5 on 2)" if skewed else ""),
+    step_s = ms_graph / steps / 1e3
+    # The step's roofline is the larger of its two algorithmic times (useful FLOPs at the bf16
+    # peak, least bytes at the HBM peak); at this workload that is the FLOPs.
+    t_flops, t_bytes = useful / (peak_burst * 1e12), alg_bytes / (hbm_peak * 1e9)
+    measured = ncu_sparse_traffic()
+    bound = "tensor" if t_flops >= t_bytes else "hbm"
+    roof = {"bound": bound,
+            "achieved": round(tf_graph * world, 2) if bound == "tensor" else round(alg_bytes / step_s / 1e9 * world, 1),
+            "peak": peak_burst if bound == "tensor" else hbm_peak,
+            "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+            "frac": round((t_flops if bound == "tensor" else t_bytes) / step_s, 4),
+            "peak_kind": "measured bf16 burst" if bound == "tensor" else "measured HBM copy",
+            "frac_useful_flops_of_burst": round(t_flops / step_s, 4),
+            "frac_algorithmic_bytes_of_hbm": round(t_bytes / step_s, 4),
+            "algorithmic_bytes_per_step": alg_bytes,
+            "traffic": measured["dram_bytes_per_step"] if measured else None,
+            "traffic_basis": measured["from"] if measured else
+                             "none: no per-kernel ncu capture of the current sparse sources",
+            "design_bytes_per_step": design_bytes, "padded_pair_rows": R,
+            "basis": "CUDA-graph step time; useful FLOPs 2 M d ng spg + 18 M d K G; least bytes "
+                     "sparse_step_algorithmic_bytes"}
+    if measured:
+        roof["traffic_over_algorithmic"] = round(measured["dram_bytes_per_step"] / alg_bytes, 2)
+    total_k = sum(v for _, v in kern.values()) or 1.0
+    kernels = {k: {"launches_per_step": round(n / steps, 2), "us_per_step": round(v / steps * 1e3, 1),
+                   "share": round(v / total_k, 4)}
+               for k, (n, v) in sorted(kern.items(), key=lambda kv: -kv[1][1])}
+    line = {"workload": w["name"] + (" (skewed bias: +0.5 on 2 groups, -0.5 on 2)" if skewed else ""),
             "useful_tflops": round(tf * world, 3),
-            "pct_of_peak": round(100 * tf / peak, 2), "ms_per_step": round(ms / steps, 3),
+            "pct_of_peak": {"burst": round(100 * tf / peak_burst, 2), "sustained": round(100 * tf / peak_sus, 2)},
+            "ms_per_step": round(ms / steps, 3),
             "steps": steps, "useful_flops_per_step": useful,
             "cuda_graph": {"ms_per_step": round(ms_graph / steps, 3),
-                           "useful_tflops": round(useful * steps / (ms_graph / 1e3) / 1e12 * world, 3)},
+                           "useful_tflops": round(tf_graph * world, 3),
+                           "pct_of_burst_peak": round(100 * tf_graph / peak_burst, 2)},
             "tokens_per_group": {"max": int(per_group.max()), "mean": round(M * K / ng, 1),
                                  "min": int(per_group.min())},
-            "roofline": {"bound": "hbm", "achieved": round(hbm_gbs * world, 1), "peak": hbm_peak,
-                         "unit": "GB/s", "frac": round(hbm_gbs / hbm_peak, 4), "traffic": None,
-                         "bytes_per_step": hbm_bytes, "padded_pair_rows": R,
-                         "basis": "the step's design traffic (sparse_step_hbm_bytes) over the CUDA-graph "
-                                  "step time"}}
+            "kernels_eager": kernels,
+            "roofline": roof}
+    return line, idx.cpu()
 
 
-def secondary_mlp2(api, steps, warmup, world, peak):
+def secondary_mlp2(api, steps, warmup, world, peaks):
     """parameter-golf PR 1105's LeakyReLU(0.5)^2 MLP: fwd + bwd, 12 * M * d * hidden FLOPs."""
+    peak_burst, peak_sus = peaks
     w = synth.WORKLOADS[5]
     M, d, f = w["M"], w["d_model"], w["d_ff"]
     dev = torch.device("cuda")
@@ -430,12 +611,17 @@ def secondary_mlp2(api, steps, warmup, world, peak):
     ms = timed(fn, steps, world)
     flops = 12.0 * M * d * f
     tf = flops * steps / (ms / 1e3) / 1e12
-    return {"workload": w["name"], "tflops": round(tf * world, 2), "pct_of_peak": round(100 * tf / peak, 2),
+    return {"workload": w["name"], "tflops": round(tf * world, 2),
+            "pct_of_peak": {"burst": round(100 * tf / peak_burst, 2), "sustained": round(100 * tf / peak_sus, 2)},
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
-def secondary_mhffn(api, steps, warmup, world, peak):
-    """FlashFFN multi-head FFN forward (one fused kernel) at the 1.3B configuration."""
+def secondary_mhffn(api, steps, warmup, world, peaks):
+    """FlashFFN multi-head FFN forward (one fused kernel) at the 1.3B configuration, the block
+    from x, the core's backward and the block's whole training step.  FLOPs are algorithmic:
+    the core's forward 6 T H d_h E d_e, its backward 12 T H d_h E d_e (the recomputed S of the
+    fused backward is not counted as work)."""
+    peak_burst, peak_sus = peaks
     w = synth.WORKLOADS[6]
     T, H, dh, E, de = (w[k] for k in ("T", "H", "d_h", "E", "d_e"))
     dev = torch.device("cuda")
@@ -474,7 +660,7 @@ def secondary_mhffn(api, steps, warmup, world, peak):
     for _ in range(warmup):
         bwd()
     ms_bwd = timed(bwd, max(3, steps // 4), world)
-    flops_bwd = 16.0 * T * H * dh * E * de
+    flops_bwd = 12.0 * T * H * dh * E * de
     # the whole block's training step from x: prologue, fused core, core backward, prologue backward
     ws_p = torch.empty(max(16, api.flash_mhffn_prologue_bwd_workspace_bytes(T, d_model, H, dh, E)),
                        device=dev, dtype=torch.uint8)
@@ -493,7 +679,8 @@ def secondary_mhffn(api, steps, warmup, world, peak):
     ms_step = timed(step, n_step, world)
     flops_step = flops_b + flops_bwd + 2 * 2.0 * T * d_model * (H * dh + H * E)
     del ws, ws_p
-    return {"workload": w["name"], "tflops": round(tf * world, 1), "pct_of_peak": round(100 * tf / peak, 2),
+    return {"workload": w["name"], "tflops": round(tf * world, 1),
+            "pct_of_peak": {"burst": round(100 * tf / peak_burst, 2), "sustained": round(100 * tf / peak_sus, 2)},
             "ms_per_step": round(ms / steps, 3), "steps": steps, "flops_per_step": flops,
             "intermediate_bytes_not_written": 2 * T * H * E * de,
             "backward": {"ms_per_step": round(ms_bwd / max(3, steps // 4), 3), "flops_per_step": flops_bwd,
@@ -523,9 +710,10 @@ def run_ours(args, world, rank, local):
     # ---- timed region: device-resident inputs, per-kernel events on
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
     api.profile_enable(True)
+    clocks.mark_start()
     ms = timed(lambda: dense_step(api, t), args.steps, world)
+    clocks.mark_end()
     kern = api.profile_read()
     api.profile_enable(False)
     clk = clocks.stop()
@@ -543,16 +731,21 @@ def run_ours(args, world, rank, local):
     achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_kind = choose_peak(ms / 1e3, peak_burst, peak_sus, peak_src)
     roofline = {"kernel": dom_name, "bound": "tensor", "achieved": round(achieved, 2),
-                "peak": peak_sus, "unit": "TFLOP/s", "frac": round(achieved / peak_sus, 4),
-                "peak_kind": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_kind": peak_kind,
                 "frac_of_burst_peak": round(achieved / peak_burst, 4),
+                "frac_of_sustained_peak": round(achieved / peak_sus, 4),
                 "flops_per_launch": dom_flops, "launches": dom_n,
                 "avg_launch_ms": round(dom_ms / dom_n, 4),
+                "timed_region_s": round(ms / 1e3, 4),
                 "traffic": ncu_traffic(dom_name)}
     kernels = {k: {"launches": n, "ms_total": round(v, 3), "share": round(v / total_k, 4),
                    "avg_ms": round(v / n, 4),
-                   **({"tflops": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / n / 1e3) / 1e12, 1)}
+                   **({"tflops": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / n / 1e3) / 1e12, 1),
+                       "frac_of_burst_peak": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / n / 1e3) / 1e12
+                                                   / peak_burst, 4)}
                       if k in KERNEL_FLOP_UNITS else {})}
                for k, (n, v) in sorted(kern.items(), key=lambda kv: -kv[1][1])}
 
@@ -615,30 +808,33 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
 
     secondary = {}
+    sparse_idx = None
     if not args.no_secondary:
         try:
             secondary["inference_forward"] = secondary_infer(api, max(3, args.steps // 2), 3, world)
         except Exception as exc:  # report, never hide
             secondary["inference_forward"] = {"error": str(exc)[:200]}
         torch.cuda.empty_cache()
+        peaks_pair = (peak_burst, peak_sus)
         try:
-            secondary["group_sparse_step"] = secondary_sparse(api, max(3, args.steps // 2), 3, world, peak_sus)
+            secondary["group_sparse_step"], sparse_idx = secondary_sparse(api, max(3, args.steps // 2), 3, world,
+                                                                          peaks_pair)
         except Exception as exc:
             secondary["group_sparse_step"] = {"error": str(exc)[:200]}
         try:
-            secondary["group_sparse_step_skewed"] = secondary_sparse(api, max(3, args.steps // 2), 3, world,
-                                                                     peak_sus, skewed=True)
+            secondary["group_sparse_step_skewed"], _ = secondary_sparse(api, max(3, args.steps // 2), 3, world,
+                                                                        peaks_pair, skewed=True)
         except Exception as exc:  # reported, not fatal
             secondary["group_sparse_step_skewed"] = {"error": str(exc)[:200]}
         torch.cuda.empty_cache()
         try:
-            secondary["leaky_relu_sq_mlp_step"] = secondary_mlp2(api, max(3, args.steps // 2), 3, world, peak_sus)
+            secondary["leaky_relu_sq_mlp_step"] = secondary_mlp2(api, max(3, args.steps // 2), 3, world, peaks_pair)
         except Exception as exc:
             secondary["leaky_relu_sq_mlp_step"] = {"error": str(exc)[:200]}
         torch.cuda.empty_cache()
         try:
             secondary["flashffn_multihead_forward"] = secondary_mhffn(api, max(3, args.steps // 2), 3, world,
-                                                                      peak_sus)
+                                                                      peaks_pair)
         except Exception as exc:
             secondary["flashffn_multihead_forward"] = {"error": str(exc)[:200]}
 
@@ -647,6 +843,12 @@ def run_ours(args, world, rank, local):
         v, threads, desc, reps, el = oracle_sample_time(args.cpu_tokens)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc}
+        # the same leg checks the GPU's group selection against the oracle's on every token
+        if sparse_idx is not None and isinstance(secondary.get("group_sparse_step"), dict):
+            try:
+                secondary["group_sparse_step"]["selection_vs_oracle"] = selection_check(sparse_idx)
+            except Exception as exc:  # reported, not fatal
+                secondary["group_sparse_step"]["selection_vs_oracle"] = {"error": str(exc)[:200]}
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -657,9 +859,7 @@ def run_ours(args, world, rank, local):
                            "global_batch": 8 * world, "seq_len": 4096,
                            "flops_per_step": flops_step, "parallelism": "replicas",
                            "l2": "inputs larger than L2 (x, dY 134 MB each); no flush"},
-                "pct_of_peak": {"sustained": round(100 * value / world / peak_sus, 2),
-                                "burst": round(100 * value / world / peak_burst, 2),
-                                "source": peak_src},
+                "pct_of_peak": pct_of_peak(value / world, peak_burst, peak_sus, peak_src, clk),
                 "roofline": roofline, "kernels": kernels, "gpu_launches": gpu_launches,
                 "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "secondary": secondary}
         print(json.dumps(line), flush=True)

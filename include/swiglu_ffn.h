@@ -128,8 +128,8 @@ swf_status swiglu_ffn_bwd(const void* dy, const void* x, const void* w_gate, con
 /* Inference forward that allocates nothing and takes no workspace.  The pages have no
  * counterpart: it exists for callers that cannot provide device memory for the intermediate
  * h, such as a host program that reaches the library only through this ABI and has no device
- * allocator, a plug-in inside a runtime that forbids allocation on its execution path, or code
- * recording a stream capture in a mode where cudaMalloc is an error.  Computes the same y as
+ * allocator, or a plug-in inside a runtime that forbids allocation on its execution path.
+ * Computes the same y as
  * swiglu_ffn_fwd_infer, keeping h [M, d_ff] in a file-scope device array of
  * SWF_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the process exits.
  *  - Returns SWF_ERR_WORKSPACE, launching nothing, when M * d_ff * element size exceeds
@@ -271,7 +271,8 @@ swf_status grouped_topk_select(const void* x, const void* w_gate, const int32_t*
 /* Group-major bucketing of the (token, group) pairs (eugen_sparse README, "Pitfalls": the
  * CSR bucketing is deterministic).  offsets [num_groups + 1] int32 and tokens [M * K] int32:
  * tokens[offsets[c] .. offsets[c+1]) are the ids of the tokens whose group_idx row holds c, in
- * ascending order.  group_idx rows must hold distinct in-range groups (unchecked). */
+ * ascending order.  group_idx rows must hold distinct in-range groups: slots out of range or
+ * repeating an earlier slot of the row are dropped (checked only in debug mode, swf_set_debug). */
 swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t num_active_groups,
                              int32_t num_groups, int32_t* offsets, int32_t* tokens,
                              void* workspace, size_t workspace_bytes, void* stream);
@@ -321,6 +322,32 @@ swf_status swf_group_frequency(const int32_t* group_idx, int64_t M, int32_t num_
 swf_status update_load_balance_bias(float* bias, float* freq_ema, const float* current_freq,
                                     float target_freq, float gamma, float bias_max,
                                     float momentum, int32_t num_groups, void* stream);
+
+/* ------------------------------------------------------------------ group_idx checks */
+
+/* The eugen_sparse README ("Pitfalls and limitations") leaves group_idx unchecked: it must come
+ * from grouped_topk_select, and nothing validates the input beyond the shape rules.  This
+ * library's kernels never index out of bounds on a bad group_idx -- a slot whose group is out of
+ * [0, num_groups) or repeats an earlier slot of its row is dropped by the bucketing -- but the
+ * result then differs from what the caller meant.  These calls find such slots.
+ *
+ * swf_validate_group_idx counts the invalid slots of group_idx [M, num_active_groups] on
+ * `stream`, WAITS for the count (it synchronises the stream) and writes it to *bad_slots when
+ * non-null.  Returns SWF_OK when every slot is valid, SWF_ERR_INVALID_ARG when any is not; never
+ * traps.  Uses one device counter per GPU: concurrent validations on one device are serialised
+ * by the library (host mutex held across the synchronisation). */
+swf_status swf_validate_group_idx(const int32_t* group_idx, int64_t M, int32_t num_active_groups,
+                                  int32_t num_groups, int64_t* bad_slots, void* stream);
+
+/* Debug mode (default: on when the environment variable SWF_DEBUG is set and not "0" at the
+ * first query).  While it is on, every entry point that reads group_idx (swf_group_buckets,
+ * swf_group_frequency, sparse_swiglu_ffn_fwd, sparse_swiglu_ffn_bwd) first runs
+ * swf_validate_group_idx on its stream -- so it synchronises that stream -- and returns
+ * SWF_ERR_INVALID_ARG, having launched nothing else and left its outputs untouched, if any slot
+ * is invalid.  swf_set_debug(0 or 1) overrides the environment (else SWF_ERR_INVALID_ARG);
+ * swf_get_debug returns the mode in effect. */
+swf_status swf_set_debug(int32_t enable);
+int32_t swf_get_debug(void);
 
 /* ------------------------------------------------------------------ planning and queries */
 

@@ -56,6 +56,9 @@ SIGNATURES = {
     "swf_sparse_saved_bytes": (SZ, [I64, I64, I64, I32, I32, I32]),
     "swf_supported": (I32, [I32, I64, I64, I64, I32, I32, I32, I32]),
     "swf_plan": (I32, [I32, I64, I64, I64, I32, I32, I32, I32, C.POINTER(swf_plan_info)]),
+    "swf_validate_group_idx": (I32, [P, I64, I32, I32, C.POINTER(C.c_int64), P]),
+    "swf_set_debug": (I32, [I32]),
+    "swf_get_debug": (I32, []),
     "swf_device_status": (I32, [P]),
     "swf_selftest_wait_timeout": (I32, [I32, P]),
     "swf_status_string": (C.c_char_p, [I32]),

@@ -269,6 +269,27 @@ def group_frequency(group_idx, num_groups, freq=None, stream=None):
     return freq
 
 
+def validate_group_idx(group_idx, num_groups, stream=None):
+    """Counts the slots of group_idx [M, K] that are out of [0, num_groups) or repeat an earlier
+    slot of their row; synchronises the stream.  Returns (status, count): status 0 when every
+    slot is valid, 1 (SWF_ERR_INVALID_ARG) otherwise."""
+    M, K = group_idx.shape
+    bad = C.c_int64(-1)
+    st = _lib.lib().swf_validate_group_idx(_p(group_idx), M, K, num_groups, C.byref(bad), _stream(stream))
+    if st not in (_lib.SWF_OK, 1):
+        raise SwfError("swf_validate_group_idx", st)
+    return st, int(bad.value)
+
+
+def set_debug(enable: bool) -> None:
+    """Debug mode: entry points that read group_idx validate it first (and synchronise)."""
+    _check("swf_set_debug", _lib.lib().swf_set_debug(1 if enable else 0))
+
+
+def get_debug() -> bool:
+    return bool(_lib.lib().swf_get_debug())
+
+
 def update_load_balance_bias(bias, freq_ema, current_freq, target_freq, gamma=1e-3, bias_max=0.5,
                              momentum=0.99, stream=None):
     """In-place balancing step on the device buffers bias and freq_ema (fp32 [num_groups])."""

@@ -1,10 +1,11 @@
 // Inference forward that allocates nothing and needs no caller workspace.
 //
 // Some callers cannot hand the library a workspace: a host program that reaches the library
-// only through the C ABI and owns no device allocator of its own, a plug-in inside a runtime
-// that forbids device allocation on its execution path, or code running while a stream is
-// being captured in a mode where cudaMalloc is an error.  For them this entry point keeps the
+// only through the C ABI and owns no device allocator of its own, or a plug-in inside a runtime
+// that forbids device allocation on its execution path.  For them this entry point keeps the
 // intermediate h = SiLU(x W_gate^T) * (x W_up^T) in a fixed, file-scope device array instead.
+// Its first call on a device looks up the array's device address with that device current;
+// make that first call before any stream capture on the device.
 //
 // The array lives in every GPU that loads the library, until the process exits.  All calls
 // share it and it keeps the last call's contents; nothing in it needs to start at zero (the

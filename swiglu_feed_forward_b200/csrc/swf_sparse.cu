@@ -9,6 +9,9 @@
 // tile is past the last group).  row_token[r] is the token of padded row r (-1: padding);
 // padding rows of every group-major buffer are zero, so they add nothing to any sum.
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "swf_launch.cuh"
@@ -676,6 +679,100 @@ extern "C" swf_status grouped_topk_select(const void* x, const void* w_gate,
   return launch_topk<64>(E, bias, M, ng, K, group_idx, st);
 }
 
+// ------------------------------------------------------------------ group_idx validation
+
+// Count of invalid group_idx slots found by the last validation on this device.
+static __device__ unsigned long long g_swf_bad_slots;
+
+namespace swf {
+namespace {
+
+// One warp per row: a slot is invalid if its group is out of [0, ng) or repeats an earlier
+// slot of the same row (exactly the slots the bucketing drops).  Adds the count of invalid
+// slots to *bad.
+__global__ void validate_idx_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
+                                    unsigned long long* __restrict__ bad) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  unsigned long long n = 0;
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < M; t += warps) {
+    const int32_t* row = idx + t * K;
+    for (int k = lane; k < K; k += 32) n += valid_slot(row, k, ng) ? 0ull : 1ull;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+  if (lane == 0 && n) atomicAdd(bad, n);
+}
+
+std::mutex g_debug_mu;
+int g_debug = -1;  // -1: not yet read from the environment
+
+bool debug_on() {
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  if (g_debug < 0) {
+    const char* e = std::getenv("SWF_DEBUG");
+    g_debug = (e && *e && std::strcmp(e, "0") != 0) ? 1 : 0;
+  }
+  return g_debug == 1;
+}
+
+std::mutex g_validate_mu;
+unsigned long long* g_bad_ptr[64] = {};
+
+// Runs the validation of group_idx on `st` and waits for it.  SWF_ERR_INVALID_ARG if any slot
+// is invalid (its count in *bad_out when given).
+swf_status validate_idx(const int32_t* idx, int64_t M, int32_t K, int32_t ng, int64_t* bad_out,
+                        cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SWF_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lock(g_validate_mu);
+  if (!g_bad_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_swf_bad_slots) != cudaSuccess || !p) return SWF_ERR_LAUNCH;
+    g_bad_ptr[dev] = static_cast<unsigned long long*>(p);
+  }
+  unsigned long long* bad = g_bad_ptr[dev];
+  if (cudaMemsetAsync(bad, 0, sizeof(*bad), st) != cudaSuccess) return SWF_ERR_LAUNCH;
+  {
+    ProfScope prof(SWF_K_ELEMENTWISE, st);
+    validate_idx_kernel<<<grid_for(M, 8), 256, 0, st>>>(idx, M, K, ng, bad);
+    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
+  }
+  unsigned long long host = 0;
+  if (cudaMemcpyAsync(&host, bad, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SWF_ERR_LAUNCH;
+  if (bad_out) *bad_out = (int64_t)host;
+  return host ? SWF_ERR_INVALID_ARG : SWF_OK;
+}
+
+// In debug mode: the validation, before an entry point that reads group_idx launches anything.
+swf_status debug_check_idx(const int32_t* idx, int64_t M, int32_t K, int32_t ng, cudaStream_t st) {
+  return debug_on() ? validate_idx(idx, M, K, ng, nullptr, st) : SWF_OK;
+}
+
+}  // namespace
+}  // namespace swf
+
+extern "C" swf_status swf_set_debug(int32_t enable) {
+  if (enable != 0 && enable != 1) return SWF_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(swf::g_debug_mu);
+  swf::g_debug = enable;
+  return SWF_OK;
+}
+
+extern "C" int32_t swf_get_debug(void) { return swf::debug_on() ? 1 : 0; }
+
+extern "C" swf_status swf_validate_group_idx(const int32_t* group_idx, int64_t M,
+                                             int32_t num_active_groups, int32_t num_groups,
+                                             int64_t* bad_slots, void* stream) {
+  if (!group_idx || M <= 0 || num_active_groups <= 0 || num_groups <= 0) return SWF_ERR_INVALID_ARG;
+  if (!aligned16(group_idx)) return SWF_ERR_ALIGNMENT;
+  if (M * (int64_t)num_active_groups >= (int64_t(1) << 31)) return SWF_ERR_UNSUPPORTED;
+  return validate_idx(group_idx, M, num_active_groups, num_groups, bad_slots,
+                      static_cast<cudaStream_t>(stream));
+}
+
 // ------------------------------------------------------------------ bucketing
 
 extern "C" swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t K, int32_t ng,
@@ -687,6 +784,7 @@ extern "C" swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int
   if (ng > 12288) return SWF_ERR_UNSUPPORTED;
   if (!aligned16(workspace)) return SWF_ERR_ALIGNMENT;
   if (ws_bytes < buckets_workspace_bytes(M, K, ng)) return SWF_ERR_WORKSPACE;
+  if ((s = debug_check_idx(group_idx, M, K, ng, static_cast<cudaStream_t>(stream))) != SWF_OK) return s;
   const SparseDims d = dims_of(M, 16, (int64_t)ng * 16, 16, K);
   return run_buckets(group_idx, d, static_cast<int32_t*>(workspace), offsets, tokens, nullptr,
                      nullptr, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
@@ -735,6 +833,7 @@ extern "C" swf_status swf_group_frequency(const int32_t* group_idx, int64_t M, i
   if (ng > 12288) return SWF_ERR_UNSUPPORTED;
   if (!aligned16(group_idx) || !aligned16(freq)) return SWF_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = debug_check_idx(group_idx, M, K, ng, st)) != SWF_OK) return s;
   ProfScope prof(SWF_K_BALANCE, st);
   group_frequency_kernel<<<1, 1024, ng * sizeof(int32_t), st>>>(group_idx, M, K, ng, freq);
   return launched();
@@ -781,6 +880,7 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
   const FwdWs w = fwd_ws(workspace, sd, &need_ws);
   if (saved_bytes < need_saved || ws_bytes < need_ws) return SWF_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = debug_check_idx(group_idx, M, K, sd.ng, st)) != SWF_OK) return s;
 
   if ((s = run_buckets(group_idx, sd, w.counts, v.offs, v.tokens, v.seg_start, v.seg_rows,
                        v.tile_group, v.row_token, v.pair_row, st)) != SWF_OK)
@@ -841,6 +941,7 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
   const BwdWs w = bwd_ws(workspace, sd, &need_ws);
   if (saved_bytes < need_saved || ws_bytes < need_ws) return SWF_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = debug_check_idx(group_idx, M, K, sd.ng, st)) != SWF_OK) return s;
 
   // the forward's gathered x rows are in `saved`; only dY is gathered here
   if ((s = run_gather(dy, v, sd, w.dyc, st)) != SWF_OK) return s;

@@ -141,3 +141,22 @@ def test_subsample_index_errors(lib):
     assert lib.swf_make_subsample_index(4096, 64, 65, 0, ptr) == 2
     assert lib.swf_make_subsample_index(4000, 64, 8, 0, ptr) == 2
     assert lib.swf_make_subsample_index(4096, 64, 8, 0, None) == 1
+
+
+def test_group_idx_validation_rejects_bad_arguments_on_the_host(lib):
+    """swf_validate_group_idx checks its arguments before touching the GPU; the debug switch
+    takes only 0 or 1 and reports what it was set to."""
+    bad = C.c_int64(-1)
+    assert lib.swf_validate_group_idx(None, 10, 2, 8, C.byref(bad), None) == 1       # null
+    assert lib.swf_validate_group_idx(C.c_void_p(16), 0, 2, 8, C.byref(bad), None) == 1  # M = 0
+    assert lib.swf_validate_group_idx(C.c_void_p(16), 10, 0, 8, C.byref(bad), None) == 1  # K = 0
+    assert lib.swf_validate_group_idx(C.c_void_p(20), 10, 2, 8, C.byref(bad), None) == 3  # misaligned
+    assert lib.swf_validate_group_idx(C.c_void_p(16), 1 << 30, 4, 8, C.byref(bad), None) == 2  # M*K >= 2^31
+    assert bad.value == -1  # nothing written
+    prev = lib.swf_get_debug()
+    try:
+        assert lib.swf_set_debug(2) == 1
+        assert lib.swf_set_debug(1) == 0 and lib.swf_get_debug() == 1
+        assert lib.swf_set_debug(0) == 0 and lib.swf_get_debug() == 0
+    finally:
+        lib.swf_set_debug(prev)
