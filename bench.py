@@ -478,22 +478,21 @@ def sparse_step_algorithmic_bytes(M, d, f, G, K, spg):
 def sparse_step_design_bytes(M, d, f, G, K, spg, R):
     """HBM bytes the group-sparse step's kernels move in this design (bf16 data, int32
     indices), with R the padded pair rows: selection (x, the sampled gate rows, the chosen
-    groups), the gathers (x and dY rows written group-major; the token rows come from L2), the
-    row-grouped GEMMs (gathered rows, the group's weights, h, a, b, [dG | dU]), the per-pair y and
-    dx contributions written and summed, and the grouped weight gradients.  The [dG | dU] rows
-    are 128 columns wide for every group size (each half padded to 64 columns)."""
+    groups), bucketing, the row-grouped GEMMs (the token rows of x and dY gathered from L2, so
+    each read from HBM once per GEMM; the group's weights; h, a, b; [dG | dU]), the per-pair y
+    and dx contributions written and summed per token, and the grouped weight gradients.  The
+    [dG | dU] rows are 128 columns wide for every group size (each half padded to 64 columns)."""
     b, ng = 2, f // G
     P = 1 << max(0, (spg - 1).bit_length())
     select = b * M * d + b * ng * P * d + 4 * M * K
     buckets = 3 * 4 * M * K
-    gather = b * R * d + b * M * d                               # one of x, dY
-    up = b * R * d + 2 * b * f * d + 3 * b * R * G
+    up = b * M * d + 2 * b * f * d + 3 * b * R * G
     down = b * R * G + b * d * f + b * R * d
     pair_sum = b * R * d + b * M * d + 4 * M * K                 # one of y, dx
-    dgate = b * R * d + b * d * f + 2 * b * R * G + b * R * 128
+    dgate = b * M * d + b * d * f + 2 * b * R * G + b * R * 128
     dxg = b * R * 128 + 2 * b * f * d + b * R * d
-    dw = (b * R * 128 + b * R * d + 2 * b * f * d) + (b * R * d + b * R * G + b * d * f)
-    return select + buckets + 2 * gather + up + down + 2 * pair_sum + dgate + dxg + dw
+    dw = (b * R * 128 + b * M * d + 2 * b * f * d) + (b * M * d + b * R * G + b * d * f)
+    return select + buckets + up + down + 2 * pair_sum + dgate + dxg + dw
 
 
 def secondary_sparse(api, steps, warmup, world, peaks, skewed=False):

@@ -282,10 +282,10 @@ swf_status swf_group_buckets(const int32_t* group_idx, int64_t M, int32_t num_ac
  * with W_*[c] the group's G rows.  Each (token, group) contribution is computed in fp32 and
  * stored in `dtype`; a token's contributions are then summed in fp32 in the order of its
  * group_idx slots, so y is bitwise deterministic (the README's kernel uses fp32 atomics
- * instead).  `saved`
- * (swf_sparse_saved_bytes bytes) receives what the backward needs: the bucketing, the
- * compact per-pair h, a, b and the gathered x rows; the caller keeps it for
- * sparse_swiglu_ffn_bwd (which reads x from it, not from its own x argument). */
+ * instead).  The GEMMs gather the token rows of x themselves (from L2); no gathered copy of x
+ * is written.  `saved` (swf_sparse_saved_bytes bytes) receives what the backward needs: the
+ * bucketing and the compact per-pair h, a, b; the caller keeps it for sparse_swiglu_ffn_bwd,
+ * together with x and the group_idx (the backward reads both again). */
 swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, const void* w_up,
                                  const void* w_down, const int32_t* group_idx, int32_t group_size,
                                  int32_t num_active_groups, void* y, void* saved,

@@ -12,7 +12,7 @@ inline int cdiv(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 
 // Launches tc_gemm_kernel on min(tiles, SMs) persistent CTAs, bracketed for profiling as `kind`.
 template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense,
-          bool TMA_EPI = false>
+          bool TMA_EPI = false, int GATHER = kGatherNone>
 swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
                      const CUtensorMap& tb1, TcGemmArgs args, cudaStream_t st,
                      const EpiMaps& em = EpiMaps{}) {
@@ -26,14 +26,14 @@ swf_status launch_tc(int kind, const CUtensorMap& ta, const CUtensorMap& tb0,
   args.status = ctx.status;
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;
   args.raster = std::max(1, std::min(args.raster, args.num_m_blk));
-  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE, false, TMA_EPI>;
+  auto kern = tc_gemm_kernel<BN, A_MN, B_MN, B_DUAL, EPI, MODE, false, TMA_EPI, GATHER>;
   constexpr int smem = TcSmem<BN, false, epi_smem_bytes<EPI, TMA_EPI, false>()>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   const int64_t units = args.unit > 1 ? (tiles + args.unit - 1) / args.unit : tiles;
   const int grid = (int)std::min<int64_t>(units, ctx.num_sms);
   ProfScope prof(kind, st);
-  kern<<<grid, kGemmThreads, smem, st>>>(ta, tb0, tb1, em, args);
+  kern<<<grid, gemm_threads<GATHER>(), smem, st>>>(ta, tb0, tb1, em, args);
   return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
 }
 

@@ -69,7 +69,6 @@ struct Carver {
 struct SavedView {
   int32_t *offs, *tokens, *seg_start, *seg_rows, *tile_group, *row_token, *pair_row;
   __nv_bfloat16 *h, *a, *b;
-  __nv_bfloat16* xc;  // the gathered x rows (group-major), reused by the backward
 };
 
 SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
@@ -85,7 +84,6 @@ SavedView saved_view(void* base, const SparseDims& s, size_t* bytes) {
   v.h = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.a = c.take<__nv_bfloat16>(s.rmax * s.G);
   v.b = c.take<__nv_bfloat16>(s.rmax * s.G);
-  v.xc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
   return v;
 }
@@ -104,13 +102,12 @@ FwdWs fwd_ws(void* base, const SparseDims& s, size_t* bytes) {
 }
 
 struct BwdWs {
-  __nv_bfloat16 *dyc, *dgu;
+  __nv_bfloat16* dgu;
   __nv_bfloat16* dxc;  // per-pair contributions to dx, group-major rows
 };
 BwdWs bwd_ws(void* base, const SparseDims& s, size_t* bytes) {
   Carver c{static_cast<char*>(base)};
   BwdWs w;
-  w.dyc = c.take<__nv_bfloat16>(s.rmax * s.d);
   w.dgu = c.take<__nv_bfloat16>(s.rmax * 128);
   w.dxc = c.take<__nv_bfloat16>(s.rmax * s.d);
   if (bytes) *bytes = c.off;
@@ -338,26 +335,6 @@ __global__ void pair_sum_kernel(const uint4* __restrict__ rows, const int32_t* _
   }
 }
 
-// dst[r, :] = src[row_token[r], :] (zero for padding) for the padded rows in use; one warp per
-// row, 16-byte vectors.
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ row_token,
-                                   const int32_t* __restrict__ seg_start_total, int64_t row_vecs,
-                                   uint4* __restrict__ dst) {
-  const int64_t rows = *seg_start_total;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const int32_t tok = row_token[r];
-    uint4* d = dst + r * row_vecs;
-    if (tok < 0) {
-      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
-    } else {
-      const uint4* s = src + (int64_t)tok * row_vecs;
-      for (int64_t v = lane; v < row_vecs; v += 32) d[v] = s[v];
-    }
-  }
-}
-
 // Wsub[c*P + i, :] = w_gate[sub[c*spg + i], :] for i < spg, zero rows for spg <= i < P (zero rows
 // add |SiLU(0)| = 0 to the energy).  Row ids outside group c are treated as zero rows.
 __global__ void select_gather_kernel(const uint4* __restrict__ w, const int32_t* __restrict__ sub,
@@ -480,20 +457,20 @@ swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts,
   return launched();
 }
 
-swf_status run_gather(const void* src, const SavedView& v, const SparseDims& s, void* dst,
-                      cudaStream_t st) {
-  ProfScope prof(SWF_K_SPARSE_GATHER, st);
-  gather_rows_kernel<<<148 * 8, 256, 0, st>>>(static_cast<const uint4*>(src), v.row_token,
-                                              v.seg_start + s.ng, s.d / 8, static_cast<uint4*>(dst));
-  return launched();
-}
-
 swf_status run_pair_sum(const void* rows, const int32_t* pair_row, const SparseDims& s, void* out,
                         cudaStream_t st) {
   ProfScope prof(SWF_K_PAIR_SUM, st);
   pair_sum_kernel<<<grid_for(s.M, 8), 256, 0, st>>>(static_cast<const uint4*>(rows), pair_row, s.M, s.K,
                                                    s.d / 8, static_cast<uint4*>(out));
   return launched();
+}
+
+// The gathered operand of a sparse GEMM: padded row r is row row_token[r] of src [tokens, d].
+void set_gather(TcGemmArgs& a, const int32_t* row_token, const void* src, int64_t d) {
+  a.gather_token = row_token;
+  a.gather_src = src;
+  a.gather_ld = d;
+  a.gather_cols = (int)d;
 }
 
 template <int VPL>
@@ -555,13 +532,13 @@ void sparse_plan(int op, int64_t M, int64_t d, int64_t f, int32_t G, int32_t K, 
       p->gemm_tiles = (int64_t)cdiv(M, 128) * cdiv((int64_t)s.ng * P, 256);
       break;
     case SWF_OP_SPARSE_FWD:
-      p->num_kernels = 8;
+      p->num_kernels = 7;  // bucketing (count, scan, fill, place), gate|up, down, pair sum
       p->flops = 6 * M * d * (int64_t)K * G;
       p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256));
       p->tile_n = 2 * G;
       break;
     case SWF_OP_SPARSE_BWD:
-      p->num_kernels = 8;
+      p->num_kernels = 5;  // dgate, dx, pair sum, dW_gate|dW_up, dW_down
       p->flops = 12 * M * d * (int64_t)K * G;
       p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256)) + (int64_t)s.ng * (cdiv(d, 256) + cdiv(d, 128));
       break;
@@ -885,12 +862,10 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
   if ((s = run_buckets(group_idx, sd, w.counts, v.offs, v.tokens, v.seg_start, v.seg_rows,
                        v.tile_group, v.row_token, v.pair_row, st)) != SWF_OK)
     return s;
-  if ((s = run_gather(x, v, sd, v.xc, st)) != SWF_OK) return s;
-
-  {  // gate|up per group: [h|a|b] rows = SiLU/gating of Xc [W_g[g] | W_u[g]]^T
-    CUtensorMap txc, twg, twu;
-    if (!encode_tmap_bf16(&txc, v.xc, d, sd.rmax, d, 64, 128) ||
-        !encode_tmap_bf16(&twg, w_gate, d, f, d, 64, G) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, G))
+  {  // gate|up per group: [h|a|b] rows = SiLU/gating of X rows [W_g[g] | W_u[g]]^T, the X rows
+     // of each tile gathered from x by the kernel (from L2)
+    CUtensorMap twg, twu;
+    if (!encode_tmap_bf16(&twg, w_gate, d, f, d, 64, G) || !encode_tmap_bf16(&twu, w_up, d, f, d, 64, G))
       return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, G, 2 * G, d);
     a.num_n_blk = 1;
@@ -901,9 +876,13 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     a.aux0 = v.a;
     a.aux1 = v.b;
     a.ld_aux = G;
-    if (G == 16) s = launch_tc<32, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
-    else if (G == 32) s = launch_tc<64, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
-    else s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped>(SWF_K_SPARSE_UP, txc, twg, twu, a, st);
+    set_gather(a, v.row_token, x, d);
+    if (G == 16)
+      s = launch_tc<32, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
+    else if (G == 32)
+      s = launch_tc<64, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
+    else
+      s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
     if (s != SWF_OK) return s;
   }
   {  // down per group: yc[r] = h_row W_d[:, g*G .. g*G+G]^T
@@ -943,12 +922,10 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = debug_check_idx(group_idx, M, K, sd.ng, st)) != SWF_OK) return s;
 
-  // the forward's gathered x rows are in `saved`; only dY is gathered here
-  if ((s = run_gather(dy, v, sd, w.dyc, st)) != SWF_OK) return s;
-  {  // dH = dYc W_d[:, g]; dG = dH * a, dU = dH * b -> dgu [R, 128] (halves padded to 64)
-    CUtensorMap tdyc, twd;
-    if (!encode_tmap_bf16(&tdyc, w.dyc, d, sd.rmax, d, 64, 128) || !encode_tmap_bf16(&twd, w_down, f, d, f, 64, 64))
-      return SWF_ERR_LAUNCH;
+  // the token rows of x and dY are gathered by the GEMMs that read them (from L2)
+  {  // dH = dY rows W_d[:, g]; dG = dH * a, dU = dH * b -> dgu [R, 128] (halves padded to 64)
+    CUtensorMap twd;
+    if (!encode_tmap_bf16(&twd, w_down, f, d, f, 64, 64)) return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(sd.rmax, G, 64, d);
     a.num_n_blk = 1;
     a.tile_group = v.tile_group;
@@ -960,7 +937,8 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.aux0 = v.a;
     a.aux1 = v.b;
     a.ld_aux = G;
-    s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped>(SWF_K_SPARSE_DGATE, tdyc, twd, twd, a, st);
+    set_gather(a, v.row_token, dy, d);
+    s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_DGATE, twd, twd, twd, a, st);
     if (s != SWF_OK) return s;
   }
   {  // dxc[r] = dG_row W_g[g] + dU_row W_u[g]
@@ -980,11 +958,9 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     if (s != SWF_OK) return s;
   }
   if ((s = run_pair_sum(w.dxc, v.pair_row, sd, dx, st)) != SWF_OK) return s;
-  {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ Xc_seg
-    CUtensorMap tdgu, txc;
-    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64) ||
-        !encode_tmap_bf16(&txc, v.xc, d, sd.rmax, d, 64, 64))
-      return SWF_ERR_LAUNCH;
+  {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ X rows of the segment (gathered from x)
+    CUtensorMap tdgu;
+    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64)) return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(128, d, 256, 0);
     a.n_groups = sd.ng;
     a.seg_start = v.seg_start;
@@ -994,13 +970,13 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.out0 = dw_gate;
     a.out1 = dw_up;
     a.ld_out = d;
-    s = launch_tc<256, true, true, false, kEpiGroupDWgu, kModeKGrouped>(SWF_K_SPARSE_DW, tdgu, txc, txc, a, st);
+    set_gather(a, v.row_token, x, d);
+    s = launch_tc<256, true, true, false, kEpiGroupDWgu, kModeKGrouped, false, kGatherB>(SWF_K_SPARSE_DW, tdgu, tdgu, tdgu, a, st);
     if (s != SWF_OK) return s;
   }
-  {  // per group: dW_d[:, g] = dYc_segᵀ h_seg
-    CUtensorMap tdyc, th;
-    if (!encode_tmap_bf16(&tdyc, w.dyc, d, sd.rmax, d, 64, 64) || !encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64))
-      return SWF_ERR_LAUNCH;
+  {  // per group: dW_d[:, g] = (dY rows of the segment)ᵀ h_seg, the dY rows gathered from dy
+    CUtensorMap th;
+    if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64)) return SWF_ERR_LAUNCH;
     TcGemmArgs a = base_args(d, G, 64, 0);
     a.n_groups = sd.ng;
     a.seg_start = v.seg_start;
@@ -1009,7 +985,8 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.group_size = G;
     a.out0 = dw_down;
     a.ld_out = f;
-    s = launch_tc<64, true, true, false, kEpiGroupDWd, kModeKGrouped>(SWF_K_SPARSE_DW, tdyc, th, th, a, st);
+    set_gather(a, v.row_token, dy, d);
+    s = launch_tc<64, true, true, false, kEpiGroupDWd, kModeKGrouped, false, kGatherA>(SWF_K_SPARSE_DW, th, th, th, a, st);
   }
   return s;
 }

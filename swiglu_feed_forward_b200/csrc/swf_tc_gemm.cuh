@@ -81,6 +81,20 @@ constexpr int kTileK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;
 constexpr int kGemmThreads = 192;
 
+// Operands whose rows are gathered from token rows (group-sparse path) instead of loaded by TMA:
+//   kGatherA  row-grouped mode: the K-major A tile's 128 rows (padded pair rows); per-group-K
+//             mode: the MN-major A tile's 64 K rows
+//   kGatherB  per-group-K mode: the MN-major B tile's 64 K rows
+// Padded row r holds token gather_token[r] of gather_src (-1: a zero row).  kGatherWarps extra
+// warps (6 ..) copy the rows 16 bytes at a time with cp.async into the stage's 128-byte-swizzled
+// layout, each warp taking every kGatherWarps-th k-block; the token rows (x or dY) come from L2.
+enum : int { kGatherNone = 0, kGatherA = 1, kGatherB = 2 };
+constexpr int kGatherWarps = 4;
+template <int GATHER>
+constexpr int gemm_threads() {
+  return GATHER != kGatherNone ? kGemmThreads + 32 * kGatherWarps : kGemmThreads;
+}
+
 struct TcGemmArgs {
   int M;            // rows of C (kModeKGrouped: rows of each group's C)
   int N;            // columns of C that exist (kEpiSwiGLU*: d_ff; sparse: group_size)
@@ -122,6 +136,11 @@ struct TcGemmArgs {
   int64_t part_plane;     //   elements per split (M * N)
   int* status;            // device status word
   uint64_t wait_limit_ns;
+  // gathered operand (GATHER != kGatherNone)
+  const int32_t* gather_token;  // token of each padded row (-1: zero row)
+  const void* gather_src;       // bf16 token rows [tokens][gather_ld]
+  int64_t gather_ld;            // elements between token rows
+  int gather_cols;              // columns that exist (the rest of a tile reads as zero)
 };
 
 // Epilogues that move their tiles with TMA: bf16 outputs staged per warp in shared memory
@@ -352,8 +371,8 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float* v) {
 // and runs its own epilogue.  Both CTAs' TMA loads complete on the even CTA's stage barrier,
 // and the MMA commits arrive on the stage and accumulator barriers of both CTAs.
 template <int BN, bool A_MN, bool B_MN, bool B_DUAL, int EPI, int MODE = kModeDense,
-          bool PAIR = false, bool TMA_EPI = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+          bool PAIR = false, bool TMA_EPI = false, int GATHER = kGatherNone>
+__global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ EpiMaps emaps,
                    const TcGemmArgs args) {
@@ -365,6 +384,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
   static_assert(!B_MN || kBRows % 64 == 0, "MN-major B tiles are whole 64-column boxes");
   static_assert(!PAIR || (MODE == kModeDense && BN % 32 == 0), "pair mode: dense tiles");
+  static_assert(GATHER == kGatherNone ||
+                    (!PAIR && ((GATHER == kGatherA && MODE == kModeRowGrouped && !A_MN) ||
+                               (GATHER == kGatherA && MODE == kModeKGrouped && A_MN) ||
+                               (GATHER == kGatherB && MODE == kModeKGrouped && B_MN))),
+                "gathered operands: K-major A of row-grouped tiles, MN-major A or B of per-group-K tiles");
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
                                                     EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
                                                     EPI == kEpiScale || EPI == kEpiLeakySq)) ||
@@ -395,7 +419,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      // gathered operand: one arrival per lane of the gathering warp after its copies land
+      mbar_init(&full[s], GATHER != kGatherNone ? 33 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -444,7 +469,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&empty[s], ph ^ 1u, ctl)) { ok = false; break; }
           uint8_t* sA = smem + s * L::kStageBytes;
           uint8_t* sB = sA + L::kABytes;
-          if (!PAIR) mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+          if (!PAIR)
+            mbar_arrive_expect_tx(&full[s], GATHER == kGatherA   ? L::kBBytes
+                                            : GATHER == kGatherB ? L::kABytes
+                                                                 : L::kStageBytes);
           else if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kStageBytes);
           auto load = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
             if constexpr (PAIR) tma_load_2d_pair(dst, m, c0, c1, full_lead + s * 8);
@@ -453,7 +481,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const bool seg1 = kb >= args.kb_seg0;
           const int kk = (seg1 ? kb - args.kb_seg0 : kb) * kTileK;  // K inside the segment
           const int ka = t.a_k + (seg1 ? args.a_koff1 + kk : kk);
-          if (A_MN) {
+          if (GATHER == kGatherA) {
+            // rows copied by the gather warps
+          } else if (A_MN) {
             load(sA, &tmA, t.a_m, ka);
             load(sA + 8192, &tmA, t.a_m + 64, ka);
           } else {
@@ -468,6 +498,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               load(sB, &tmB0, t.b_k + kk, t.b_n);
               load(sB + (BN / 2) * 128, &tmB1, t.b_k + kk, t.b_n);
             }
+          } else if (GATHER == kGatherB) {
+            // rows copied by the gather warps
           } else if (B_MN) {
 #pragma unroll
             for (int j = 0; j < kBRows / 64; ++j) load(sB + j * 8192, mapB, b_n + j * 64, t.b_k + kk);
@@ -516,6 +548,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t d_tmem = tmem_base + buf * BN;
         for (int kb = 0; kb < t.kb; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl)) { ok = false; break; }
+          // gathered rows were written by cp.async (generic proxy); the barrier made them
+          // visible to this thread, the fence orders them before the MMAs' async-proxy reads
+          if constexpr (GATHER != kGatherNone) fence_proxy_async_smem();
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(s) * (L::kStageBytes / 16);
 #pragma unroll
@@ -550,6 +585,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         quick.abort = &no_abort;
         mbar_wait(drain, 0, quick);
       }
+    }
+  } else if (GATHER != kGatherNone && warp >= 6) {
+    // ------------------------------------------------------------ gather warps 6 ..
+    if constexpr (GATHER != kGatherNone) {
+      constexpr bool kKGrp = MODE == kModeKGrouped;
+      constexpr int kRows = kKGrp ? kTileK : kTileM;          // rows of the gathered tile
+      constexpr int kBlocks = GATHER == kGatherA ? (kKGrp ? 2 : 1) : kBRows / 64;  // 64-col blocks
+      constexpr int kPerLane = kRows / 4;                     // rows per lane (4 rows per warp step)
+      constexpr uint32_t kOpOff = GATHER == kGatherA ? 0u : (uint32_t)L::kABytes;
+      const int gw = warp - 6;
+      const int ch = lane & 7;     // 16-byte chunk of a 128-byte row piece
+      const int rsub = lane >> 3;  // row of the warp's 4-row step
+      const char* src = static_cast<const char*>(args.gather_src);
+      const int64_t ld_bytes = args.gather_ld * 2;
+      const uint32_t sbase = smem_u32(smem) + kOpOff;
+      uint32_t it = 0;
+      bool ok = true;
+      int tok[kPerLane];
+      for (int i_ = 0, tile = tile0 * unit_; ok && tile < num_tiles; tile = sched_tile(++i_, tile0, tile_step, unit_)) {
+        const Tile t = decode_tile<BN, B_DUAL, MODE>(tile, args);
+        if (t.grp < 0) continue;
+        if constexpr (!kKGrp) {  // the tile's 128 padded rows are its M rows: same for every k-block
+#pragma unroll
+          for (int i = 0; i < kPerLane; ++i) tok[i] = args.gather_token[t.a_m + rsub + 4 * i];
+        }
+        for (int kb = 0; kb < t.kb; ++kb, ++it) {
+          if ((int)(it % kGatherWarps) != gw) continue;
+          const int s = (int)(it % S);
+          const uint32_t ph = (it / S) & 1u;
+          const bool got = mbar_wait(&empty[s], ph ^ 1u, ctl);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          int col0;
+          if constexpr (kKGrp) {  // the K rows change with every k-block
+            const int r0 = (GATHER == kGatherA ? t.a_k : t.b_k) + kb * kTileK;
+#pragma unroll
+            for (int i = 0; i < kPerLane; ++i) tok[i] = args.gather_token[r0 + rsub + 4 * i];
+            col0 = GATHER == kGatherA ? t.a_m : t.b_n;
+          } else {
+            col0 = t.a_k + kb * kTileK;
+          }
+          const uint32_t sop = sbase + (uint32_t)s * L::kStageBytes;
+#pragma unroll
+          for (int j = 0; j < kBlocks; ++j) {
+            const int col = col0 + j * 64 + ch * 8;
+            const bool col_ok = col < args.gather_cols;
+#pragma unroll
+            for (int i = 0; i < kPerLane; ++i) {
+              const int r = rsub + 4 * i;
+              const uint32_t dst = sop + (uint32_t)(j * kRows * 128 + r * 128 + ((ch ^ (r & 7)) << 4));
+              const bool v = col_ok && tok[i] >= 0;
+              cp_async16(dst, src + (v ? (int64_t)tok[i] * ld_bytes + (int64_t)col * 2 : 0), v);
+            }
+          }
+          cp_async_arrive_noinc(&full[s]);
+        }
+      }
+      cp_async_wait_all();  // copies still in flight land before the CTA leaves
     }
   } else if constexpr (TMA_EPI) {
     // ------------------------------------------------------------ epilogue warps 2..5 (TMA I/O)

@@ -85,7 +85,8 @@ def test_sparse_algorithmic_bytes_at_workload3():
     alg = bench.sparse_step_algorithmic_bytes(16384, 1024, 4096, 64, 8, 8)
     assert 0.37e9 < alg < 0.39e9
     R = 16384 * 8 + 64 * 64  # padded pair rows of a balanced selection
-    assert bench.sparse_step_design_bytes(16384, 1024, 4096, 64, 8, 8, R) > 5 * alg
+    design = bench.sparse_step_design_bytes(16384, 1024, 4096, 64, 8, 8, R)
+    assert 3 * alg < design < 1.7e9  # mostly the per-pair y and dx rows: 4 x 277 MB
     # the algorithmic bytes do not depend on the padding and grow with the number of groups kept
     assert bench.sparse_step_algorithmic_bytes(16384, 1024, 4096, 64, 4, 8) < alg
 
