@@ -735,19 +735,19 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
         } else if constexpr (kGLU) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float hv[2], av[2], bv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float g = v0[2 * i + e], u = v1[2 * i + e];
-              const float sg = sigmoidf_(g);
-              bv[e] = g * sg;
-              hv[e] = bv[e] * u;
-              av[e] = u * sg * (1.f + g * (1.f - sg));
-            }
-            w[0][i] = pack_bf16x2(hv[0], hv[1]);
+            // two columns per f32x2 multiply / FMA (2.2% fewer cycles per k-block on B200: the
+            // epilogue shares an issue slot with the MMA-issuing warp)
+            const float2 g2 = make_float2(v0[2 * i], v0[2 * i + 1]);
+            const float2 u2 = make_float2(v1[2 * i], v1[2 * i + 1]);
+            const float2 s2 = make_float2(sigmoidf_(g2.x), sigmoidf_(g2.y));
+            const float2 b2 = __fmul2_rn(g2, s2);
+            const float2 h2 = __fmul2_rn(b2, u2);
+            w[0][i] = pack_bf16x2(h2.x, h2.y);
             if constexpr (EPI == kEpiSwiGLU) {
-              w[1][i] = pack_bf16x2(av[0], av[1]);
-              w[2][i] = pack_bf16x2(bv[0], bv[1]);
+              const float2 oms = __ffma2_rn(s2, make_float2(-1.f, -1.f), make_float2(1.f, 1.f));
+              const float2 a2 = __fmul2_rn(u2, __ffma2_rn(b2, oms, s2));  // u (s + SiLU(g) (1 - s))
+              w[1][i] = pack_bf16x2(a2.x, a2.y);
+              w[2][i] = pack_bf16x2(b2.x, b2.y);
             }
           }
         } else if constexpr (EPI == kEpiLeakySq) {
