@@ -177,8 +177,9 @@ swf_status dense_bwd_bf16(const void* dy, const void* x, const void* wg, const v
     // dG and dU leave by TMA through two views of dGU (each [M, f], rows 2f apart)
     EpiMaps e3{};
     const __nv_bfloat16* dgu_b = static_cast<const __nv_bfloat16*>(dgu);
-    if (!epi_map(&e3.o[0], dgu_b, f, M, 2 * f) || !epi_map(&e3.o[1], dgu_b + f, f, M, 2 * f) ||
-        !epi_map(&e3.o[2], a, f, M, f) || !epi_map(&e3.o[3], b, f, M, f))
+    constexpr int kBc = tma_epi_cols<kEpiDGate>();
+    if (!epi_map(&e3.o[0], dgu_b, f, M, 2 * f, kBc) || !epi_map(&e3.o[1], dgu_b + f, f, M, 2 * f, kBc) ||
+        !epi_map(&e3.o[2], a, f, M, f, kBc) || !epi_map(&e3.o[3], b, f, M, f, kBc))
       return SWF_ERR_LAUNCH;
     TcGemmArgs k3 = base_args(M, f, 256, d, 2 * kTileM);
     s = launch_tc_pair<256, false, true, false, kEpiDGate, true>(SWF_K_DGATE, tdy, twd, twd, e3, k3, st);

@@ -177,16 +177,29 @@ constexpr int tma_epi_out_bufs() {
 // two or eight k-blocks, so each tile is mostly epilogue, and half the chunks means half the
 // TMEM-load waits, proxy fences and TMA copies (sparse down 84 -> 62 us, LeakyReLU^2 up 186 ->
 // 167 us on B200).  The others keep 32 x 32 boxes (64-byte swizzle).
+//
+// kEpiDGate works in place: its two factor boxes (a, b: 32 rows x 64 columns, 128-byte swizzle)
+// receive dG = dH a and dU = dH b and are stored from there, so it needs no output boxes and
+// moves whole 128-byte rows.  Measured with a %clock64 probe of the MMA issuer on B200, the dH
+// kernel's k-blocks take about 544 cycles when its epilogue moves nothing and 620-650 with the
+// factor loads and output stores of 32-column chunks: the epilogue's TMA operations delay the
+// operand loads of the main loop (the same at 74, 48 and 32 clusters, so not a DRAM limit).
 template <int EPI>
 constexpr int tma_epi_cols() {
-  return (EPI == kEpiStore || EPI == kEpiLeakySq || EPI == kEpiScale) ? 64 : 32;
+  return (EPI == kEpiStore || EPI == kEpiLeakySq || EPI == kEpiScale || EPI == kEpiDGate) ? 64 : 32;
+}
+template <int EPI>
+constexpr bool tma_epi_in_place() {
+  return EPI == kEpiDGate;
 }
 template <int EPI, bool TMA_EPI, bool PAIR>
 constexpr int epi_smem_bytes() {
-  return EPI == kEpiEnergyTopK ? kTopKMaxGroups * kTileM * 4
-                               : (TMA_EPI ? 4 * (tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>() * 64 * tma_epi_cols<EPI>() +
-                                                 tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>() * 64 * tma_epi_cols<EPI>())
-                                          : 0);
+  return EPI == kEpiEnergyTopK
+             ? kTopKMaxGroups * kTileM * 4
+             : (TMA_EPI ? 4 * ((tma_epi_in_place<EPI>() ? 0 : tma_epi_out_bufs<PAIR>() * tma_epi_outputs<EPI>()) *
+                                   64 * tma_epi_cols<EPI>() +
+                               tma_epi_aux_bufs<EPI>() * tma_epi_aux<EPI>() * 64 * tma_epi_cols<EPI>())
+                        : 0);
 }
 
 // Tensor maps of a TMA epilogue: outputs in o[0..], then the factors it loads by TMA from
@@ -650,7 +663,8 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
     constexpr bool kGLU = EPI == kEpiSwiGLU || EPI == kEpiSwiGLUInf;
     constexpr bool kDual = kGLU;  // [g | u] accumulator halves
     constexpr int CWO = tma_epi_cols<EPI>();  // output columns per chunk
-    static_assert(CWO == 32 || (CWO == 64 && !kDual && NAUX <= 1), "64-column chunks");
+    constexpr bool kInPlace = tma_epi_in_place<EPI>();
+    static_assert(CWO == 32 || (CWO == 64 && !kDual && (NAUX <= 1 || kInPlace)), "64-column chunks");
     constexpr int kOutBox = 64 * CWO;         // bytes of one 32-row output (or factor) box
     constexpr int NCH = (kDual ? BN / 2 : BN) / CWO;
     static_assert((kDual ? BN / 2 : BN) % CWO == 0, "whole chunks");
@@ -658,8 +672,9 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
     const int ew = warp - 2;
     constexpr int AB = tma_epi_aux_bufs<EPI>();
     constexpr int OB = tma_epi_out_bufs<PAIR>();
-    uint8_t* ebase = smem + L::kEpiOffset + ew * (OB * NOUT + AB * NAUX) * kOutBox;  // boxes [NOUT][OB]
-    uint8_t* abase = ebase + OB * NOUT * kOutBox;  // aux buffers [AB][NAUX]
+    constexpr int kOutBoxes = kInPlace ? 0 : OB * NOUT;
+    uint8_t* ebase = smem + L::kEpiOffset + ew * (kOutBoxes + AB * NAUX) * kOutBox;  // boxes [NOUT][OB]
+    uint8_t* abase = ebase + kOutBoxes * kOutBox;  // aux buffers [AB][NAUX]
     uint64_t* abar = auxbar + ew * AB;
     const uint32_t tempty_lead = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
     const int swz = (lane >> 1) & 3;  // 64-byte swizzle phase of this lane's staging row
@@ -688,7 +703,10 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
           ++aux_issued;
         }
       };
-      // the factors do not depend on the accumulator: fetch the first chunks' early
+      // the factors do not depend on the accumulator: fetch the first chunks' early (in place:
+      // once the stores of the chunk that last used the buffer have read it)
+      if (kInPlace && lane == 0) bulk_wait_read<AB - 2>();
+      __syncwarp();
       for (int c = 0; c < AB - 1 && c < NCH; ++c) issue_aux(c);
       const bool ready = mbar_wait(&tfull[buf], use & 1u, ctl);
       __syncwarp();
@@ -703,7 +721,11 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
       for (int c = 0; c < NCH; ++c) {
         const uint8_t* aux = nullptr;
         if constexpr (NAUX > 0) {
-          if (c + AB - 1 < NCH) issue_aux(c + AB - 1);
+          if (c + AB - 1 < NCH) {
+            if (kInPlace && lane == 0) bulk_wait_read<AB - 2>();  // that buffer's stores have read it
+            __syncwarp();
+            issue_aux(c + AB - 1);
+          }
           const int db = aux_done % AB;
           const bool got = mbar_wait(&abar[db], (aux_done / AB) & 1u, ctl);
           __syncwarp();
@@ -778,33 +800,41 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
                                              vh[(c4 & 3) * 8 + p * 2 + 1] * bf16_hi(aw[p]));
           }
         } else if constexpr (EPI == kEpiDGate) {
+          // in place: each 16-byte piece of this lane's factor rows becomes the same piece of dG, dU
+          uint8_t* fa = const_cast<uint8_t*>(aux);
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int off = lane * 64 + ((c4 ^ swz) * 16);
-            const uint4 av = *reinterpret_cast<const uint4*>(aux + off);
-            const uint4 bv = *reinterpret_cast<const uint4*>(aux + kOutBox + off);
+          for (int c8 = 0; c8 < CWO / 8; ++c8) {
+            const int off = lane * (2 * CWO) + ((c8 ^ (lane & 7)) * 16);
+            const uint4 av = *reinterpret_cast<const uint4*>(fa + off);
+            const uint4 bv = *reinterpret_cast<const uint4*>(fa + kOutBox + off);
             const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+            const float* vh = c8 < 4 ? v0 : v1;  // resolved at compile time (unrolled)
+            uint32_t gw[4], uw[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-              const float d0 = v0[c4 * 8 + p * 2], d1 = v0[c4 * 8 + p * 2 + 1];
-              w[0][c4 * 4 + p] = pack_bf16x2(d0 * bf16_lo(aw[p]), d1 * bf16_hi(aw[p]));
-              w[1][c4 * 4 + p] = pack_bf16x2(d0 * bf16_lo(bw[p]), d1 * bf16_hi(bw[p]));
+              const float d0 = vh[(c8 & 3) * 8 + p * 2], d1 = vh[(c8 & 3) * 8 + p * 2 + 1];
+              gw[p] = pack_bf16x2(d0 * bf16_lo(aw[p]), d1 * bf16_hi(aw[p]));
+              uw[p] = pack_bf16x2(d0 * bf16_lo(bw[p]), d1 * bf16_hi(bw[p]));
             }
+            *reinterpret_cast<uint4*>(fa + off) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+            *reinterpret_cast<uint4*>(fa + kOutBox + off) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
           }
         }
         // stage this warp's 32-row box of every output, then one lane stores them with TMA
         const int db = OB > 1 ? static_cast<int>(chunks & 1u) : 0;
-        if (lane == 0) bulk_wait_read<OB - 1>();  // the store that last used box db has read it
-        __syncwarp();
+        if constexpr (!kInPlace) {
+          if (lane == 0) bulk_wait_read<OB - 1>();  // the store that last used box db has read it
+          __syncwarp();
 #pragma unroll
-        for (int o = 0; o < NOUT; ++o) {
-          uint8_t* ob = ebase + (o * OB + db) * kOutBox;
+          for (int o = 0; o < NOUT; ++o) {
+            uint8_t* ob = ebase + (o * OB + db) * kOutBox;
 #pragma unroll
-          for (int c4 = 0; c4 < CWO / 8; ++c4) {  // 16-byte pieces of this lane's row, swizzled
-            const int phys = CWO == 64 ? (c4 ^ (lane & 7)) : (c4 ^ swz);
-            *reinterpret_cast<uint4*>(ob + lane * (2 * CWO) + phys * 16) =
-                make_uint4(w[o][c4 * 4], w[o][c4 * 4 + 1], w[o][c4 * 4 + 2], w[o][c4 * 4 + 3]);
+            for (int c4 = 0; c4 < CWO / 8; ++c4) {  // 16-byte pieces of this lane's row, swizzled
+              const int phys = CWO == 64 ? (c4 ^ (lane & 7)) : (c4 ^ swz);
+              *reinterpret_cast<uint4*>(ob + lane * (2 * CWO) + phys * 16) =
+                  make_uint4(w[o][c4 * 4], w[o][c4 * 4 + 1], w[o][c4 * 4 + 2], w[o][c4 * 4 + 3]);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -819,7 +849,8 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
           } else {
 #pragma unroll
             for (int o = 0; o < NOUT; ++o)
-              tma_store_2d(&emaps.o[o], n0, m_slab, ebase + (o * OB + db) * kOutBox);
+              tma_store_2d(&emaps.o[o], n0, m_slab,
+                           kInPlace ? aux + o * kOutBox : ebase + (o * OB + db) * kOutBox);
           }
           bulk_commit();
         }
