@@ -22,6 +22,7 @@ namespace swf {
 namespace {
 
 constexpr int kBucketSmemBytes = 98304;
+constexpr int kBucketRowsSmemBytes = 32768;  // the place kernel stages its group_idx tile up to this
 // The plain-store TMA epilogue's staging boxes: 32 rows x kStoreBoxCols columns, swizzled by
 // the width in bytes (the tensor maps of its outputs must match them).
 constexpr int kStoreBoxCols = tma_epi_cols<kEpiStore>();
@@ -46,7 +47,9 @@ SparseDims dims_of(int64_t M, int64_t d, int64_t f, int32_t G, int32_t K) {
   s.pairs = M * K;
   s.rmax = (int64_t)round_up((size_t)(s.pairs + (int64_t)s.ng * 127), 128);
   s.mblk = (int)(s.rmax / 128);
-  const int words_smem = std::max(1, std::min(32, kBucketSmemBytes / (8 * std::max(1, s.ng))));
+  // the place kernel's shared memory: bitmaps and prefixes (8 ng words bytes) and per-group bases
+  // (8 ng bytes), within kBucketSmemBytes where possible
+  const int words_smem = std::max(1, std::min(32, (kBucketSmemBytes - 8 * s.ng) / (8 * std::max(1, s.ng))));
   const int64_t words_fill = (M + 32 * 296 - 1) / (32 * 296);  // about two blocks per SM
   s.words = (int)std::max<int64_t>(1, std::min<int64_t>(words_smem, words_fill));
   s.tok_blk = 32 * s.words;
@@ -148,9 +151,15 @@ __device__ __forceinline__ bool valid_slot(const int32_t* row, int k, int ng) {
 }
 
 __global__ void bucket_count_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
-                                    int tok_blk, int32_t* __restrict__ counts) {
+                                    int tok_blk, int32_t* __restrict__ counts,
+                                    int32_t* __restrict__ row_token, int64_t rmax) {
   extern __shared__ int32_t hist[];
   for (int c = threadIdx.x; c < ng; c += blockDim.x) hist[c] = 0;
+  // the row -> token table starts as all padding (-1); the place kernel fills the rows in use
+  if (row_token) {
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rmax; r += (int64_t)gridDim.x * blockDim.x)
+      row_token[r] = -1;
+  }
   __syncthreads();
   const int64_t t0 = (int64_t)blockIdx.x * tok_blk;
   for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
@@ -175,20 +184,29 @@ __global__ void bucket_scan_kernel(int32_t* __restrict__ counts, int nblk, int n
   int32_t* tot = sh;            // [ng]
   int32_t* sstart = sh + ng;    // [ng + 1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  constexpr int kBatch = 8;  // 32-block chunks whose counts are loaded together (one latency)
   for (int c = warp; c < ng; c += nwarps) {
     int32_t* row = counts + (int64_t)c * nblk;
     int32_t run = 0;
-    for (int b0 = 0; b0 < nblk; b0 += 32) {
-      const int b = b0 + lane;
-      const int32_t v = b < nblk ? row[b] : 0;
-      int32_t incl = v;
+    for (int b0 = 0; b0 < nblk; b0 += 32 * kBatch) {
+      int32_t v[kBatch];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int32_t n = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += n;
+      for (int j = 0; j < kBatch; ++j) {
+        const int b = b0 + j * 32 + lane;
+        v[j] = b < nblk ? row[b] : 0;
       }
-      if (b < nblk) row[b] = run + incl - v;
-      run += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int b = b0 + j * 32 + lane;
+        int32_t incl = v[j];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += n;
+        }
+        if (b < nblk) row[b] = run + incl - v[j];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
     if (lane == 0) tot[c] = run;
   }
@@ -245,25 +263,38 @@ __global__ void bucket_scan_kernel(int32_t* __restrict__ counts, int nblk, int n
 
 // Places every valid (token, group) pair: rank among the block's tokens of the same group from
 // a per-group bitmap of the block's tokens, so the order within a group is ascending token id.
+// The block's group_idx rows and, per group, its base (CSR offset + the block's scanned count)
+// and padded segment start are staged in shared memory first, so the placement itself makes no
+// dependent global loads.
 __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, int K, int ng,
                                     int words, const int32_t* __restrict__ counts,
                                     const int32_t* __restrict__ offs, int32_t* __restrict__ tokens,
                                     const int32_t* __restrict__ seg_start,
                                     int32_t* __restrict__ row_token,
-                                    int32_t* __restrict__ pair_row) {
+                                    int32_t* __restrict__ pair_row, int stage_rows) {
   extern __shared__ uint32_t smem_bits[];
-  uint32_t* bits = smem_bits;                                        // [ng][words]
-  int32_t* pre = reinterpret_cast<int32_t*>(smem_bits + (size_t)ng * words);  // [ng][words]
   const int tok_blk = 32 * words;
-  for (int i = threadIdx.x; i < ng * words; i += blockDim.x) bits[i] = 0;
-  __syncthreads();
+  uint32_t* bits = smem_bits;                                           // [ng][words]
+  int32_t* pre = reinterpret_cast<int32_t*>(smem_bits + (size_t)ng * words);  // [ng][words]
+  int32_t* base_tok = pre + (size_t)ng * words;                         // [ng]
+  int32_t* base_row = base_tok + ng;                                    // [ng]
+  int32_t* rows_smem = base_row + ng;                                   // [tok_blk * K] if staged
   const int64_t t0 = (int64_t)blockIdx.x * tok_blk;
-  for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
-    const int tl = i / K;
-    const int64_t t = t0 + tl;
-    if (t >= M) break;
-    const int32_t* row = idx + t * K;
-    const int k = i % K;
+  const int64_t left = M - t0;
+  const int nslots = (int)(left < tok_blk ? left : (int64_t)tok_blk) * K;
+  for (int i = threadIdx.x; i < ng * words; i += blockDim.x) bits[i] = 0;
+  if (stage_rows)
+    for (int i = threadIdx.x; i < nslots; i += blockDim.x) rows_smem[i] = idx[t0 * K + i];
+  const int32_t* rows = stage_rows ? rows_smem : idx + t0 * K;
+  for (int c = threadIdx.x; c < ng; c += blockDim.x) {
+    const int32_t cb = counts[(int64_t)c * gridDim.x + blockIdx.x];
+    base_tok[c] = offs[c] + cb;
+    base_row[c] = seg_start ? seg_start[c] + cb : 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
+    const int tl = i / K, k = i % K;
+    const int32_t* row = rows + tl * K;
     if (valid_slot(row, k, ng)) atomicOr(&bits[row[k] * words + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
@@ -275,12 +306,10 @@ __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, 
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < tok_blk * K; i += blockDim.x) {
-    const int tl = i / K;
+  for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
+    const int tl = i / K, k = i % K;
     const int64_t t = t0 + tl;
-    if (t >= M) break;
-    const int32_t* row = idx + t * K;
-    const int k = i % K;
+    const int32_t* row = rows + tl * K;
     if (!valid_slot(row, k, ng)) {
       if (pair_row) pair_row[t * K + k] = -1;
       continue;
@@ -288,16 +317,10 @@ __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, 
     const int c = row[k];
     const int w = tl >> 5;
     const int rank = pre[c * words + w] + __popc(bits[c * words + w] & ((1u << (tl & 31)) - 1u));
-    const int32_t base = counts[(int64_t)c * gridDim.x + blockIdx.x] + rank;
-    tokens[offs[c] + base] = (int32_t)t;
-    if (row_token) row_token[seg_start[c] + base] = (int32_t)t;
-    if (pair_row) pair_row[t * K + k] = seg_start[c] + base;
+    tokens[base_tok[c] + rank] = (int32_t)t;
+    if (row_token) row_token[base_row[c] + rank] = (int32_t)t;
+    if (pair_row) pair_row[t * K + k] = base_row[c] + rank;
   }
-}
-
-__global__ void fill_i32_kernel(int32_t* __restrict__ p, int64_t n, int32_t v) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = v;
 }
 
 // out[t, :] = sum over t's valid slots k (in slot order) of rows[pair_row[t*K + k], :], fp32
@@ -430,7 +453,8 @@ swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts,
                        int32_t* tile_group, int32_t* row_token, int32_t* pair_row, cudaStream_t st) {
   {
     ProfScope prof(SWF_K_BUCKETS, st);
-    bucket_count_kernel<<<s.nblk, 256, s.ng * sizeof(int32_t), st>>>(idx, s.M, s.K, s.ng, s.tok_blk, counts);
+    bucket_count_kernel<<<s.nblk, 256, s.ng * sizeof(int32_t), st>>>(idx, s.M, s.K, s.ng, s.tok_blk, counts,
+                                                                    row_token, s.rmax);
     if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
   }
   const size_t scan_smem = (2 * (size_t)s.ng + 1) * sizeof(int32_t);
@@ -443,17 +467,14 @@ swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts,
                                                    tile_group, s.mblk);
     if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
   }
-  if (row_token) {
-    ProfScope prof(SWF_K_ELEMENTWISE, st);
-    fill_i32_kernel<<<grid_for(s.rmax, 256), 256, 0, st>>>(row_token, s.rmax, -1);
-    if (launched() != SWF_OK) return SWF_ERR_LAUNCH;
-  }
-  const size_t place_smem = (size_t)8 * s.ng * s.words;
+  const size_t rows_bytes = (size_t)4 * s.tok_blk * s.K;
+  const int stage_rows = rows_bytes <= (size_t)kBucketRowsSmemBytes ? 1 : 0;
+  const size_t place_smem = (size_t)8 * s.ng * s.words + (size_t)8 * s.ng + (stage_rows ? rows_bytes : 0);
   if (cudaFuncSetAttribute(bucket_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)place_smem) != cudaSuccess)
     return SWF_ERR_LAUNCH;
   ProfScope prof(SWF_K_BUCKETS, st);
   bucket_place_kernel<<<s.nblk, 256, place_smem, st>>>(idx, s.M, s.K, s.ng, s.words, counts, offs,
-                                                       tokens, seg_start, row_token, pair_row);
+                                                       tokens, seg_start, row_token, pair_row, stage_rows);
   return launched();
 }
 
@@ -532,7 +553,7 @@ void sparse_plan(int op, int64_t M, int64_t d, int64_t f, int32_t G, int32_t K, 
       p->gemm_tiles = (int64_t)cdiv(M, 128) * cdiv((int64_t)s.ng * P, 256);
       break;
     case SWF_OP_SPARSE_FWD:
-      p->num_kernels = 7;  // bucketing (count, scan, fill, place), gate|up, down, pair sum
+      p->num_kernels = 6;  // bucketing (count with the row -> token fill, scan, place), gate|up, down, pair sum
       p->flops = 6 * M * d * (int64_t)K * G;
       p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256));
       p->tile_n = 2 * G;
@@ -941,6 +962,22 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_DGATE, twd, twd, twd, a, st);
     if (s != SWF_OK) return s;
   }
+  {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ X rows of the segment (gathered from x)
+    CUtensorMap tdgu;
+    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64)) return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(128, d, 256, 0);
+    a.n_groups = sd.ng;
+    a.seg_start = v.seg_start;
+    a.seg_rows = v.seg_rows;
+    a.kb_seg0 = 1 << 30;
+    a.group_size = G;
+    a.out0 = dw_gate;
+    a.out1 = dw_up;
+    a.ld_out = d;
+    set_gather(a, v.row_token, x, d);
+    s = launch_tc<256, true, true, false, kEpiGroupDWgu, kModeKGrouped, false, kGatherB>(SWF_K_SPARSE_DW, tdgu, tdgu, tdgu, a, st);
+    if (s != SWF_OK) return s;
+  }
   {  // dxc[r] = dG_row W_g[g] + dU_row W_u[g]
     CUtensorMap tdgu, twg, twu;
     if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 128) ||
@@ -958,22 +995,6 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     if (s != SWF_OK) return s;
   }
   if ((s = run_pair_sum(w.dxc, v.pair_row, sd, dx, st)) != SWF_OK) return s;
-  {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ X rows of the segment (gathered from x)
-    CUtensorMap tdgu;
-    if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64)) return SWF_ERR_LAUNCH;
-    TcGemmArgs a = base_args(128, d, 256, 0);
-    a.n_groups = sd.ng;
-    a.seg_start = v.seg_start;
-    a.seg_rows = v.seg_rows;
-    a.kb_seg0 = 1 << 30;
-    a.group_size = G;
-    a.out0 = dw_gate;
-    a.out1 = dw_up;
-    a.ld_out = d;
-    set_gather(a, v.row_token, x, d);
-    s = launch_tc<256, true, true, false, kEpiGroupDWgu, kModeKGrouped, false, kGatherB>(SWF_K_SPARSE_DW, tdgu, tdgu, tdgu, a, st);
-    if (s != SWF_OK) return s;
-  }
   {  // per group: dW_d[:, g] = (dY rows of the segment)ᵀ h_seg, the dY rows gathered from dy
     CUtensorMap th;
     if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64)) return SWF_ERR_LAUNCH;
