@@ -323,11 +323,18 @@ __global__ void bucket_place_kernel(const int32_t* __restrict__ idx, int64_t M, 
   }
 }
 
+// Drops a 128-byte line from L2 without writing it back (its contents become undefined).
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 // out[t, :] = sum over t's valid slots k (in slot order) of rows[pair_row[t*K + k], :], fp32
 // accumulation, bf16 result: the deterministic reduction of the per-pair contributions.  One
 // warp per token; each lane issues the (up to 8) row loads of a slot chunk before summing them.
+// With discard set (rows whose length is a multiple of 128 bytes), the lines a warp has read are
+// dropped from L2 afterwards: each belongs to one (token, group) pair and is read only here.
 __global__ void pair_sum_kernel(const uint4* __restrict__ rows, const int32_t* __restrict__ pair_row,
-                                int64_t M, int K, int64_t row_vecs, uint4* __restrict__ out) {
+                                int64_t M, int K, int64_t row_vecs, uint4* __restrict__ out, int discard) {
   constexpr int kChunk = 8;
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -354,6 +361,17 @@ __global__ void pair_sum_kernel(const uint4* __restrict__ rows, const int32_t* _
       }
       out[t * row_vecs + v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+      if (discard) {
+        // The 8 lanes of each 128-byte line read it in this iteration (row_vecs is a multiple of
+        // 8); the lanes still in the loop are the first min(32, row_vecs - (v - lane)).
+        const int64_t left = row_vecs - (v - lane);
+        __syncwarp(left >= 32 ? 0xffffffffu : ((1u << left) - 1u));
+        if ((v & 7) == 0)
+          for (int k = 0; k < K; ++k) {
+            const int32_t r = pr[k];
+            if (r >= 0) discard_l2_line(rows + (int64_t)r * row_vecs + v);
+          }
+      }
     }
   }
 }
@@ -478,11 +496,15 @@ swf_status run_buckets(const int32_t* idx, const SparseDims& s, int32_t* counts,
   return launched();
 }
 
+// The per-token sums.  Each per-pair row is read once, so when rows are whole 128-byte lines the
+// lines are dropped from L2 after they are read instead of being written back to DRAM.
 swf_status run_pair_sum(const void* rows, const int32_t* pair_row, const SparseDims& s, void* out,
                         cudaStream_t st) {
   ProfScope prof(SWF_K_PAIR_SUM, st);
+  // a line may be dropped only when no other row shares it
+  const int discard = ((s.d * 2) % 128 == 0 && (reinterpret_cast<uintptr_t>(rows) & 127) == 0) ? 1 : 0;
   pair_sum_kernel<<<grid_for(s.M, 8), 256, 0, st>>>(static_cast<const uint4*>(rows), pair_row, s.M, s.K,
-                                                   s.d / 8, static_cast<uint4*>(out));
+                                                   s.d / 8, static_cast<uint4*>(out), discard);
   return launched();
 }
 

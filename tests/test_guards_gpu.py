@@ -137,6 +137,7 @@ def check_sparse_outputs(g, inp, idx, G):
     (513, 48, 1024, 64, 5, 8),    # ragged M, d below one k-block
     (1, 64, 256, 16, 2, None),    # one token, exact energies
     (300, 272, 768, 32, 24, 3),   # K = all groups
+    (2048, 2048, 4096, 64, 8, 8),  # per-pair rows of whole 128-byte lines (dropped from L2 once summed)
 ])
 def test_selection_and_sparse_write_only_their_buffers(M, d, f, G, K, spg):
     inp = synth.dense_inputs(M, d, f, seed=M + G, dtype=torch.bfloat16)
