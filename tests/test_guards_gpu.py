@@ -221,6 +221,41 @@ def test_invalid_group_idx_refused_in_debug_mode_and_dropped_otherwise():
         api.set_debug(prev)
 
 
+def test_tokens_without_valid_slots_get_zero_rows_and_runs_repeat_bitwise():
+    """Whole 64-token chunks and a few single tokens whose every slot is out of range: the
+    bucketing drops them, so the per-token sums of the down and dx GEMMs never hear of them and
+    must still write their zero rows.  The rest must match the oracle on the valid tokens alone,
+    and a second run must reproduce every output bit for bit (the sums take a fixed order
+    whichever CTA ends up summing a chunk)."""
+    M, d, f, G, K = 300, 256, 1024, 64, 4
+    ng = f // G
+    rng = np.random.default_rng(7)
+    idx = np.sort(np.stack([rng.choice(ng, size=K, replace=False) for _ in range(M)]), axis=1).astype(np.int32)
+    dead = np.zeros(M, bool)
+    dead[64:192] = True       # chunks 1 and 2
+    dead[250:260] = True      # part of a chunk
+    dead[M - 1] = True        # the last token
+    idx[dead] = -1
+    inp = synth.dense_inputs(M, d, f, seed=11, dtype=torch.bfloat16)
+    idx_dev = torch.from_numpy(idx).cuda()
+    g1 = sparse_guarded_step(inp, idx_dev, G, K)
+    assert_guards(g1, "sparse with empty tokens")
+    g2 = sparse_guarded_step(inp, idx_dev, G, K)
+    assert_guards(g2, "sparse with empty tokens, second run")
+    for k in ("y", "dx", "dwg", "dwu", "dwd"):
+        assert torch.equal(g1[k].t, g2[k].t), f"{k} differs between two runs"
+    for k in ("y", "dx"):
+        assert torch.count_nonzero(g1[k].t[torch.from_numpy(dead).cuda()]).item() == 0, f"{k} rows of empty tokens"
+    live = ~dead
+    x, wg, wu, wd, dy = (f64(inp[k]) for k in ("x", "w_gate", "w_up", "w_down", "dy"))
+    fw = O.sparse_forward(x[live], wg, wu, wd, idx[live], G)
+    bw = O.sparse_backward(x[live], wg, wu, wd, idx[live], G, dy[live])
+    assert_close("y", f64(g1["y"].t)[live], fw["y"], torch.bfloat16)
+    assert_close("dx", f64(g1["dx"].t)[live], bw["dx"], torch.bfloat16)
+    for k, ref in (("dwg", "dw_gate"), ("dwu", "dw_up"), ("dwd", "dw_down")):
+        assert_close(k, f64(g1[k].t), bw[ref], torch.bfloat16)
+
+
 def test_flashffn_core_and_prologue_write_only_their_buffers():
     T, H, dh, E, de = 300, 2, 128, 3, 128
     bf = torch.bfloat16
