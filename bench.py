@@ -42,7 +42,8 @@ from swiglu_feed_forward_b200 import synth  # noqa: E402
 METRIC = "SwiGLU FFN fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 tensor peak"
 WORKLOAD = 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Algorithmic FLOPs of one launch of each dense kernel, in units of M * d_model * d_ff.
+# Algorithmic FLOPs of each dense kernel in one step (all of its launches: a weight-gradient GEMM may
+# run as two, its whole waves and its K-split last wave), in units of M * d_model * d_ff.
 KERNEL_FLOP_UNITS = {"gate_up_swiglu": 4, "gate_up_swiglu_infer": 4, "down_proj": 2, "dgate": 2,
                      "dx": 4, "dw_gate_up": 4, "dw_down": 2}
 KERNEL_SOURCES = ["swiglu_feed_forward_b200/csrc/swf_tc_gemm.cuh",
@@ -129,8 +130,8 @@ def source_sha(read=None, files=None):
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when absent or
-    taken on other kernel sources."""
+    """DRAM bytes of `kernel` in one step (all of its launches) from the committed ncu summary, or
+    None when absent or taken on other kernel sources."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -139,7 +140,7 @@ def ncu_traffic(kernel):
     e = d.get(kernel)
     if not e or e.get("source_sha") != source_sha():
         return None
-    return e.get("dram_bytes_per_launch")
+    return e.get("dram_bytes_per_step")
 
 
 # ------------------------------------------------------------------ clocks
@@ -726,8 +727,8 @@ def run_ours(args, world, rank, local):
     total_k = sum(v for _, v in kern.values()) or 1.0
     dom = max(kern.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_n, dom_ms) = dom
-    dom_flops = KERNEL_FLOP_UNITS.get(dom_name, 0) * M * d * f
-    achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12
+    dom_flops = KERNEL_FLOP_UNITS.get(dom_name, 0) * M * d * f  # per step
+    achieved = dom_flops / (dom_ms / args.steps / 1e3) / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak, peak_kind = choose_peak(ms / 1e3, peak_burst, peak_sus, peak_src)
@@ -736,14 +737,16 @@ def run_ours(args, world, rank, local):
                 "peak_kind": peak_kind,
                 "frac_of_burst_peak": round(achieved / peak_burst, 4),
                 "frac_of_sustained_peak": round(achieved / peak_sus, 4),
-                "flops_per_launch": dom_flops, "launches": dom_n,
+                "flops_per_step": dom_flops, "launches": dom_n,
+                "launches_per_step": round(dom_n / args.steps, 2),
+                "ms_per_step": round(dom_ms / args.steps, 4),
                 "avg_launch_ms": round(dom_ms / dom_n, 4),
                 "timed_region_s": round(ms / 1e3, 4),
                 "traffic": ncu_traffic(dom_name)}
     kernels = {k: {"launches": n, "ms_total": round(v, 3), "share": round(v / total_k, 4),
-                   "avg_ms": round(v / n, 4),
-                   **({"tflops": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / n / 1e3) / 1e12, 1),
-                       "frac_of_burst_peak": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / n / 1e3) / 1e12
+                   "avg_ms": round(v / n, 4), "ms_per_step": round(v / args.steps, 4),
+                   **({"tflops": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / args.steps / 1e3) / 1e12, 1),
+                       "frac_of_burst_peak": round(KERNEL_FLOP_UNITS[k] * M * d * f / (v / args.steps / 1e3) / 1e12
                                                    / peak_burst, 4)}
                       if k in KERNEL_FLOP_UNITS else {})}
                for k, (n, v) in sorted(kern.items(), key=lambda kv: -kv[1][1])}

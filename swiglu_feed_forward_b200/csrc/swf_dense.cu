@@ -47,12 +47,90 @@ __global__ void splitk_reduce_kernel(const float4* __restrict__ part, int64_t pl
   }
 }
 
-// K splits the planner gives a weight-gradient GEMM of rows x cols over K (pair tiles 256 x 256).
-int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
-  const int64_t tiles = (int64_t)cdiv(rows, 2 * kTileM) * cdiv(cols, cols <= 128 ? 128 : 256);
+// How a weight-gradient GEMM of rows x cols over K (pair tiles 256 x BN) is scheduled:
+//   uniform K split into ks planes (ks = 1: direct bf16 stores), or
+//   hybrid: the first `head` output tiles (whole waves of the 74 clusters) with direct stores,
+//   and the remaining ones in a second launch split ks ways along K into fp32 partial planes,
+//   summed per tile by splitk_reduce_tiles_kernel.
+// A persistent launch of n tiles takes ceil(n / 74) tile times, so 344 tiles take 5 where 4.65
+// would do; splitting only the last, partial wave recovers most of that without the partial
+// traffic of a uniform split.  Costs are the same model as choose_ksplit (k-block time, partial
+// bytes at HBM speed), plus a launch for the tail and its reduction.
+struct DwPlan {
+  int ks;    // uniform split (hybrid: the tail's split)
+  int head;  // hybrid: output tiles of the first launch (0: uniform)
+  int tiles, bn;
+};
+
+DwPlan dw_plan(int64_t rows, int64_t cols, int64_t K) {
+  constexpr double kClusters = 74.0, kKblockUs = 0.27, kBytesPerUs = 5.0e6, kLaunchUs = 6.0;
+  DwPlan p{};
+  p.bn = cols <= 128 ? 128 : 256;
+  p.tiles = cdiv(rows, 2 * kTileM) * cdiv(cols, p.bn);
   const int kb = cdiv(K, kTileK);
-  const int ks = choose_ksplit(tiles, kb, rows * cols);
-  return ks > 1 ? cdiv(kb, cdiv(kb, ks)) : 1;  // no empty trailing split
+  const int ks = choose_ksplit(p.tiles, kb, rows * cols);
+  p.ks = ks > 1 ? cdiv(kb, cdiv(kb, ks)) : 1;  // no empty trailing split
+  p.head = 0;
+  auto uniform_us = [&](int k) {
+    const double per = std::ceil((double)kb / k);
+    const double us = std::ceil(p.tiles * k / kClusters) * per * kKblockUs;
+    return k > 1 ? us + (8.0 * k * rows * cols + 2.0 * rows * cols) / kBytesPerUs + kLaunchUs : us;
+  };
+  double best = uniform_us(p.ks);
+  const int waves = (int)(p.tiles / kClusters), tail = p.tiles - waves * (int)kClusters;
+  if (waves >= 1 && tail > 0) {
+    const double tile_elems = 2.0 * kTileM * p.bn;
+    for (int k = 2; k <= 16 && kb / k >= 8; ++k) {
+      const double per = std::ceil((double)kb / k);
+      const double us = waves * kb * kKblockUs + std::ceil(tail * k / kClusters) * per * kKblockUs +
+                        (8.0 * k * tail * tile_elems + 2.0 * tail * tile_elems) / kBytesPerUs + 2 * kLaunchUs;
+      if (us < best) {
+        best = us;
+        p.ks = k;
+        p.head = waves * (int)kClusters;
+      }
+    }
+  }
+  return p;
+}
+
+// The tail tiles [tile0, tile0 + ntiles) of a hybrid weight-gradient GEMM (pair tiles of 256 x BN,
+// raster order as the GEMM's): out = bf16(sum over splits s = 0, 1, ... of part[s]) in that order;
+// rows at or past row_split go to out1 (row - row_split).  8 elements per thread.
+__global__ void splitk_reduce_tiles_kernel(const float* __restrict__ part, int64_t plane, int ks, int64_t rows,
+                                           int64_t cols, int64_t row_split, __nv_bfloat16* __restrict__ out0,
+                                           __nv_bfloat16* __restrict__ out1, int num_m_blk, int num_n_blk,
+                                           int raster, int tile0, int ntiles, int bn) {
+  const int per_tile = 2 * kTileM * bn / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)ntiles * per_tile;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int lt = (int)(i / per_tile), e = (int)(i - (int64_t)lt * per_tile) * 8;
+    int mb, nb;
+    tile_coords(tile0 + lt, num_m_blk, num_n_blk, raster, mb, nb);
+    const int64_t m = (int64_t)mb * 2 * kTileM + e / bn, n = (int64_t)nb * bn + e % bn;
+    if (m >= rows || n >= cols) continue;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const float* src = part + m * cols + n;
+    for (int s0 = 0; s0 < ks; s0 += 4) {  // the loads of up to four splits in flight, summed in order
+      float4 a[4], b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool in = s0 + j < ks;
+        const float4* p4 = reinterpret_cast<const float4*>(src + (int64_t)(in ? s0 + j : s0) * plane);
+        a[j] = in ? p4[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+        b[j] = in ? p4[1] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (s0 + j >= ks) break;
+        acc[0] += a[j].x, acc[1] += a[j].y, acc[2] += a[j].z, acc[3] += a[j].w;
+        acc[4] += b[j].x, acc[5] += b[j].y, acc[6] += b[j].z, acc[7] += b[j].w;
+      }
+    }
+    __nv_bfloat16* dst = m < row_split ? out0 + m * cols + n : out1 + (m - row_split) * cols + n;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
 }
 
 }  // namespace
@@ -60,44 +138,51 @@ int dw_ksplit(int64_t rows, int64_t cols, int64_t K) {
 swf_status splitk_reduce(const float* part, int ks, int64_t rows, int64_t cols, int64_t row_split,
                          void* out0, void* out1, cudaStream_t st);
 
-// Weight-gradient GEMM (both operands MN-major, K = tokens): split-K into fp32 partial planes
-// plus a fixed-order reduction when the planner finds too few output tiles, else direct stores.
+// Weight-gradient GEMM (both operands MN-major, K = tokens), scheduled as dw_plan says: direct
+// stores, a uniform K split into fp32 partial planes plus a fixed-order reduction, or the hybrid
+// of the two (whole waves direct, the last partial wave split).
+template <int BN>
+swf_status launch_dw_bn(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int64_t cols,
+                        int64_t K, void* out0, void* out1, int64_t row_split, float* part, const DwPlan& p,
+                        cudaStream_t st) {
+  TcGemmArgs a = base_args(rows, cols, BN, K, 2 * kTileM);
+  a.out0 = out0;
+  a.out1 = out1;
+  a.row_split = (int)row_split;
+  a.ld_out = cols;
+  if (p.ks <= 1) return launch_tc_pair<BN, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st);
+  swf_status s = SWF_OK;
+  if (p.head > 0) {  // whole waves: direct stores
+    a.tile_count = p.head;
+    if ((s = launch_tc_pair<BN, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st)) != SWF_OK) return s;
+    a.tile_offset = p.head;
+    a.tile_count = p.tiles - p.head;
+  }
+  a.ksplit = p.ks;
+  a.kb_per_split = cdiv(a.kb_total, p.ks);
+  a.part = part;
+  a.part_plane = rows * cols;
+  if ((s = launch_tc_pair<BN, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st)) != SWF_OK)
+    return s;
+  if (p.head == 0) return splitk_reduce(part, p.ks, rows, cols, row_split, out0, out1, st);
+  ProfScope prof(SWF_K_SPLITK_REDUCE, st);
+  const int ntail = p.tiles - p.head;
+  const int64_t work = (int64_t)ntail * 2 * kTileM * BN / 8;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 148 * 16));
+  splitk_reduce_tiles_kernel<<<grid, 256, 0, st>>>(part, rows * cols, p.ks, rows, cols, row_split,
+                                                   static_cast<__nv_bfloat16*>(out0),
+                                                   static_cast<__nv_bfloat16*>(out1), a.num_m_blk, a.num_n_blk,
+                                                   std::max(1, std::min(a.raster, a.num_m_blk)), p.head, ntail, BN);
+  return cudaGetLastError() == cudaSuccess ? SWF_OK : SWF_ERR_LAUNCH;
+}
+
 swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
                      int64_t cols, int64_t K, void* out0, void* out1, int64_t row_split,
                      float* part, cudaStream_t st) {
-  const int ks = dw_ksplit(rows, cols, K);
-  if (cols <= 128) {  // narrow outputs: pair tiles of 256 x 128
-    TcGemmArgs a = base_args(rows, cols, 128, K, 2 * kTileM);
-    if (ks <= 1) {
-      a.out0 = out0;
-      a.out1 = out1;
-      a.row_split = (int)row_split;
-      a.ld_out = cols;
-      return launch_tc_pair<128, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st);
-    }
-    a.ksplit = ks;
-    a.kb_per_split = cdiv(a.kb_total, ks);
-    a.part = part;
-    a.part_plane = rows * cols;
-    swf_status s = launch_tc_pair<128, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st);
-    if (s != SWF_OK) return s;
-    return splitk_reduce(part, ks, rows, cols, row_split, out0, out1, st);
-  }
-  TcGemmArgs a = base_args(rows, cols, 256, K, 2 * kTileM);
-  if (ks <= 1) {
-    a.out0 = out0;
-    a.out1 = out1;
-    a.row_split = (int)row_split;
-    a.ld_out = cols;
-    return launch_tc_pair<256, true, true, false, kEpiStore>(kind, ta, tb, tb, EpiMaps{}, a, st);
-  }
-  a.ksplit = ks;
-  a.kb_per_split = cdiv(a.kb_total, ks);
-  a.part = part;
-  a.part_plane = rows * cols;
-  swf_status s = launch_tc_pair<256, true, true, false, kEpiPartialF32>(kind, ta, tb, tb, EpiMaps{}, a, st);
-  if (s != SWF_OK) return s;
-  return splitk_reduce(part, ks, rows, cols, row_split, out0, out1, st);
+  const DwPlan p = dw_plan(rows, cols, K);
+  if (p.bn == 128)  // narrow outputs: pair tiles of 256 x 128
+    return launch_dw_bn<128>(kind, ta, tb, rows, cols, K, out0, out1, row_split, part, p, st);
+  return launch_dw_bn<256>(kind, ta, tb, rows, cols, K, out0, out1, row_split, part, p, st);
 }
 
 swf_status splitk_reduce(const float* part, int ks, int64_t rows, int64_t cols, int64_t row_split,
@@ -113,8 +198,8 @@ swf_status splitk_reduce(const float* part, int ks, int64_t rows, int64_t cols, 
 }
 
 int64_t part_elems(int64_t rows, int64_t cols, int64_t K) {
-  const int ks = dw_ksplit(rows, cols, K);
-  return ks > 1 ? ks * rows * cols : 0;
+  const DwPlan p = dw_plan(rows, cols, K);
+  return p.ks > 1 ? p.ks * rows * cols : 0;
 }
 
 int64_t dense_bwd_part_elems(int64_t M, int64_t d, int64_t f) {

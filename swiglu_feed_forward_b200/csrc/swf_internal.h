@@ -74,7 +74,8 @@ swf_status mlp2_bwd_f32(const float* dy, const float* x, const float* wu, const 
 
 // Weight-gradient GEMM out = A^T B of rows x cols over K (tokens), both operands MN-major (maps
 // with 64 x 64 boxes), as pair tiles of 256 x 256; split-K into `part` (part_elems(...) fp32) and
-// a fixed-order reduction when the planner finds too few tiles.  Rows >= row_split go to out1.
+// a fixed-order reduction when the planner finds too few tiles (of the whole GEMM, or of its last
+// partial wave only).  Rows >= row_split go to out1.
 swf_status launch_dw(int kind, const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
                      int64_t cols, int64_t K, void* out0, void* out1, int64_t row_split,
                      float* part, cudaStream_t st);

@@ -47,8 +47,10 @@ swf_status launch_tc_pair(int kind, const CUtensorMap& ta, const CUtensorMap& tb
   DevCtx ctx;
   swf_status s = get_ctx(&ctx);
   if (s != SWF_OK) return s;
-  const int64_t tiles = (int64_t)args.num_m_blk * args.num_n_blk * std::max(1, args.ksplit);
-  if (tiles == 0) return SWF_OK;
+  const int64_t tiles = (args.tile_count > 0 ? (int64_t)args.tile_count
+                                              : (int64_t)args.num_m_blk * args.num_n_blk - args.tile_offset) *
+                        std::max(1, args.ksplit);
+  if (tiles <= 0) return SWF_OK;
   if (tiles > INT32_MAX) return SWF_ERR_UNSUPPORTED;
   args.status = ctx.status;
   if (args.wait_limit_ns == 0) args.wait_limit_ns = kDefaultWaitNs;

@@ -131,6 +131,8 @@ struct TcGemmArgs {
   int sel_k;
   int unit;               // tiles a CTA takes back to back (<= 1: one); tile ids are unit-major
   int ksplit;             // kModeDense: K splits per output tile (1: none)
+  int tile_offset;        // kModeDense: first output tile (raster order) of this launch
+  int tile_count;         //   output tiles of this launch (0: all from tile_offset)
   int kb_per_split;       //   k-blocks of each split (the last may be shorter)
   float* part;            // kEpiPartialF32: [ksplit][M][N] fp32 partial sums
   int64_t part_plane;     //   elements per split (M * N)
@@ -275,6 +277,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const TcGemmArgs& a) {
       t.ks = tile % a.ksplit;
       tile /= a.ksplit;
     }
+    if (MODE == kModeDense) tile += a.tile_offset;
     tile_coords(tile, a.num_m_blk, a.num_n_blk, a.raster, t.mb, t.nb);
     t.grp = MODE == kModeRowGrouped ? a.tile_group[t.mb] : 0;
     const int g = t.grp < 0 ? 0 : t.grp;
@@ -424,7 +427,8 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
   const int lane = threadIdx.x & 31;
   const int num_tiles = MODE == kModeKGrouped
                             ? args.num_m_blk * args.num_n_blk * args.n_groups
-                            : args.num_m_blk * args.num_n_blk * (args.ksplit > 1 ? args.ksplit : 1);
+                            : (args.tile_count > 0 ? args.tile_count : args.num_m_blk * args.num_n_blk - args.tile_offset) *
+                                  (args.ksplit > 1 ? args.ksplit : 1);
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;

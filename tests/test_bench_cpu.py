@@ -41,10 +41,10 @@ def test_committed_traffic_matches_current_code():
             else:
                 assert got is None
             continue
-        assert e["dram_bytes_per_launch"] > 0
+        assert e["dram_bytes_per_step"] > 0
         assert os.path.exists(os.path.join(bench.ROOT, "profiles", e["from"].split()[0])), e["from"]
         if e["source_sha"] == bench.source_sha():
-            assert bench.ncu_traffic(name) == e["dram_bytes_per_launch"]
+            assert bench.ncu_traffic(name) == e["dram_bytes_per_step"]
         else:
             assert bench.ncu_traffic(name) is None
 
