@@ -920,12 +920,19 @@ extern "C" swf_status sparse_swiglu_ffn_fwd(const void* x, const void* w_gate, c
     a.aux1 = v.b;
     a.ld_aux = G;
     set_gather(a, v.row_token, x, d);
+    // G >= 32: h, a, b leave through 32-row x 32-column staging boxes and TMA stores (whole
+    // 64-byte row pieces) instead of each thread's 16-byte stores into 32 different rows
+    EpiMaps em{};
+    if (G >= 32 && (!encode_tmap_bf16(&em.o[0], v.h, G, sd.rmax, G, 32, 32, 64) ||
+                    !encode_tmap_bf16(&em.o[1], v.a, G, sd.rmax, G, 32, 32, 64) ||
+                    !encode_tmap_bf16(&em.o[2], v.b, G, sd.rmax, G, 32, 32, 64)))
+      return SWF_ERR_LAUNCH;
     if (G == 16)
       s = launch_tc<32, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
     else if (G == 32)
-      s = launch_tc<64, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
+      s = launch_tc<64, false, false, true, kEpiSwiGLU, kModeRowGrouped, true, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st, em);
     else
-      s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st);
+      s = launch_tc<128, false, false, true, kEpiSwiGLU, kModeRowGrouped, true, kGatherA>(SWF_K_SPARSE_UP, twg, twg, twu, a, st, em);
     if (s != SWF_OK) return s;
   }
   {  // down per group: yc[r] = h_row W_d[:, g*G .. g*G+G]^T
@@ -981,7 +988,16 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     a.aux1 = v.b;
     a.ld_aux = G;
     set_gather(a, v.row_token, dy, d);
-    s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped, false, kGatherA>(SWF_K_SPARSE_DGATE, twd, twd, twd, a, st);
+    // the factors a, b come in and dG, dU leave as 32-row x 64-column boxes by TMA, dG and dU
+    // computed in place in the factor boxes (columns G .. 64 read as zero and are stored as zero)
+    EpiMaps em{};
+    if (!encode_tmap_bf16(&em.o[0], w.dgu, 64, sd.rmax, 128, 64, 32, 128) ||
+        !encode_tmap_bf16(&em.o[1], w.dgu + 64, 64, sd.rmax, 128, 64, 32, 128) ||
+        !encode_tmap_bf16(&em.o[2], v.a, G, sd.rmax, G, 64, 32, 128) ||
+        !encode_tmap_bf16(&em.o[3], v.b, G, sd.rmax, G, 64, 32, 128))
+      return SWF_ERR_LAUNCH;
+    s = launch_tc<64, false, true, false, kEpiDGate, kModeRowGrouped, true, kGatherA>(SWF_K_SPARSE_DGATE, twd, twd, twd, a,
+                                                                                        st, em);
     if (s != SWF_OK) return s;
   }
   {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ X rows of the segment (gathered from x)

@@ -408,8 +408,11 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
   static_assert(!TMA_EPI || (MODE == kModeDense && (EPI == kEpiStore || EPI == kEpiSwiGLU ||
                                                     EPI == kEpiSwiGLUInf || EPI == kEpiDGate ||
                                                     EPI == kEpiScale || EPI == kEpiLeakySq)) ||
-                    (MODE == kModeRowGrouped && EPI == kEpiStore),
-                "TMA epilogue: dense bf16 outputs, or row-grouped plain stores");
+                    (MODE == kModeRowGrouped && (EPI == kEpiStore || EPI == kEpiSwiGLU || EPI == kEpiDGate)),
+                "TMA epilogue: dense bf16 outputs, or row-grouped plain / SwiGLU / gating stores");
+  // each gather warp owns whole ring stages: more warps than stages would let two of them wait on
+  // the same stage's barriers one phase apart
+  static_assert(GATHER == kGatherNone || S >= kGatherWarps, "a ring stage per gather warp");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

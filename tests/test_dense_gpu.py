@@ -93,6 +93,28 @@ def test_workload2_full_size_sampled():
     assert_close("dw_down[:,cols]", f64(out["dw_down"])[:, cols], sub["dw_down"], torch.bfloat16)
 
 
+def test_weight_gradient_last_wave_split_on_a_ragged_edge():
+    """d_ff = 1200 at 16384 tokens: [dW_gate ; dW_up] is 2400 x 2048, 80 pair tiles, so its 74
+    whole tiles are stored directly and the last six (the ragged 96-row block among them, all in
+    dW_up) run as K splits summed per tile; every dW_up row from the split tiles and a sample of
+    the others are checked against the oracle over all tokens, and the split tiles' dW_gate
+    neighbours too."""
+    M, d, f = 16384, 2048, 1200
+    inp = synth.dense_inputs(M, d, f, seed=21, dtype=torch.bfloat16)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    y, h, a, b = api.swiglu_ffn_fwd(dev["x"], dev["w_gate"], dev["w_up"], dev["w_down"])
+    dx, dwg, dwu, dwd = api.swiglu_ffn_bwd(dev["dy"], dev["x"], dev["w_gate"], dev["w_up"], dev["w_down"], h, a, b)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    rng = np.random.default_rng(3)
+    cols = np.unique(np.concatenate([np.arange(848, 1200, 11), [848, 1199], rng.choice(848, 16, replace=False), [0]]))
+    x, wg, wu, wd, dy = (f64(inp[k]) for k in ("x", "w_gate", "w_up", "w_down", "dy"))
+    sub = O.dense_backward(x, wg[cols], wu[cols], wd[:, cols], dy)
+    assert_close("dw_gate[cols]", f64(dwg)[cols], sub["dw_gate"], torch.bfloat16)
+    assert_close("dw_up[cols]", f64(dwu)[cols], sub["dw_up"], torch.bfloat16)
+    assert_close("dw_down[:,cols]", f64(dwd)[:, cols], sub["dw_down"], torch.bfloat16)
+
+
 def test_workload4_inference_full_size_sampled():
     """The inference forward at 262144 tokens x 2048 x 5504, the launch configuration of the
     bench's inference line: sampled token rows against the oracle."""
