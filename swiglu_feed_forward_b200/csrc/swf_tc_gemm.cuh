@@ -395,6 +395,15 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
   using L = TcSmem<BN, PAIR, epi_smem_bytes<EPI, TMA_EPI, PAIR>()>;
   constexpr int S = L::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(PAIR ? 2 * kTileM : kTileM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+  // A pair tile whose N-block holds at most BN / 2 columns of the output (the last block of an N
+  // that is not a multiple of BN, e.g. d_ff = 5504 in 256-column blocks) is computed with N = BN / 2:
+  // each CTA stages BN / 4 of its columns (the odd CTA the second quarter, not the second half),
+  // and half the MMA work of an all-zero half is not spent.
+  constexpr bool kHalfTiles = PAIR && !B_DUAL && MODE == kModeDense && BN % 64 == 0;
+  constexpr uint32_t kIdescHalf = idesc_bf16(2 * kTileM, BN / 2, A_MN ? 1 : 0, B_MN ? 1 : 0);
+  auto half_tile = [&](const Tile& t_) {
+    return kHalfTiles && t_.nb == args.num_n_blk - 1 && args.N - t_.nb * BN <= BN / 2;
+  };
   constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators
   constexpr int kBRows = L::kBRows;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N");
@@ -510,7 +519,7 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
             load(sA, &tmA, ka, t.a_m);
           }
           const CUtensorMap* mapB = seg1 ? &tmB1 : &tmB0;
-          const int b_n = t.b_n + (PAIR && !B_DUAL ? (int)rank * kBRows : 0);
+          const int b_n = t.b_n + (PAIR && !B_DUAL ? (int)rank * (half_tile(t) ? kBRows / 2 : kBRows) : 0);
           if (B_DUAL) {
             if constexpr (PAIR) {
               load(sB, rank ? &tmB1 : &tmB0, t.b_k + kk, t.b_n);  // even CTA: gate rows, odd: up
@@ -566,6 +575,7 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
+        const uint32_t idesc = half_tile(t) ? kIdescHalf : kIdesc;
         for (int kb = 0; kb < t.kb; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl)) { ok = false; break; }
           // gathered rows were written by cp.async (generic proxy); the barrier made them
@@ -577,7 +587,7 @@ __global__ void __launch_bounds__(gemm_threads<GATHER>(), 1)
           for (int k = 0; k < kTileK / kUmmaK; ++k) {
             const uint64_t ad = a_desc0 + so + k * kAStep;
             const uint64_t bd = b_desc0 + so + k * kBStep;
-            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
             else umma_bf16(d_tmem, ad, bd, kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
           if constexpr (PAIR) umma_commit_pair(&empty[s], 3);
