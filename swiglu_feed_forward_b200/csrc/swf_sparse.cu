@@ -581,7 +581,7 @@ void sparse_plan(int op, int64_t M, int64_t d, int64_t f, int32_t G, int32_t K, 
       p->tile_n = 2 * G;
       break;
     case SWF_OP_SPARSE_BWD:
-      p->num_kernels = 5;  // dgate, dx, pair sum, dW_gate|dW_up, dW_down
+      p->num_kernels = 5;  // dgate, dW_down, dW_gate|dW_up, dx, pair sum
       p->flops = 12 * M * d * (int64_t)K * G;
       p->gemm_tiles = (int64_t)s.mblk * (1 + cdiv(d, 256)) + (int64_t)s.ng * (cdiv(d, 256) + cdiv(d, 128));
       break;
@@ -1000,6 +1000,22 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
                                                                                         st, em);
     if (s != SWF_OK) return s;
   }
+  // dW_down right after dgate: both gather the same dY rows, which are then still in L2
+  {  // per group: dW_d[:, g] = (dY rows of the segment)ᵀ h_seg, the dY rows gathered from dy
+    CUtensorMap th;
+    if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64)) return SWF_ERR_LAUNCH;
+    TcGemmArgs a = base_args(d, G, 64, 0);
+    a.n_groups = sd.ng;
+    a.seg_start = v.seg_start;
+    a.seg_rows = v.seg_rows;
+    a.kb_seg0 = 1 << 30;
+    a.group_size = G;
+    a.out0 = dw_down;
+    a.ld_out = f;
+    set_gather(a, v.row_token, dy, d);
+    s = launch_tc<64, true, true, false, kEpiGroupDWd, kModeKGrouped, false, kGatherA>(SWF_K_SPARSE_DW, th, th, th, a, st);
+  }
+  if (s != SWF_OK) return s;
   {  // per group: [dW_g[g] ; dW_u[g]] = dgu_segᵀ X rows of the segment (gathered from x)
     CUtensorMap tdgu;
     if (!encode_tmap_bf16(&tdgu, w.dgu, 128, sd.rmax, 128, 64, 64)) return SWF_ERR_LAUNCH;
@@ -1033,19 +1049,5 @@ extern "C" swf_status sparse_swiglu_ffn_bwd(const void* dy, const void* x, const
     if (s != SWF_OK) return s;
   }
   if ((s = run_pair_sum(w.dxc, v.pair_row, sd, dx, st)) != SWF_OK) return s;
-  {  // per group: dW_d[:, g] = (dY rows of the segment)ᵀ h_seg, the dY rows gathered from dy
-    CUtensorMap th;
-    if (!encode_tmap_bf16(&th, v.h, G, sd.rmax, G, 64, 64)) return SWF_ERR_LAUNCH;
-    TcGemmArgs a = base_args(d, G, 64, 0);
-    a.n_groups = sd.ng;
-    a.seg_start = v.seg_start;
-    a.seg_rows = v.seg_rows;
-    a.kb_seg0 = 1 << 30;
-    a.group_size = G;
-    a.out0 = dw_down;
-    a.ld_out = f;
-    set_gather(a, v.row_token, dy, d);
-    s = launch_tc<64, true, true, false, kEpiGroupDWd, kModeKGrouped, false, kGatherA>(SWF_K_SPARSE_DW, th, th, th, a, st);
-  }
   return s;
 }
