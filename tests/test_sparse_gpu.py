@@ -106,7 +106,8 @@ def test_minus_inf_bias_chosen_last(f, G):
     assert np.all(idx == np.array([g for g in range(ng) if g not in (5, 9)]))
 
 
-@pytest.mark.parametrize("M,K,ng", [(16384, 8, 64), (1000, 3, 7), (5000, 1, 300), (77, 20, 20)])
+# (20000, 2, 600): 600 groups over 209 blocks of 96 tokens
+@pytest.mark.parametrize("M,K,ng", [(16384, 8, 64), (1000, 3, 7), (5000, 1, 300), (77, 20, 20), (20000, 2, 600)])
 def test_buckets_bit_exact(M, K, ng):
     rng = np.random.default_rng(M + ng)
     idx = np.sort(np.stack([rng.choice(ng, size=K, replace=False) for _ in range(M)]), axis=1)
